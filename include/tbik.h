@@ -1,0 +1,238 @@
+/*
+ * tbik.h -- C ABI of the tree-ordered invariant kernels (TBIK-style) for NVIDIA
+ * B200 (sm_100a).
+ *
+ * What the library computes (sources are web pages, cited by title/section):
+ *  - "Deterministic Inference across Tensor Parallel Sizes That Eliminates
+ *    Training-Inference Mismatch" (paper summary page), sections 核心思路 and
+ *    技术框架 and the abstract: matrix multiplication and reduction primitives
+ *    whose local (per-GPU) and global (cross-GPU) reductions follow ONE
+ *    hierarchical binary tree, so results are bitwise identical for any
+ *    tensor-parallel (TP) size.
+ *  - Rounding-location alignment article (winzheng.jp), section
+ *    "外科手術的な修正：3つのノード": RoPE, SwiGLU and residual RMSNorm keep FP32
+ *    intermediates and round to BF16 once, at the output.
+ *  - IsoExec executive brief (nxmr.cn), sections 壹, 叁 and 伍: the per-token
+ *    logprob is the quantity that must agree bit for bit.
+ *
+ * The tree.  A reduction over L leaves uses TREE(P, lo, n): n == 1 gives P[lo];
+ * otherwise h = ceil(n/2) and the value is TREE(P,lo,h) + TREE(P,lo+h,n-h)
+ * (binary32 add, round to nearest even).  T shards of the reduced dimension
+ * are contiguous ranges of L/T leaves; for T in {1,2,4,8} with T | L each
+ * shard is one whole subtree, so the result does not depend on T.  On one GPU
+ * T is emulated: each shard's partial goes to its own fp32 buffer and the
+ * partials are combined with TREE over T.
+ *
+ * Conventions for every entry point:
+ *  - bf16 buffers are passed as raw 16-bit patterns (IEEE bfloat16).
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises on these paths (exceptions are
+ *    named: tbik_rope_table and tbik_get_error).  Pointers must be 16-byte
+ *    aligned (TBIK_ERR_ALIGN otherwise).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    All work is enqueued on it; results do not depend on the stream or on
+ *    other work running concurrently.
+ *  - Host-detected errors return a status immediately and enqueue nothing.
+ *    Device-detected errors (bad target or position, a bounded wait that
+ *    expired) are recorded in a per-device error word read by tbik_get_error.
+ *  - Functions are thread-safe; concurrent calls must not share a workspace.
+ */
+#ifndef TBIK_H
+#define TBIK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TBIK_API __attribute__((visibility("default")))
+#else
+#define TBIK_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TBIK_OK = 0,
+    TBIK_ERR_ARG = 1,         /* null pointer, negative size, unknown mode bit */
+    TBIK_ERR_SHAPE = 2,       /* K % leaf, T not in {1,2,4,8}, T does not divide the leaves ... */
+    TBIK_ERR_ALIGN = 3,       /* pointer or row stride not 16-byte aligned */
+    TBIK_ERR_WORKSPACE = 4,   /* workspace missing or smaller than the *_workspace() query */
+    TBIK_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed */
+    TBIK_ERR_TIMEOUT = 6,     /* a device-side bounded wait expired (kernel returned early) */
+    TBIK_ERR_TARGET = 7,      /* a logprob target outside [0, V) (its output is NaN) */
+    TBIK_ERR_POSITION = 8,    /* a RoPE position outside [0, max_pos) (its outputs are NaN) */
+    TBIK_ERR_UNSUPPORTED = 9  /* not a B200-class device (sm_100) */
+} tbik_status;
+
+/* ---- mode bits ---------------------------------------------------------- */
+/* Arithmetic of the leaf partials (exactly one of the two): */
+#define TBIK_EXACT 0x1u  /* CUDA cores: per output, per leaf, acc = fmaf(a, b, acc) in
+                            ascending k from +0.0f, then the tree.  Bit-exact to the
+                            definition. */
+#define TBIK_TC 0x2u     /* tcgen05 tensor cores: each leaf is one chain of 128x128x16
+                            bf16 MMAs accumulating in fp32 (TMEM) from zero; leaves are
+                            then combined by the same tree in fp32.  The leaf bits are
+                            fixed by the hardware and identical for every T and M. */
+/* Deliberately non-invariant baseline (with EXACT or TC): each shard
+   accumulates its whole K range in one chain and the shard partials are summed
+   left to right, ((Q0+Q1)+Q2)+...; logprob also combines leaves left to right. */
+#define TBIK_NONINV 0x4u
+/* Layout of B in tbik_gemm (row-major in both cases): */
+#define TBIK_B_KN 0x00u  /* B is [K,N] (N contiguous) */
+#define TBIK_B_NK 0x10u  /* B is [N,K] (K contiguous), e.g. an nn.Linear weight */
+/* Output type of tbik_gemm: */
+#define TBIK_OUT_F32 0x000u  /* C fp32 [M,N] */
+#define TBIK_OUT_BF16 0x100u /* C bf16 [M,N], rounded once (RNE) from the fp32 tree root */
+
+/* Vocabulary columns per logprob leaf, and the largest shard count the vocab
+   padding is sized for: V is padded to Vpad = ceil(V / (128*8)) * 128*8 with
+   identity leaves (max -inf, sum 0), independent of T. */
+#define TBIK_VOCAB_LEAF 128
+#define TBIK_T_MAX 8
+
+TBIK_API const char* tbik_version(void);
+TBIK_API const char* tbik_status_string(tbik_status s);
+
+/* ---- tree-ordered GEMM -------------------------------------------------- */
+
+/*
+ * Bytes of device workspace tbik_gemm needs for these arguments (0 is a valid
+ * answer: T = 1 at a size with enough output tiles writes C directly).
+ * Returns (size_t)-1 when the arguments would be rejected.
+ */
+TBIK_API size_t tbik_gemm_workspace(int M, int N, int K, int T, int leaf, unsigned mode);
+
+/*
+ * C = A * B with the K reduction in tree order (TBIK summary page, 技术框架:
+ * local reduction on each GPU, then a binary-tree reduction across GPUs;
+ * tutorial page section 2.1.1 / figure 5: T-way row-parallel split of K).
+ *
+ *   A  bf16 [M,K] row-major.          B  bf16 [K,N] or [N,K] (mode TBIK_B_*).
+ *   C  fp32 or bf16 [M,N] row-major (mode TBIK_OUT_*); may not alias A or B.
+ *   leaf  K elements per leaf; K % leaf == 0; L = K/leaf leaves.
+ *   T  emulated shard count in {1,2,4,8}; (K/leaf) % T == 0.  Shard t owns
+ *      leaves [t*L/T, (t+1)*L/T); its partial is written to its own fp32
+ *      buffer in the workspace and the T partials are combined by TREE.
+ *   TBIK_TC needs leaf % 16 == 0, N % 8 == 0 and K % 8 == 0 (16-byte TMA
+ *   strides); with TBIK_NONINV, (K/T) % 16 == 0 instead of the leaf rule.
+ *   ws/ws_bytes  device workspace of at least tbik_gemm_workspace() bytes,
+ *      256-byte aligned; may be NULL when that query returns 0.
+ * Row i of C depends only on row i of A: any batch size, split or order gives
+ * the same bits per row.  M == 0 is a no-op.
+ */
+TBIK_API tbik_status tbik_gemm(const uint16_t* A, const uint16_t* B, void* C, int M, int N, int K, int T,
+                      int leaf, unsigned mode, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- residual RMSNorm ---------------------------------------------------- */
+
+/*
+ * Residual RMSNorm with fp32 intermediates and one bf16 rounding
+ * (rounding-location article, 3つのノード: residual RMSNorm):
+ *   r = f32(x) + f32(res);  leaf j = elements [8j, 8j+8), P_j = fmaf(r,r,acc)
+ *   ascending from +0;  ss = TREE over the H/8 leaves (T shards of H/(8T)
+ *   leaves, shard partials combined by TREE);  ms = ss / H;
+ *   inv = 1 / sqrt(ms + eps) (correctly rounded ops);
+ *   y = bf16((r * inv) * gamma);  res_out = bf16(r).
+ * x, res, y, res_out: bf16 [tokens,H]; gamma bf16 [H]; res_out may be NULL;
+ * y may alias x.  H % 8 == 0 and H/8 a power of two in [32, 1024]
+ * (H in {256, 512, ..., 8192}); T in {1,2,4,8}.
+ */
+TBIK_API tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16_t* gamma,
+                                  uint16_t* y, uint16_t* res_out, int tokens, int H, float eps,
+                                  int T, void* stream);
+
+/* ---- RoPE + SwiGLU (fp32 intermediates, one rounding) -------------------- */
+
+/*
+ * Fills the DEVICE buffer `table` (fp32 [max_pos][head_dim/2][2], cos then
+ * sin) from binary64 arithmetic rounded once to fp32:
+ *   theta_i = base^(-2i/head_dim),  angle = pos * theta_i.
+ * The table is computed on the host and copied synchronously (set-up call,
+ * not for the hot path).  head_dim even, 2 <= head_dim <= 512.
+ */
+TBIK_API tbik_status tbik_rope_table(float* table, int max_pos, int head_dim, double base, void* stream);
+
+typedef struct {
+    /* RoPE group, rotate-half form (skipped when q and k are both NULL):
+       for i < head_dim/2:  o_i = x_i*c_i - x_{i+half}*s_i,
+                            o_{i+half} = x_{i+half}*c_i + x_i*s_i,
+       each product rounded separately (no fma), one bf16 rounding.
+       q/k bf16 [tokens][heads][head_dim]; outputs may alias inputs; either of
+       q or k may be NULL.  head_dim % 16 == 0, head_dim <= 512. */
+    const uint16_t* q;
+    const uint16_t* k;
+    uint16_t* q_out;
+    uint16_t* k_out;
+    const int32_t* pos;  /* [tokens], each in [0, max_pos) */
+    const float* table;  /* from tbik_rope_table */
+    int tokens;
+    int heads;
+    int head_dim;
+    int max_pos;
+    /* SwiGLU group (skipped when g is NULL): out = bf16((g / (1 + exp(-g))) * u)
+       in fp32 with the library's exp specification (Cody-Waite reduction by a
+       split ln 2, degree-7 Taylor polynomial, correctly rounded scaling).
+       g/u bf16 or fp32 (in_f32 = 1) [n]; out bf16 [n]; n % 8 == 0. */
+    const void* g;
+    const void* u;
+    uint16_t* out;
+    long long n;
+    int in_f32;
+} tbik_rope_swiglu_args;
+
+TBIK_API tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* args, void* stream);
+
+/* ---- fused lm_head -> log-softmax -> target logprob ---------------------- */
+
+TBIK_API size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, unsigned mode);
+
+/*
+ * out[i] = log softmax(hidden[i] . W_lm^T)[targets[i]] (IsoExec brief 壹/叁:
+ * the logprob is the compared quantity; TBIK page: tree-ordered reductions),
+ * without materialising the logits (TBIK_TC):
+ *   z[i,v]  = tree-ordered dot product over H (leaves of `leaf`, TREE over
+ *             all H/leaf leaves), kept fp32;
+ *   vocab leaf j = columns [128j, 128j+128) cut at V: m_j = max in ascending
+ *             column order, s_j = sum in ascending order of exp(z - m_j);
+ *   (m,s) combine: m = max(ma,mb); s = sa*exp(ma-m) + sb*exp(mb-m) (products
+ *             rounded separately); identity (-inf, 0);
+ *   shard t (of T) owns the vocab leaves [t*Lv/T, (t+1)*Lv/T) of the padded
+ *             Lv = Vpad/128; shard summaries and then the T shards combine by TREE;
+ *   out[i]  = (z[i,target] - m) - log(s)  (library log specification).
+ * hidden bf16 [M,H]; W_lm bf16 [V,H] row-major; targets int32 [M]; out fp32 [M].
+ * H % leaf == 0, leaf % 16 == 0, H % 8 == 0, T in {1,2,4,8}.  A target outside
+ * [0,V) gives NaN and records TBIK_ERR_TARGET.  TBIK_EXACT materialises the
+ * fp32 logits in the workspace (CUDA-core reference mode).
+ */
+TBIK_API tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W_lm, const int32_t* targets,
+                         float* out, int M, int V, int H, int T, int leaf, unsigned mode, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* ---- errors -------------------------------------------------------------- */
+
+/*
+ * Synchronises `stream`, then returns and clears the error word of the
+ * current device (TBIK_OK when no device-side error was recorded).  Returns
+ * TBIK_ERR_CUDA if the synchronisation itself reports an error.
+ */
+TBIK_API tbik_status tbik_get_error(void* stream);
+
+/*
+ * Test hooks.  flags: TBIK_DEBUG_WITHHOLD_ACC_ARRIVE makes the tensor-core GEMM
+ * epilogue withhold its "accumulator drained" arrive, so the MMA issuer's
+ * bounded wait expires: the kernel must record TBIK_ERR_TIMEOUT, drain its own
+ * copies in flight, free its TMEM and return.  wait_limit_ns bounds every
+ * device-side wait (0 keeps the default of 2 s).  TBIK_DEBUG_SWAP_MN_STRIDES
+ * swaps the two stride fields of the [K,N] B operand descriptor (layout check).
+ */
+#define TBIK_DEBUG_WITHHOLD_ACC_ARRIVE 0x1u
+#define TBIK_DEBUG_SWAP_MN_STRIDES 0x2u
+TBIK_API tbik_status tbik_debug_set(unsigned flags, unsigned long long wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TBIK_H */

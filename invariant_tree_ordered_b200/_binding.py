@@ -1,0 +1,264 @@
+"""ctypes binding of ``libtbik.so`` (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only turns torch tensors into device pointers and sizes, allocates workspaces
+with torch (the library itself never allocates), and raises on a non-zero
+status.  There is no fallback: if the library cannot be loaded, importing the
+functions raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtbik.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "tbik.h")
+
+TBIK_OK = 0
+TBIK_ERR_ARG = 1
+TBIK_ERR_SHAPE = 2
+TBIK_ERR_ALIGN = 3
+TBIK_ERR_WORKSPACE = 4
+TBIK_ERR_CUDA = 5
+TBIK_ERR_TIMEOUT = 6
+TBIK_ERR_TARGET = 7
+TBIK_ERR_POSITION = 8
+TBIK_ERR_UNSUPPORTED = 9
+
+EXACT = 0x1
+TC = 0x2
+NONINV = 0x4
+B_KN = 0x00
+B_NK = 0x10
+OUT_F32 = 0x000
+OUT_BF16 = 0x100
+DEBUG_WITHHOLD_ACC_ARRIVE = 0x1
+DEBUG_SWAP_MN_STRIDES = 0x2
+VOCAB_LEAF = 128
+T_MAX = 8
+
+_lock = threading.Lock()
+_lib = None
+
+
+class TbikError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: tbik status {status} ({status_string(status)})")
+
+
+class RopeSwigluArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("q_out", ctypes.c_void_p), ("k_out", ctypes.c_void_p),
+        ("pos", ctypes.c_void_p), ("table", ctypes.c_void_p),
+        ("tokens", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("max_pos", ctypes.c_int),
+        ("g", ctypes.c_void_p), ("u", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("n", ctypes.c_longlong), ("in_f32", ctypes.c_int),
+    ]
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load ``libtbik.so`` (raises OSError if it is missing: build it first)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path == LIB_PATH:
+            return _lib
+        if not os.path.exists(path):
+            raise OSError(f"{path} not found: run `python -m invariant_tree_ordered_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, i32, u32, sz, f32, f64, ull = (ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_size_t,
+                                            ctypes.c_float, ctypes.c_double, ctypes.c_ulonglong)
+        sigs = {
+            "tbik_version": (ctypes.c_char_p, []),
+            "tbik_status_string": (ctypes.c_char_p, [i32]),
+            "tbik_gemm_workspace": (sz, [i32, i32, i32, i32, i32, u32]),
+            "tbik_gemm": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
+            "tbik_rmsnorm_residual": (i32, [vp, vp, vp, vp, vp, i32, i32, f32, i32, vp]),
+            "tbik_rope_table": (i32, [vp, i32, i32, f64, vp]),
+            "tbik_rope_swiglu_fp32": (i32, [ctypes.POINTER(RopeSwigluArgs), vp]),
+            "tbik_logprob_workspace": (sz, [i32, i32, i32, i32, i32, u32]),
+            "tbik_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
+            "tbik_get_error": (i32, [vp]),
+            "tbik_debug_set": (i32, [u32, ull]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        if path == LIB_PATH:
+            _lib = lib
+        return lib
+
+
+def declared_functions(header: str = HEADER):
+    """Names of the functions ``include/tbik.h`` declares."""
+    with open(header) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tbik_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    try:
+        return load_library().tbik_status_string(status).decode()
+    except OSError:
+        return "library not loaded"
+
+
+def _check(status: int, what: str):
+    if status != TBIK_OK:
+        raise TbikError(status, what)
+
+
+# ------------------------------------------------------------ torch plumbing
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(nbytes: int, device, workspace):
+    torch = _torch()
+    if nbytes == (1 << 64) - 1 or nbytes < 0:
+        raise TbikError(TBIK_ERR_SHAPE, "workspace query")
+    if nbytes == 0:
+        return workspace, 0
+    if workspace is not None:
+        return workspace, workspace.numel() * workspace.element_size()
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, nbytes
+
+
+# ---------------------------------------------------------------- entry points
+
+def gemm_workspace(M, N, K, T, leaf, mode) -> int:
+    return int(load_library().tbik_gemm_workspace(M, N, K, T, leaf, mode))
+
+
+def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = False, b_nk: bool = False,
+         out_bf16: bool = False, out=None, workspace=None, stream=None):
+    """C = A @ B with the K reduction in tree order (see tbik_gemm in tbik.h)."""
+    torch = _torch()
+    lib = load_library()
+    _need(A, torch.bfloat16, "A")
+    _need(B, torch.bfloat16, "B")
+    M, K = A.shape
+    N = B.shape[0] if b_nk else B.shape[1]
+    kb = B.shape[1] if b_nk else B.shape[0]
+    if kb != K:
+        raise ValueError("inner dimensions differ")
+    mode = (TC if tc else EXACT) | (NONINV if noninv else 0) | (B_NK if b_nk else B_KN) | (OUT_BF16 if out_bf16 else OUT_F32)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16 if out_bf16 else torch.float32, device=A.device)
+    ws, wsb = _workspace(lib.tbik_gemm_workspace(M, N, K, T, leaf, mode), A.device, workspace)
+    _check(lib.tbik_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, T, leaf, mode, _ptr(ws), wsb,
+                         _stream_handle(stream)), "tbik_gemm")
+    return out
+
+
+def rmsnorm_residual(x, res, gamma, *, eps: float = 1e-6, T: int = 1, y=None, res_out=None, want_res_out=True,
+                     stream=None):
+    torch = _torch()
+    lib = load_library()
+    for t, n in ((x, "x"), (res, "res"), (gamma, "gamma")):
+        _need(t, torch.bfloat16, n)
+    tokens, H = x.shape
+    if y is None:
+        y = torch.empty_like(x)
+    if res_out is None and want_res_out:
+        res_out = torch.empty_like(x)
+    _check(lib.tbik_rmsnorm_residual(_ptr(x), _ptr(res), _ptr(gamma), _ptr(y), _ptr(res_out), tokens, H,
+                                     float(eps), T, _stream_handle(stream)), "tbik_rmsnorm_residual")
+    return y, res_out
+
+
+def rope_table(max_pos: int, head_dim: int = 128, base: float = 1e6, device="cuda", stream=None):
+    torch = _torch()
+    lib = load_library()
+    t = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+    _check(lib.tbik_rope_table(_ptr(t), max_pos, head_dim, float(base), _stream_handle(stream)), "tbik_rope_table")
+    return t
+
+
+def rope_swiglu(*, q=None, k=None, pos=None, table=None, q_out=None, k_out=None, g=None, u=None, out=None,
+                stream=None):
+    """RoPE on q/k and/or SwiGLU on g/u in one call (see tbik_rope_swiglu_fp32)."""
+    torch = _torch()
+    lib = load_library()
+    a = RopeSwigluArgs()
+    if q is not None or k is not None:
+        ref = q if q is not None else k
+        _need(ref, torch.bfloat16, "q/k")
+        _need(pos, torch.int32, "pos")
+        _need(table, torch.float32, "table")
+        tokens, heads, hd = ref.shape
+        if q is not None and q_out is None:
+            q_out = torch.empty_like(q)
+        if k is not None and k_out is None:
+            k_out = torch.empty_like(k)
+        a.q, a.k, a.q_out, a.k_out = _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out)
+        a.pos, a.table = _ptr(pos), _ptr(table)
+        a.tokens, a.heads, a.head_dim, a.max_pos = tokens, heads, hd, table.shape[0]
+    if g is not None:
+        if g.dtype not in (torch.bfloat16, torch.float32) or u.dtype != g.dtype:
+            raise TypeError("g and u must both be bf16 or both fp32")
+        _need(g, g.dtype, "g")
+        _need(u, g.dtype, "u")
+        if out is None:
+            out = torch.empty(g.shape, dtype=torch.bfloat16, device=g.device)
+        a.g, a.u, a.out, a.n, a.in_f32 = _ptr(g), _ptr(u), _ptr(out), g.numel(), int(g.dtype == torch.float32)
+    _check(lib.tbik_rope_swiglu_fp32(ctypes.byref(a), _stream_handle(stream)), "tbik_rope_swiglu_fp32")
+    return q_out, k_out, out
+
+
+def logprob_workspace(M, V, H, T, leaf, mode) -> int:
+    return int(load_library().tbik_logprob_workspace(M, V, H, T, leaf, mode))
+
+
+def logprob(hidden, W, targets, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = False, out=None,
+            workspace=None, stream=None):
+    torch = _torch()
+    lib = load_library()
+    _need(hidden, torch.bfloat16, "hidden")
+    _need(W, torch.bfloat16, "W_lm")
+    _need(targets, torch.int32, "targets")
+    M, H = hidden.shape
+    V = W.shape[0]
+    mode = (TC if tc else EXACT) | (NONINV if noninv else 0)
+    if out is None:
+        out = torch.empty(M, dtype=torch.float32, device=hidden.device)
+    ws, wsb = _workspace(lib.tbik_logprob_workspace(M, V, H, T, leaf, mode), hidden.device, workspace)
+    _check(lib.tbik_logprob(_ptr(hidden), _ptr(W), _ptr(targets), _ptr(out), M, V, H, T, leaf, mode, _ptr(ws), wsb,
+                            _stream_handle(stream)), "tbik_logprob")
+    return out
+
+
+def get_error(stream=None) -> int:
+    return int(load_library().tbik_get_error(_stream_handle(stream)))
+
+
+def debug_set(flags: int = 0, wait_limit_ns: int = 0):
+    _check(load_library().tbik_debug_set(flags, wait_limit_ns), "tbik_debug_set")

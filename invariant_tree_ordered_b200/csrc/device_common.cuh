@@ -1,0 +1,354 @@
+// Device-side helpers shared by the library's kernels: bf16 conversion, the
+// error word, bounded waits, the tree walk and thin inline-PTX wrappers for
+// mbarrier, TMA (cp.async.bulk.tensor) and tcgen05 (sm_100a), written from the
+// PTX ISA description of those instructions.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tbik.h"
+
+namespace tbik {
+
+// ------------------------------------------------------------------ errors
+
+// Per-device error word: the first device-detected error wins.
+__device__ unsigned int g_err;
+
+__device__ __forceinline__ void set_error(unsigned code) { atomicCAS(&g_err, 0u, code); }
+
+// ------------------------------------------------------------------ bf16
+
+__device__ __forceinline__ float bf2f(uint16_t h) { return __uint_as_float(((uint32_t)h) << 16); }
+
+// fp32 -> bf16 bits, round to nearest even (NaN stays NaN).
+__device__ __forceinline__ uint16_t f2bf(float f) {
+    __nv_bfloat16 b = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t*>(&b);
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
+}
+
+// ----------------------------------------------------- exp / log specs
+// Cody-Waite style specifications (W. J. Cody and W. Waite, "Software Manual
+// for the Elementary Functions", 1980): additive reduction by a split ln 2 and
+// a short polynomial.  Every operation is an explicit round-to-nearest
+// intrinsic so the compiler cannot contract or reorder it.
+
+__device__ __forceinline__ float pow2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
+
+// e^x: clamp to [-104, 89]; k = rint(x*log2e); r = (x - k*ln2hi) - k*ln2lo;
+// degree-7 Taylor polynomial of e^r (coefficients: nearest floats to 1/n!);
+// scale by 2^(k/2) exactly, then by 2^(k-k/2) (one rounding).
+__device__ __forceinline__ float exp_spec(float x) {
+    if (x != x) return __fadd_rn(x, x);
+    x = fminf(fmaxf(x, -104.0f), 89.0f);
+    const float log2e = 0x1.715476p+0f, ln2hi = 0x1.62e4p-1f, ln2lo = 0x1.7f7d1cp-20f;
+    float kf = rintf(__fmul_rn(x, log2e));
+    float r = __fmaf_rn(-kf, ln2hi, x);
+    r = __fmaf_rn(-kf, ln2lo, r);
+    float p = 0x1.a01a02p-13f;
+    p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+    p = __fmaf_rn(p, r, 0x1.111112p-7f);
+    p = __fmaf_rn(p, r, 0x1.555556p-5f);
+    p = __fmaf_rn(p, r, 0x1.555556p-3f);
+    p = __fmaf_rn(p, r, 0.5f);
+    p = __fmaf_rn(p, r, 1.0f);
+    p = __fmaf_rn(p, r, 1.0f);
+    int k = (int)kf;
+    int k1 = k / 2;
+    int k2 = k - k1;
+    return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));
+}
+
+// log x for x > 0: x = 2^e * m, m in [sqrt(1/2), sqrt 2]; t = f/(2+f), f = m-1;
+// log m = s + s*w*(1/3 + w/5 + w^2/7 + w^3/9 + w^4/11), s = 2t, w = t^2;
+// result = e*ln2hi + (e*ln2lo + log m).
+__device__ __forceinline__ float log_spec(float x) {
+    if (x != x) return __fadd_rn(x, x);
+    if (x < 0.0f) return __int_as_float(0x7fc00000);
+    if (x == 0.0f) return -INFINITY;
+    if (x == INFINITY) return x;
+    int e = 0;
+    uint32_t u = __float_as_uint(x);
+    if (u < 0x00800000u) {
+        x = __fmul_rn(x, 0x1p23f);
+        u = __float_as_uint(x);
+        e = -23;
+    }
+    e += (int)(u >> 23) - 127;
+    float m = __uint_as_float((u & 0x007fffffu) | 0x3f800000u);
+    if (m > 0x1.6a09e6p+0f) {
+        m = __fmul_rn(m, 0.5f);
+        e += 1;
+    }
+    float f = __fsub_rn(m, 1.0f);
+    float t = __fdiv_rn(f, __fadd_rn(2.0f, f));
+    float w = __fmul_rn(t, t);
+    float q = 0x1.745d18p-4f;
+    q = __fmaf_rn(q, w, 0x1.c71c72p-4f);
+    q = __fmaf_rn(q, w, 0x1.24924ap-3f);
+    q = __fmaf_rn(q, w, 0x1.99999ap-3f);
+    q = __fmaf_rn(q, w, 0x1.555556p-2f);
+    float s = __fadd_rn(t, t);
+    float lm = __fmaf_rn(__fmul_rn(s, w), q, s);
+    float ef = (float)e;
+    float r = __fmaf_rn(ef, 0x1.7f7d1cp-20f, lm);
+    return __fmaf_rn(ef, 0x1.62e4p-1f, r);
+}
+
+// (max, sum-exp) summary and its combine (identity: -inf, 0).  `a` is the left
+// operand of the tree; the larger-of rule keeps `a` on ties.
+struct MS {
+    float m, s;
+};
+
+__device__ __forceinline__ MS ms_combine(MS a, MS b) {
+    MS r;
+    r.m = (b.m > a.m) ? b.m : a.m;
+    if (r.m == -INFINITY) {
+        r.s = 0.0f;
+        return r;
+    }
+    float ea = exp_spec(__fsub_rn(a.m, r.m));
+    float eb = exp_spec(__fsub_rn(b.m, r.m));
+    r.s = __fadd_rn(__fmul_rn(a.s, ea), __fmul_rn(b.s, eb));
+    return r;
+}
+
+// ------------------------------------------------------------- tree walk
+
+// Streaming (post-order) evaluation of TREE over n leaves: after leaf j arrives,
+// the nodes whose last leaf is j close, deepest first; each close adds the
+// pending result of that node's left child (size pop_size[i]).  The shallowest
+// closed node (or the leaf itself) is then pushed, unless it is the root.
+struct LeafOps {
+    int npop;
+    int pop_size[24];
+    int push_size;
+    bool final_;
+};
+
+__device__ __forceinline__ void leaf_ops(int n, int j, LeafOps& o) {
+    int lo = 0, sz = n, depth = 0;
+    int plo[24], psz[24], ph[24];
+    while (sz > 1) {
+        int h = (sz + 1) >> 1;
+        plo[depth] = lo;
+        psz[depth] = sz;
+        ph[depth] = h;
+        ++depth;
+        if (j < lo + h) {
+            sz = h;
+        } else {
+            lo += h;
+            sz -= h;
+        }
+    }
+    o.npop = 0;
+    int top = 1;
+    for (int d = depth - 1; d >= 0; --d) {
+        if (plo[d] + psz[d] - 1 != j) break;
+        o.pop_size[o.npop++] = ph[d];
+        top = psz[d];
+    }
+    o.push_size = top;
+    o.final_ = (top == n);
+}
+
+// ------------------------------------------------------------ PTX: misc
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------- PTX: mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on one phase of an mbarrier.  Gives up (returns false) when the
+// CTA-wide abort flag is raised by another role, or after limit_ns, in which
+// case it records TBIK_ERR_TIMEOUT and raises the abort flag itself.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer();
+    while (true) {
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > limit_ns) {
+            *abort_flag = 1;
+            set_error(TBIK_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Bounded wait used on the way out: no abort check, only the time limit.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > limit_ns) {
+            set_error(TBIK_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// --------------------------------------------------------------- PTX: TMA
+
+__device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// 2-D tiled bulk tensor load global -> shared, completion counted in bytes on `bar`.
+// x is the innermost coordinate (elements); it must be a multiple of 8 for bf16.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ------------------------------------------------------------ PTX: tcgen05
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 inputs, fp32 accumulate).
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 op issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp receives
+// row (lane base + t), columns [col, col+32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for tcgen05.mma (PTX ISA, "Shared memory
+// descriptor"): start address >> 4 in bits [0,14), leading byte offset >> 4 in
+// [16,30), stride byte offset >> 4 in [32,46), fixed 0b001 in [46,49), base
+// offset 0, swizzle mode in [61,64) (2 = 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f16 (PTX ISA, "Instruction descriptor"):
+// D format f32 (bits 4-5 = 1), A and B bf16 (bits 7-9 = 1, 10-12 = 1),
+// A/B major in bits 15/16 (0 = K-major, 1 = MN-major), N>>3 in bits 17-22,
+// M>>4 in bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+}  // namespace tbik

@@ -1,0 +1,366 @@
+// Tensor-core (tcgen05 + TMEM + TMA) tree-ordered GEMM for sm_100a.
+//
+// Source of the arithmetic: "Deterministic Inference across Tensor Parallel
+// Sizes That Eliminates Training-Inference Mismatch" (TBIK summary page),
+// sections 核心思路 / 技术框架: the K reduction is one hierarchical binary
+// tree shared by the local and the cross-GPU steps.  Here each K leaf is a
+// chain of 128x128x16 bf16 MMAs into an fp32 TMEM accumulator that restarts
+// from zero; the leaves are then combined by the halving tree in fp32 in the
+// epilogue.  The MMA sequence of a leaf depends only on the leaf's K range,
+// never on M, N or T, so a row's bits are the same for every batch size and
+// every shard count.
+//
+// CTA layout (192 threads, one CTA per SM, persistent over work units):
+//   warp 0     TMA producer: A and B k-blocks (64 deep) into a 6-stage ring
+//   warp 1     TMEM allocator + single-thread MMA issuer
+//   warps 2-5  epilogue: drain each leaf from TMEM and apply the tree
+// TMEM (512 columns x 128 lanes, fp32): columns [0,256) hold two leaf
+// accumulators (double buffer); [256,512) hold two pending subtree results of
+// size <= 2 leaves.  Pending subtrees of >= 3 leaves (written once per 3+
+// leaves) go to a per-CTA fp32 scratch in global memory that stays in L2.
+// A work unit is (m tile, n tile, frontier node f): the node's subtree of
+// leaves is reduced by this CTA; with more than one frontier node per tile the
+// subtree results go to fp32 partial buffers that a combine kernel reduces
+// with the upper levels of the same tree.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace tbik {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 128;
+constexpr int TC_BK = 64;
+constexpr int TC_STAGES = 6;
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
+constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;
+constexpr int TC_THREADS = 192;
+constexpr int TC_TMEM_COLS = 512;
+constexpr int TC_MAX_F = 64;
+constexpr int TC_SLOT_FLOATS = TC_BM * TC_BN;
+constexpr size_t TC_SMEM_BYTES = (size_t)TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+
+enum { EPI_TREE = 0, EPI_LOGPROB = 1 };
+
+struct TcParams {
+    int M, N, K;
+    int leaf;         // K elements per leaf (multiple of 16)
+    int F;            // frontier nodes per output tile
+    int tiles_m, tiles_n, group_m;
+    int total_units;
+    int direct;       // 1: write final C; 0: write partials[f]
+    int out_bf16;
+    void* out;        // C [M,N]
+    float* partials;  // [F][M][N]
+    float* scratch;   // [gridDim.x][gs][128*128], layout per slot [col/4][row][4]
+    int gs;           // global stack slots per CTA
+    int b_mn;         // 1: B is [K,N] (MN-major operand)
+    uint32_t b_lbo, b_sbo;
+    // logprob epilogue
+    const int32_t* targets;
+    float* stats;  // [tiles_n][M][2]  (max, sum-exp) per row and vocab leaf
+    float* zt;     // [M]  logit of the target
+    int V;
+    unsigned debug;
+    unsigned long long wait_ns;
+    short lo[TC_MAX_F];
+    short nl[TC_MAX_F];
+};
+
+__device__ __forceinline__ void tc_decode(const TcParams& p, int u, int& tm, int& tn, int& f) {
+    int tiles = p.tiles_m * p.tiles_n;
+    f = u / tiles;
+    int t = u - f * tiles;
+    int group_size = p.group_m * p.tiles_n;
+    int g = t / group_size;
+    int first_m = g * p.group_m;
+    int gm = min(p.tiles_m - first_m, p.group_m);
+    int r = t - g * group_size;
+    tm = first_m + r % gm;
+    tn = r / gm;
+}
+
+__device__ __forceinline__ float* scratch_slot(const TcParams& p, int slot) {
+    return p.scratch + ((size_t)blockIdx.x * p.gs + slot) * TC_SLOT_FLOATS;
+}
+
+// 32 columns (chunk c) of one row of a scratch slot; coalesced across the warp.
+__device__ __forceinline__ void scratch_ld(const float* base, int c, int row, float (&w)[32]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float4 x = *reinterpret_cast<const float4*>(base + ((size_t)(c * 8 + q) * TC_BM + row) * 4);
+        w[4 * q + 0] = x.x;
+        w[4 * q + 1] = x.y;
+        w[4 * q + 2] = x.z;
+        w[4 * q + 3] = x.w;
+    }
+}
+__device__ __forceinline__ void scratch_st(float* base, int c, int row, const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(base + ((size_t)(c * 8 + q) * TC_BM + row) * 4) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// Row `row` (global), columns [col0, col0+32) of the output; N % 8 == 0.
+__device__ __forceinline__ void store_row32(void* out, int out_bf16, int M, int N, int row, int col0,
+                                            const float (&v)[32]) {
+    if (row >= M) return;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        int col = col0 + 8 * q;
+        if (col >= N) break;
+        size_t off = (size_t)row * N + col;
+        if (out_bf16) {
+            uint4 w;
+            w.x = pack_bf2(v[8 * q + 0], v[8 * q + 1]);
+            w.y = pack_bf2(v[8 * q + 2], v[8 * q + 3]);
+            w.z = pack_bf2(v[8 * q + 4], v[8 * q + 5]);
+            w.w = pack_bf2(v[8 * q + 6], v[8 * q + 7]);
+            *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + off) = w;
+        } else {
+            float* o = reinterpret_cast<float*>(out) + off;
+            *reinterpret_cast<float4*>(o) = make_float4(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3]);
+            *reinterpret_cast<float4*>(o + 4) = make_float4(v[8 * q + 4], v[8 * q + 5], v[8 * q + 6], v[8 * q + 7]);
+        }
+    }
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * TC_B_BYTES);
+    uint64_t* full = bars;                     // [STAGES] TMA landed
+    uint64_t* empty = bars + TC_STAGES;        // [STAGES] MMAs done reading
+    uint64_t* acc_full = bars + 2 * TC_STAGES; // [2] leaf accumulator ready
+    uint64_t* acc_empty = acc_full + 2;        // [2] leaf accumulator drained
+    uint64_t* done = acc_empty + 2;            // all MMAs retired
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint64_t wait_ns = p.wait_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 128);
+        }
+        mbar_init(done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            uint32_t q = 0;
+            for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+                int tm, tn, f;
+                tc_decode(p, u, tm, tn, f);
+                const int k0 = p.lo[f] * p.leaf;
+                const int nkb = (p.nl[f] * p.leaf + TC_BK - 1) / TC_BK;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int s = q % TC_STAGES;
+                    if (!mbar_wait(&empty[s], ((q / TC_STAGES) & 1) ^ 1, abort_flag, wait_ns)) goto producer_out;
+                    mbar_arrive_expect_tx(&full[s], TC_A_BYTES + TC_B_BYTES);
+                    const int kx = k0 + kb * TC_BK;
+                    tma_load_2d(sA + s * TC_A_BYTES, &tmA, &full[s], kx, tm * TC_BM);
+                    if (!p.b_mn) {
+                        tma_load_2d(sB + s * TC_B_BYTES, &tmB, &full[s], kx, tn * TC_BN);
+                    } else {
+                        tma_load_2d(sB + s * TC_B_BYTES, &tmB, &full[s], tn * TC_BN, kx);
+                        tma_load_2d(sB + s * TC_B_BYTES + TC_B_BYTES / 2, &tmB, &full[s], tn * TC_BN + 64, kx);
+                    }
+                    ++q;
+                }
+            }
+        producer_out:
+            // Let the copies this thread issued land before the CTA can exit.
+            for (uint32_t i = (q > (uint32_t)TC_STAGES ? q - TC_STAGES : 0u); i < q; ++i)
+                mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_ns);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN, 0, p.b_mn);
+            uint32_t q = 0, a = 0;
+            for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+                int tm, tn, f;
+                tc_decode(p, u, tm, tn, f);
+                const int nsteps = p.nl[f] * p.leaf / 16;
+                const int spl = p.leaf / 16;
+                uint32_t buf = 0;
+                int in_leaf = 0;
+                for (int st = 0; st < nsteps; ++st) {
+                    const int ks = st & 3;
+                    if (in_leaf == 0) {
+                        buf = a & 1;
+                        if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_ns)) goto mma_out;
+                        tc_fence_after();
+                    }
+                    const int s = q % TC_STAGES;
+                    if (ks == 0) {
+                        if (!mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_ns)) goto mma_out;
+                        tc_fence_after();
+                    }
+                    const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * TC_A_BYTES) + ks * 32, 16, 1024);
+                    uint64_t bdesc;
+                    if (!p.b_mn)
+                        bdesc = smem_desc_sw128(smem_u32(sB + s * TC_B_BYTES) + ks * 32, 16, 1024);
+                    else
+                        bdesc = smem_desc_sw128(smem_u32(sB + s * TC_B_BYTES) + ks * 2048, p.b_lbo, p.b_sbo);
+                    tc_mma(tmem_base + buf * TC_BN, adesc, bdesc, idesc, in_leaf != 0 ? 1u : 0u);
+                    if (ks == 3 || st == nsteps - 1) {
+                        tc_commit(&empty[s]);
+                        ++q;
+                    }
+                    if (++in_leaf == spl) {
+                        tc_commit(&acc_full[buf]);
+                        ++a;
+                        in_leaf = 0;
+                    }
+                }
+            }
+        mma_out:
+            // Every MMA issued by this thread retires before TMEM is released.
+            tc_commit(done);
+            mbar_drain(done, 0, wait_ns);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int ew = warp & 3;
+        const int rt = ew * 32 + lane;  // row within the tile
+        const uint32_t tl = tmem_base + ((uint32_t)(ew * 32) << 16);
+        uint32_t a = 0;
+        for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+            int tm, tn, f;
+            tc_decode(p, u, tm, tn, f);
+            const int n = p.nl[f];
+            const int row = tm * TC_BM + rt;
+            int tsp = 0, gsp = 0;
+            for (int j = 0; j < n; ++j) {
+                const uint32_t buf = a & 1;
+                if (!mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_ns)) goto epi_out;
+                tc_fence_after();
+                __syncwarp();
+                LeafOps ops;
+                leaf_ops(n, j, ops);
+                int pop_slot[24];
+                int t2 = tsp, g2 = gsp;
+                for (int i = 0; i < ops.npop; ++i) pop_slot[i] = (ops.pop_size[i] <= 2) ? --t2 : -(--g2) - 1;
+                const bool push_small = ops.push_size <= 2;
+                int push_slot = 0;
+                if (!ops.final_) push_slot = push_small ? t2++ : g2++;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tl + buf * TC_BN + c * 32, v);
+                    for (int i = 0; i < ops.npop; ++i) {
+                        float w[32];
+                        if (pop_slot[i] >= 0)
+                            tmem_ld32(tl + 256 + pop_slot[i] * TC_BN + c * 32, w);
+                        else
+                            scratch_ld(scratch_slot(p, -pop_slot[i] - 1), c, rt, w);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(w[k], v[k]);
+                    }
+                    if (ops.final_) {
+                        if (EPI == EPI_TREE) {
+                            if (p.direct)
+                                store_row32(p.out, p.out_bf16, p.M, p.N, row, tn * TC_BN + c * 32, v);
+                            else
+                                store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row,
+                                            tn * TC_BN + c * 32, v);
+                        } else {
+                            tmem_st32(tl + 256 + c * 32, v);  // stage the logits in slot 0
+                        }
+                    } else if (push_small) {
+                        tmem_st32(tl + 256 + push_slot * TC_BN + c * 32, v);
+                    } else {
+                        scratch_st(scratch_slot(p, push_slot), c, rt, v);
+                    }
+                    __syncwarp();
+                }
+                tsp = t2;
+                gsp = g2;
+                tc_fence_before();
+                if (!(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) mbar_arrive(&acc_empty[buf]);
+                ++a;
+            }
+            if (EPI == EPI_LOGPROB) {
+                // Vocab leaf = this tile's 128 columns: running max in ascending
+                // column order, then the ascending sum of exp(z - max).
+                const int n0 = tn * TC_BN;
+                const int tgt = (row < p.M) ? p.targets[row] : -1;
+                float m = 0.0f, zval = 0.0f;
+                bool have_t = false;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tl + 256 + c * 32, v);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int col = n0 + c * 32 + k;
+                        if (col < p.V) {
+                            if (c == 0 && k == 0)
+                                m = v[k];
+                            else if (v[k] > m)
+                                m = v[k];
+                            if (col == tgt) {
+                                zval = v[k];
+                                have_t = true;
+                            }
+                        }
+                    }
+                }
+                float s = 0.0f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float v[32];
+                    tmem_ld32(tl + 256 + c * 32, v);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int col = n0 + c * 32 + k;
+                        if (col < p.V) s = __fadd_rn(s, exp_spec(__fsub_rn(v[k], m)));
+                    }
+                }
+                if (row < p.M) {
+                    *reinterpret_cast<float2*>(p.stats + ((size_t)tn * p.M + row) * 2) = make_float2(m, s);
+                    if (have_t) p.zt[row] = zval;
+                }
+                __syncwarp();
+            }
+        }
+    epi_out:;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TC_TMEM_COLS);
+    }
+}
+
+}  // namespace tbik

@@ -1,0 +1,160 @@
+// Log-softmax over the vocabulary and gather of the target logprob, with the
+// vocabulary reduction in tree order (TBIK summary page, 技术框架) and the
+// per-token logprob as the compared quantity (IsoExec brief, 壹/叁).
+//
+//  * vocab_stats_kernel (exact mode only): per (row, vocab leaf of 128
+//    columns) the running max in ascending column order and the ascending sum
+//    of exp(z - max), from materialised fp32 logits.  The tensor-core mode
+//    computes the same summaries inside the GEMM epilogue instead.
+//  * logprob_row_kernel: one warp per row.  Lane l reduces frontier node l of
+//    the halving tree over the Lv padded leaves (a whole subtree, streamed
+//    leaf by leaf with a small stack); the upper levels are xor-butterfly
+//    levels in which the left operand of every combine is the lower lane.  The
+//    T shard summaries are taken at their own level, written to the shard
+//    buffer, read back and combined by the top levels of the same tree.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace tbik {
+
+constexpr int VLEAF = 128;
+
+__global__ void vocab_stats_kernel(const float* __restrict__ z, const int32_t* __restrict__ targets,
+                                   float* __restrict__ stats, float* __restrict__ zt, int M, int V, int nvt) {
+    const size_t total = (size_t)M * nvt;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        const int row = (int)(i / nvt);
+        const int j = (int)(i - (size_t)row * nvt);
+        const float* zr = z + (size_t)row * V;
+        const int c0 = j * VLEAF;
+        const int c1 = min(c0 + VLEAF, V);
+        float m = zr[c0];
+        for (int c = c0 + 1; c < c1; ++c)
+            if (zr[c] > m) m = zr[c];
+        float s = 0.0f;
+        for (int c = c0; c < c1; ++c) s = __fadd_rn(s, exp_spec(__fsub_rn(zr[c], m)));
+        *reinterpret_cast<float2*>(stats + ((size_t)j * M + row) * 2) = make_float2(m, s);
+        const int t = targets[row];
+        if (t >= c0 && t < c1) zt[row] = zr[t];
+    }
+}
+
+__device__ __forceinline__ MS leaf_ms(const float* stats, int M, int nvt, int row, int j) {
+    MS r;
+    if (j < nvt) {
+        const float2 v = *reinterpret_cast<const float2*>(stats + ((size_t)j * M + row) * 2);
+        r.m = v.x;
+        r.s = v.y;
+    } else {
+        r.m = -INFINITY;
+        r.s = 0.0f;
+    }
+    return r;
+}
+
+__device__ __forceinline__ MS shfl_ms(MS v, int src_lane_mask) {
+    MS o;
+    o.m = __shfl_xor_sync(0xffffffffu, v.m, src_lane_mask);
+    o.s = __shfl_xor_sync(0xffffffffu, v.s, src_lane_mask);
+    return o;
+}
+
+// One butterfly level: lanes l and l^w hold sibling subtrees; the lower lane is the left one.
+__device__ __forceinline__ MS butterfly_ms(MS v, int lane, int w) {
+    const MS o = shfl_ms(v, w);
+    return (lane & w) ? ms_combine(o, v) : ms_combine(v, o);
+}
+
+constexpr int ROW_WARPS = 8;
+
+__global__ void __launch_bounds__(ROW_WARPS * 32)
+    logprob_row_kernel(const float* __restrict__ stats, const float* __restrict__ zt,
+                       const int32_t* __restrict__ targets, float* __restrict__ out, float* shard_ms, int M, int V,
+                       int nvt, int Lv, int T, int noninv) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+    if (row >= M) return;
+    MS fin;
+    if (!noninv) {
+        int d = 0;
+        while (d < 5 && (2 << d) <= Lv) ++d;  // largest d <= 5 with 2^d <= Lv
+        const int nf = 1 << d;
+        MS v;
+        v.m = -INFINITY;
+        v.s = 0.0f;
+        if (lane < nf) {
+            int lo = 0, n = Lv;
+            for (int lvl = 0; lvl < d; ++lvl) {
+                const int h = (n + 1) >> 1;
+                if ((lane >> (d - 1 - lvl)) & 1) {
+                    lo += h;
+                    n -= h;
+                } else {
+                    n = h;
+                }
+            }
+            MS stk[24];
+            int sp = 0;
+            for (int j = 0; j < n; ++j) {
+                MS cur = leaf_ms(stats, M, nvt, row, lo + j);
+                LeafOps ops;
+                leaf_ops(n, j, ops);
+                for (int i = 0; i < ops.npop; ++i) cur = ms_combine(stk[--sp], cur);
+                if (!ops.final_) stk[sp++] = cur;
+                else v = cur;
+            }
+        }
+        const int sl = nf / T;  // lanes per shard
+        for (int w = 1; w < sl; w <<= 1) v = butterfly_ms(v, lane, w);
+        if (lane < nf && (lane % sl) == 0)
+            *reinterpret_cast<float2*>(shard_ms + ((size_t)(lane / sl) * M + row) * 2) = make_float2(v.m, v.s);
+        __syncwarp();
+        MS sv;
+        sv.m = -INFINITY;
+        sv.s = 0.0f;
+        if (lane < T) {
+            const float2 t2 = *reinterpret_cast<const float2*>(shard_ms + ((size_t)lane * M + row) * 2);
+            sv.m = t2.x;
+            sv.s = t2.y;
+        }
+        for (int w = 1; w < T; w <<= 1) sv = butterfly_ms(sv, lane, w);
+        fin = sv;
+    } else {
+        // Non-invariant baseline: left-to-right inside each shard, then across shards.
+        const int Ls = Lv / T;
+        MS sv;
+        sv.m = -INFINITY;
+        sv.s = 0.0f;
+        if (lane < T) {
+            sv = leaf_ms(stats, M, nvt, row, lane * Ls);
+            for (int j = 1; j < Ls; ++j) sv = ms_combine(sv, leaf_ms(stats, M, nvt, row, lane * Ls + j));
+            *reinterpret_cast<float2*>(shard_ms + ((size_t)lane * M + row) * 2) = make_float2(sv.m, sv.s);
+        }
+        __syncwarp();
+        if (lane == 0) {
+            const float2 t0 = *reinterpret_cast<const float2*>(shard_ms + (size_t)row * 2);
+            sv.m = t0.x;
+            sv.s = t0.y;
+            for (int t = 1; t < T; ++t) {
+                const float2 tt = *reinterpret_cast<const float2*>(shard_ms + ((size_t)t * M + row) * 2);
+                MS b;
+                b.m = tt.x;
+                b.s = tt.y;
+                sv = ms_combine(sv, b);
+            }
+        }
+        fin = sv;
+    }
+    if (lane == 0) {
+        const int t = targets[row];
+        if (t < 0 || t >= V) {
+            set_error(TBIK_ERR_TARGET);
+            out[row] = __int_as_float(0x7fc00000);
+        } else {
+            out[row] = __fsub_rn(__fsub_rn(zt[row], fin.m), log_spec(fin.s));
+        }
+    }
+}
+
+}  // namespace tbik

@@ -1,0 +1,613 @@
+// Host side of the C ABI declared in include/tbik.h: argument checks, the
+// launch plan (frontier split of the tree, workspace carving), TMA tensor
+// maps and kernel launches.  One translation unit holds every kernel so the
+// device error word is a single symbol per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "device_common.cuh"
+#include "gemm_exact.cuh"
+#include "gemm_tc.cuh"
+#include "logprob.cuh"
+#include "reduce.cuh"
+#include "tbik.h"
+
+namespace {
+
+using namespace tbik;
+
+constexpr unsigned kModeMask = TBIK_EXACT | TBIK_TC | TBIK_NONINV | TBIK_B_NK | TBIK_OUT_BF16;
+constexpr int kMaxDevices = 64;
+
+unsigned g_debug_flags = 0;
+unsigned long long g_wait_ns = 2000000000ull;
+
+struct DeviceInfo {
+    bool init = false;
+    bool ok = false;
+    int sms = 0;
+    bool attrs_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+tbik_status device_info(int& dev, DeviceInfo*& info) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TBIK_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.init) {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return TBIK_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TBIK_ERR_CUDA;
+        d.ok = (major == 10);
+        d.init = true;
+    }
+    info = &d;
+    if (!d.ok) return TBIK_ERR_UNSUPPORTED;
+    if (!d.attrs_set) {
+        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TC_SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_LOGPROB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TC_SMEM_BYTES) != cudaSuccess)
+            return TBIK_ERR_CUDA;
+        d.attrs_set = true;
+    }
+    return TBIK_OK;
+}
+
+// ---------------------------------------------------------------- TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 row-major matrix with `inner` contiguous elements per row and `outer`
+// rows; box = box_inner x box_outer elements, 128-byte swizzle, zero OOB fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- tree plan
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+int ilog2(int x) {
+    int r = 0;
+    while ((1 << (r + 1)) <= x) ++r;
+    return r;
+}
+bool valid_T(int T) { return T == 1 || T == 2 || T == 4 || T == 8; }
+
+// Nodes at depth D of the halving tree over [lo, lo+n), left to right.
+void frontier(int lo, int n, int D, std::vector<std::pair<int, int>>& out) {
+    if (D == 0 || n == 1) {
+        out.emplace_back(lo, n);
+        return;
+    }
+    int h = (n + 1) / 2;
+    frontier(lo, h, D - 1, out);
+    frontier(lo + h, n - h, D - 1, out);
+}
+
+// Largest number of simultaneously pending left subtrees of >= 3 leaves while
+// streaming the tree over n leaves (they live in the global scratch).
+int max_big_pending(int n) {
+    if (n <= 1) return 0;
+    int h = (n + 1) / 2;
+    int l = max_big_pending(h);
+    int r = max_big_pending(n - h) + (h >= 3 ? 1 : 0);
+    return l > r ? l : r;
+}
+int max_stack_depth(int n) {
+    if (n <= 1) return 0;
+    int h = (n + 1) / 2;
+    int l = max_stack_depth(h);
+    int r = max_stack_depth(n - h) + 1;
+    return l > r ? l : r;
+}
+
+struct GemmPlan {
+    bool tc = false, noninv = false, b_nk = false, out_bf16 = false;
+    int M = 0, N = 0, K = 0, T = 1, leaf = 1;
+    int L = 0, D = 0, F = 1;
+    int tiles_m = 0, tiles_n = 0, units = 0, grid = 0, gs = 0;
+    bool direct = true;
+    std::vector<std::pair<int, int>> nodes;  // (first leaf, leaves) per frontier node
+    int leaf_eff = 1;                        // K elements per leaf as launched
+    size_t off_partials = 0, off_shards = 0, off_scratch = 0, total = 0;
+};
+
+tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int sms, GemmPlan& p) {
+    if (mode & ~kModeMask) return TBIK_ERR_ARG;
+    const bool exact = mode & TBIK_EXACT, tc = mode & TBIK_TC;
+    if (exact == tc) return TBIK_ERR_ARG;
+    if (M < 0 || N <= 0 || K <= 0 || leaf <= 0) return TBIK_ERR_ARG;
+    if (!valid_T(T) || K % leaf) return TBIK_ERR_SHAPE;
+    p.tc = tc;
+    p.noninv = mode & TBIK_NONINV;
+    p.b_nk = mode & TBIK_B_NK;
+    p.out_bf16 = mode & TBIK_OUT_BF16;
+    p.M = M, p.N = N, p.K = K, p.T = T, p.leaf = leaf;
+    p.L = K / leaf;
+    if (p.L % T) return TBIK_ERR_SHAPE;
+    const int bm = tc ? TC_BM : EX_BM, bn = tc ? TC_BN : EX_BN;
+    if (tc) {
+        if (N % 8 || K % 8) return TBIK_ERR_SHAPE;
+        if (p.noninv ? (K / T) % 16 : leaf % 16) return TBIK_ERR_SHAPE;
+    }
+    p.tiles_m = (M + bm - 1) / bm;
+    p.tiles_n = (N + bn - 1) / bn;
+    const long long tiles = (long long)p.tiles_m * p.tiles_n;
+    p.nodes.clear();
+    if (p.noninv) {
+        p.leaf_eff = K / T;
+        p.D = ilog2(T);
+        p.F = T;
+        for (int t = 0; t < T; ++t) p.nodes.emplace_back(t, 1);
+    } else {
+        p.leaf_eff = leaf;
+        const int d0 = ilog2(T);
+        int dmax = ilog2(p.L);
+        if (dmax > 6) dmax = 6;
+        if (tc ? false : (max_stack_depth(p.L) > EX_MAXD)) return TBIK_ERR_SHAPE;
+        const long long want = tc ? sms : 2LL * sms;
+        int D = d0;
+        while (D < dmax && tiles * (1LL << D) < want) ++D;
+        p.D = D;
+        frontier(0, p.L, D, p.nodes);
+        p.F = (int)p.nodes.size();
+        if (p.F != (1 << D)) return TBIK_ERR_SHAPE;  // cannot happen for 2^D <= L
+    }
+    if (p.nodes.size() > (size_t)TC_MAX_F) return TBIK_ERR_SHAPE;
+    for (auto& nd : p.nodes)
+        if (nd.first > 32767 || nd.second > 32767) return TBIK_ERR_SHAPE;
+    p.direct = (p.F == 1);
+    const long long units = tiles * p.F;
+    if (units > 0x7fffffffLL) return TBIK_ERR_SHAPE;
+    p.units = (int)units;
+    p.grid = p.units < sms ? p.units : sms;
+    if (p.grid < 1) p.grid = 1;
+    p.gs = 0;
+    if (tc)
+        for (auto& nd : p.nodes) {
+            int g = max_big_pending(nd.second);
+            if (g > p.gs) p.gs = g;
+        }
+    size_t off = 0;
+    const size_t mn = (size_t)M * N * sizeof(float);
+    if (!p.direct) {
+        p.off_partials = off;
+        off = align256(off + (size_t)p.F * mn);
+        if (!p.noninv && T > 1 && p.F > T) {
+            p.off_shards = off;
+            off = align256(off + (size_t)T * mn);
+        }
+    }
+    if (tc && p.gs > 0) {
+        p.off_scratch = off;
+        off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
+    }
+    p.total = off;
+    return TBIK_OK;
+}
+
+tbik_status launch_status() { return cudaGetLastError() == cudaSuccess ? TBIK_OK : TBIK_ERR_CUDA; }
+
+template <int G>
+void launch_tree_combine(const float* P, size_t MN, int groups, void* out, int bf16, cudaStream_t s, int sms) {
+    size_t work = (MN / 4) * groups;
+    int blocks = (int)((work + 255) / 256);
+    if (blocks > sms * 8) blocks = sms * 8;
+    if (blocks < 1) blocks = 1;
+    tree_combine_kernel<G><<<blocks, 256, 0, s>>>(P, MN, groups, out, bf16);
+}
+
+tbik_status tree_combine(const float* P, size_t MN, int G, int groups, void* out, int bf16, cudaStream_t s,
+                         int sms) {
+    switch (G) {
+        case 1: launch_tree_combine<1>(P, MN, groups, out, bf16, s, sms); break;
+        case 2: launch_tree_combine<2>(P, MN, groups, out, bf16, s, sms); break;
+        case 4: launch_tree_combine<4>(P, MN, groups, out, bf16, s, sms); break;
+        case 8: launch_tree_combine<8>(P, MN, groups, out, bf16, s, sms); break;
+        case 16: launch_tree_combine<16>(P, MN, groups, out, bf16, s, sms); break;
+        case 32: launch_tree_combine<32>(P, MN, groups, out, bf16, s, sms); break;
+        case 64: launch_tree_combine<64>(P, MN, groups, out, bf16, s, sms); break;
+        default: return TBIK_ERR_SHAPE;
+    }
+    return launch_status();
+}
+
+// Upper levels of the tree after the GEMM wrote F frontier partials.
+tbik_status finish_gemm(const GemmPlan& p, uint8_t* ws, void* C, cudaStream_t s, int sms) {
+    if (p.direct) return TBIK_OK;
+    const float* P = reinterpret_cast<const float*>(ws + p.off_partials);
+    const size_t MN = (size_t)p.M * p.N;
+    if (p.noninv) {
+        int blocks = (int)((MN + 255) / 256);
+        if (blocks > sms * 8) blocks = sms * 8;
+        seq_combine_kernel<<<blocks, 256, 0, s>>>(P, MN, p.T, C, p.out_bf16);
+        return launch_status();
+    }
+    if (p.T == 1 || p.F == p.T) return tree_combine(P, MN, p.F, 1, C, p.out_bf16, s, sms);
+    // T > 1 and F > T: shard partials first (one fp32 buffer per shard), then
+    // the cross-shard levels.
+    float* Q = reinterpret_cast<float*>(ws + p.off_shards);
+    tbik_status st = tree_combine(P, MN, p.F / p.T, p.T, Q, 0, s, sms);
+    if (st != TBIK_OK) return st;
+    return tree_combine(Q, MN, p.T, 1, C, p.out_bf16, s, sms);
+}
+
+tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, void* C, uint8_t* ws,
+                     cudaStream_t s, int sms) {
+    if (p.M == 0) return TBIK_OK;
+    if (p.tc) {
+        CUtensorMap ta, tb;
+        if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, TC_BK, TC_BM)) return TBIK_ERR_CUDA;
+        bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, TC_BK, TC_BN)
+                          : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, 64, TC_BK);
+        if (!okb) return TBIK_ERR_CUDA;
+        TcParams prm;
+        memset(&prm, 0, sizeof(prm));
+        prm.M = p.M, prm.N = p.N, prm.K = p.K;
+        prm.leaf = p.leaf_eff;
+        prm.F = p.F;
+        prm.tiles_m = p.tiles_m, prm.tiles_n = p.tiles_n, prm.group_m = 8;
+        prm.total_units = p.units;
+        prm.direct = p.direct;
+        prm.out_bf16 = p.out_bf16;
+        prm.out = C;
+        prm.partials = p.direct ? nullptr : reinterpret_cast<float*>(ws + p.off_partials);
+        prm.scratch = p.gs ? reinterpret_cast<float*>(ws + p.off_scratch) : nullptr;
+        prm.gs = p.gs;
+        prm.b_mn = p.b_nk ? 0 : 1;
+        const bool swap = g_debug_flags & TBIK_DEBUG_SWAP_MN_STRIDES;
+        prm.b_lbo = swap ? 1024u : (uint32_t)(TC_B_BYTES / 2);
+        prm.b_sbo = swap ? (uint32_t)(TC_B_BYTES / 2) : 1024u;
+        prm.debug = g_debug_flags;
+        prm.wait_ns = g_wait_ns;
+        for (int f = 0; f < p.F; ++f) {
+            prm.lo[f] = (short)p.nodes[f].first;
+            prm.nl[f] = (short)p.nodes[f].second;
+        }
+        gemm_tc_kernel<EPI_TREE><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+    } else {
+        ExParams prm;
+        memset(&prm, 0, sizeof(prm));
+        prm.A = A, prm.B = B;
+        prm.M = p.M, prm.N = p.N, prm.K = p.K;
+        prm.leaf = p.leaf_eff;
+        prm.F = p.F;
+        prm.tiles_m = p.tiles_m, prm.tiles_n = p.tiles_n;
+        prm.total_units = p.units;
+        prm.direct = p.direct;
+        prm.out_bf16 = p.out_bf16;
+        prm.out = C;
+        prm.partials = p.direct ? nullptr : reinterpret_cast<float*>(ws + p.off_partials);
+        for (int f = 0; f < p.F; ++f) {
+            prm.lo[f] = (short)p.nodes[f].first;
+            prm.nl[f] = (short)p.nodes[f].second;
+        }
+        int grid = p.units < sms * 4 ? p.units : sms * 4;
+        if (p.b_nk)
+            gemm_exact_kernel<1><<<grid, EX_THREADS, 0, s>>>(prm);
+        else
+            gemm_exact_kernel<0><<<grid, EX_THREADS, 0, s>>>(prm);
+    }
+    tbik_status st = launch_status();
+    if (st != TBIK_OK) return st;
+    return finish_gemm(p, ws, C, s, sms);
+}
+
+// ----------------------------------------------------------- logprob plan
+
+struct LogprobPlan {
+    int M = 0, V = 0, H = 0, T = 1, leaf = 256;
+    bool tc = false, noninv = false;
+    int Vpad = 0, Lv = 0, nvt = 0, Lk = 0, tiles_m = 0, units = 0, grid = 0, gs = 0;
+    size_t off_stats = 0, off_zt = 0, off_shard = 0, off_scratch = 0, off_z = 0, off_zgemm = 0, total = 0;
+    GemmPlan zplan;  // exact mode: the logits GEMM
+};
+
+tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, int sms, LogprobPlan& p) {
+    if (mode & ~(TBIK_EXACT | TBIK_TC | TBIK_NONINV)) return TBIK_ERR_ARG;
+    const bool exact = mode & TBIK_EXACT, tc = mode & TBIK_TC;
+    if (exact == tc) return TBIK_ERR_ARG;
+    if (M < 0 || V <= 0 || H <= 0 || leaf <= 0) return TBIK_ERR_ARG;
+    if (!valid_T(T) || H % leaf || H % 8 || leaf % 16) return TBIK_ERR_SHAPE;
+    p.M = M, p.V = V, p.H = H, p.T = T, p.leaf = leaf;
+    p.tc = tc;
+    p.noninv = mode & TBIK_NONINV;
+    const int step = VLEAF * TBIK_T_MAX;
+    p.Vpad = (int)(((long long)V + step - 1) / step * step);
+    p.Lv = p.Vpad / VLEAF;
+    p.nvt = (V + VLEAF - 1) / VLEAF;
+    p.Lk = H / leaf;
+    if (p.Lk > 32767) return TBIK_ERR_SHAPE;
+    p.tiles_m = (M + TC_BM - 1) / TC_BM;
+    const long long units = (long long)p.tiles_m * p.nvt;
+    if (units > 0x7fffffffLL) return TBIK_ERR_SHAPE;
+    p.units = (int)units;
+    p.grid = p.units < sms ? p.units : sms;
+    if (p.grid < 1) p.grid = 1;
+    p.gs = (tc && !p.noninv) ? max_big_pending(p.Lk) : 0;
+    size_t off = 0;
+    p.off_stats = off;
+    off = align256(off + (size_t)p.nvt * M * 2 * sizeof(float));
+    p.off_zt = off;
+    off = align256(off + (size_t)M * sizeof(float));
+    p.off_shard = off;
+    off = align256(off + (size_t)T * M * 2 * sizeof(float));
+    if (tc && p.gs > 0) {
+        p.off_scratch = off;
+        off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
+    }
+    if (exact) {
+        // logits z fp32 [M][V] from the exact GEMM (one K tree, or one chain for the baseline)
+        tbik_status st = plan_gemm(M > 0 ? M : 1, V, H, 1, p.noninv ? H : leaf, TBIK_EXACT | TBIK_B_NK, sms, p.zplan);
+        if (st != TBIK_OK) return st;
+        p.off_z = off;
+        off = align256(off + (size_t)M * V * sizeof(float));
+        p.off_zgemm = off;
+        off = align256(off + p.zplan.total);
+    }
+    p.total = off;
+    return TBIK_OK;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+
+extern "C" {
+
+const char* tbik_version(void) { return "tbik-b200 0.1 (sm_100a)"; }
+
+const char* tbik_status_string(tbik_status s) {
+    switch (s) {
+        case TBIK_OK: return "ok";
+        case TBIK_ERR_ARG: return "invalid argument";
+        case TBIK_ERR_SHAPE: return "unsupported shape";
+        case TBIK_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case TBIK_ERR_WORKSPACE: return "workspace missing or too small";
+        case TBIK_ERR_CUDA: return "CUDA error";
+        case TBIK_ERR_TIMEOUT: return "device wait timed out";
+        case TBIK_ERR_TARGET: return "target index out of range";
+        case TBIK_ERR_POSITION: return "RoPE position out of range";
+        case TBIK_ERR_UNSUPPORTED: return "device is not sm_100";
+    }
+    return "unknown status";
+}
+
+size_t tbik_gemm_workspace(int M, int N, int K, int T, int leaf, unsigned mode) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return (size_t)-1;
+    GemmPlan p;
+    if (plan_gemm(M, N, K, T, leaf, mode, info->sms, p) != TBIK_OK) return (size_t)-1;
+    return p.total;
+}
+
+tbik_status tbik_gemm(const uint16_t* A, const uint16_t* B, void* C, int M, int N, int K, int T, int leaf,
+                      unsigned mode, void* ws, size_t ws_bytes, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    GemmPlan p;
+    st = plan_gemm(M, N, K, T, leaf, mode, info->sms, p);
+    if (st != TBIK_OK) return st;
+    if (M == 0) return TBIK_OK;
+    if (!A || !B || !C) return TBIK_ERR_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return TBIK_ERR_ALIGN;
+    if (p.total > 0 && (!ws || ws_bytes < p.total)) return TBIK_ERR_WORKSPACE;
+    if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return TBIK_ERR_ALIGN;
+    return run_gemm(p, A, B, C, reinterpret_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream), info->sms);
+}
+
+tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16_t* gamma, uint16_t* y,
+                                  uint16_t* res_out, int tokens, int H, float eps, int T, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (tokens < 0 || H <= 0) return TBIK_ERR_ARG;
+    if (!valid_T(T) || H % 8) return TBIK_ERR_SHAPE;
+    const int nt = H / 8;
+    if (nt < 32 || nt > 1024 || (nt & (nt - 1)) || nt % T) return TBIK_ERR_SHAPE;
+    if (tokens == 0) return TBIK_OK;
+    if (!x || !res || !gamma || !y) return TBIK_ERR_ARG;
+    if (!aligned16(x) || !aligned16(res) || !aligned16(gamma) || !aligned16(y) || (res_out && !aligned16(res_out)))
+        return TBIK_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (nt) {
+        case 32: rmsnorm_residual_kernel<32><<<tokens, 32, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 64: rmsnorm_residual_kernel<64><<<tokens, 64, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 128: rmsnorm_residual_kernel<128><<<tokens, 128, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 256: rmsnorm_residual_kernel<256><<<tokens, 256, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 512: rmsnorm_residual_kernel<512><<<tokens, 512, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 1024: rmsnorm_residual_kernel<1024><<<tokens, 1024, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+    }
+    return launch_status();
+}
+
+tbik_status tbik_rope_table(float* table, int max_pos, int head_dim, double base, void* stream) {
+    if (!table || max_pos <= 0 || head_dim < 2 || head_dim > 512 || (head_dim & 1) || !(base > 0.0))
+        return TBIK_ERR_ARG;
+    const int half = head_dim / 2;
+    std::vector<float> h((size_t)max_pos * half * 2);
+    for (int p = 0; p < max_pos; ++p)
+        for (int i = 0; i < half; ++i) {
+            const double theta = std::pow(base, -(double)(2 * i) / (double)head_dim);
+            const double ang = (double)p * theta;
+            h[((size_t)p * half + i) * 2 + 0] = (float)std::cos(ang);
+            h[((size_t)p * half + i) * 2 + 1] = (float)std::sin(ang);
+        }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(table, h.data(), h.size() * sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return TBIK_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TBIK_ERR_CUDA;
+    return TBIK_OK;
+}
+
+tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (!a) return TBIK_ERR_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (a->q || a->k) {
+        if (a->tokens < 0 || a->heads <= 0 || a->max_pos <= 0) return TBIK_ERR_ARG;
+        if (a->head_dim <= 0 || a->head_dim % 16 || a->head_dim > 512) return TBIK_ERR_SHAPE;
+        if (!a->pos || !a->table || (a->q && !a->q_out) || (a->k && !a->k_out)) return TBIK_ERR_ARG;
+        if ((a->q && (!aligned16(a->q) || !aligned16(a->q_out))) || (a->k && (!aligned16(a->k) || !aligned16(a->k_out))) ||
+            !aligned16(a->table))
+            return TBIK_ERR_ALIGN;
+    }
+    if (a->g) {
+        if (!a->u || !a->out || a->n < 0) return TBIK_ERR_ARG;
+        if (a->n % 8) return TBIK_ERR_SHAPE;
+        if (!aligned16(a->g) || !aligned16(a->u) || !aligned16(a->out)) return TBIK_ERR_ALIGN;
+    }
+    if ((a->q || a->k) && a->tokens > 0) {
+        const size_t work = (size_t)a->tokens * a->heads * (a->head_dim / 16);
+        int blocks = (int)((work + 255) / 256);
+        if (blocks > info->sms * 16) blocks = info->sms * 16;
+        rope_kernel<<<dim3(blocks, 2), 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table, a->tokens,
+                                                    a->heads, a->head_dim, a->max_pos);
+        if ((st = launch_status()) != TBIK_OK) return st;
+    }
+    if (a->g && a->n > 0) {
+        const long long nv = a->n / 8;
+        long long blocks = (nv + 255) / 256;
+        if (blocks > (long long)info->sms * 16) blocks = (long long)info->sms * 16;
+        if (a->in_f32)
+            swiglu_kernel<1><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+        else
+            swiglu_kernel<0><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+        if ((st = launch_status()) != TBIK_OK) return st;
+    }
+    return TBIK_OK;
+}
+
+size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, unsigned mode) {
+    int dev;
+    DeviceInfo* info;
+    if (device_info(dev, info) != TBIK_OK) return (size_t)-1;
+    LogprobPlan p;
+    if (plan_logprob(M, V, H, T, leaf, mode, info->sms, p) != TBIK_OK) return (size_t)-1;
+    return p.total;
+}
+
+tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* targets, float* out, int M, int V,
+                         int H, int T, int leaf, unsigned mode, void* ws, size_t ws_bytes, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    LogprobPlan p;
+    st = plan_logprob(M, V, H, T, leaf, mode, info->sms, p);
+    if (st != TBIK_OK) return st;
+    if (M == 0) return TBIK_OK;
+    if (!hidden || !W || !targets || !out) return TBIK_ERR_ARG;
+    if (!aligned16(hidden) || !aligned16(W) || !aligned16(targets) || !aligned16(out)) return TBIK_ERR_ALIGN;
+    if (!ws || ws_bytes < p.total) return TBIK_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return TBIK_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
+    float* stats = reinterpret_cast<float*>(w8 + p.off_stats);
+    float* zt = reinterpret_cast<float*>(w8 + p.off_zt);
+    float* shard = reinterpret_cast<float*>(w8 + p.off_shard);
+    if (p.tc) {
+        CUtensorMap ta, tb;
+        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, TC_BK, TC_BM)) return TBIK_ERR_CUDA;
+        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, TC_BK, TC_BN)) return TBIK_ERR_CUDA;
+        TcParams prm;
+        memset(&prm, 0, sizeof(prm));
+        prm.M = M, prm.N = V, prm.K = H;
+        prm.leaf = p.noninv ? H : leaf;
+        prm.F = 1;
+        prm.tiles_m = p.tiles_m, prm.tiles_n = p.nvt;
+        prm.group_m = p.tiles_m;  // all row tiles of a vocab tile run together: W_lm is read once
+        prm.total_units = p.units;
+        prm.direct = 1;
+        prm.scratch = p.gs ? reinterpret_cast<float*>(w8 + p.off_scratch) : nullptr;
+        prm.gs = p.gs;
+        prm.b_mn = 0;
+        prm.targets = targets;
+        prm.stats = stats;
+        prm.zt = zt;
+        prm.V = V;
+        prm.debug = g_debug_flags & ~TBIK_DEBUG_WITHHOLD_ACC_ARRIVE;
+        prm.wait_ns = g_wait_ns;
+        prm.lo[0] = 0;
+        prm.nl[0] = (short)(p.noninv ? 1 : p.Lk);
+        gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+        if ((st = launch_status()) != TBIK_OK) return st;
+    } else {
+        float* z = reinterpret_cast<float*>(w8 + p.off_z);
+        GemmPlan zp;
+        st = plan_gemm(M, V, H, 1, p.noninv ? H : leaf, TBIK_EXACT | TBIK_B_NK, info->sms, zp);
+        if (st != TBIK_OK) return st;
+        if (zp.total > p.zplan.total) return TBIK_ERR_WORKSPACE;
+        st = run_gemm(zp, hidden, W, z, w8 + p.off_zgemm, s, info->sms);
+        if (st != TBIK_OK) return st;
+        const size_t work = (size_t)M * p.nvt;
+        int blocks = (int)((work + 255) / 256);
+        if (blocks > info->sms * 16) blocks = info->sms * 16;
+        vocab_stats_kernel<<<blocks, 256, 0, s>>>(z, targets, stats, zt, M, V, p.nvt);
+        if ((st = launch_status()) != TBIK_OK) return st;
+    }
+    logprob_row_kernel<<<(M + ROW_WARPS - 1) / ROW_WARPS, ROW_WARPS * 32, 0, s>>>(stats, zt, targets, out, shard, M,
+                                                                                V, p.nvt, p.Lv, T, p.noninv);
+    return launch_status();
+}
+
+tbik_status tbik_get_error(void* stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TBIK_ERR_CUDA;
+    unsigned e = 0;
+    if (cudaMemcpyFromSymbol(&e, tbik::g_err, sizeof(e)) != cudaSuccess) return TBIK_ERR_CUDA;
+    if (e) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(tbik::g_err, &zero, sizeof(zero)) != cudaSuccess) return TBIK_ERR_CUDA;
+    }
+    return (tbik_status)e;
+}
+
+tbik_status tbik_debug_set(unsigned flags, unsigned long long wait_limit_ns) {
+    g_debug_flags = flags;
+    g_wait_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;
+    return TBIK_OK;
+}
+
+}  // extern "C"

@@ -17,7 +17,12 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
-_SO = os.path.join(_HERE, "liboracle.so")
+_FMA = None
+
+
+def _so_path() -> str:
+    # The -mfma variant only runs on CPUs with FMA; both give the same bits.
+    return os.path.join(_HERE, "liboracle_fma.so" if _cpu_has_fma() else "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
@@ -41,15 +46,15 @@ def build(force: bool = False) -> str:
     ``-mfma`` only lets gcc inline the correctly rounded ``fmaf`` the source
     calls (the value is the same either way); contraction stays off.
     """
-    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
-        flags = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-                 "-fPIC", "-shared"]
+    so = _so_path()
+    if force or not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(_SRC):
+        flags = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
         if _cpu_has_fma():
             flags.append("-mfma")
-        tmp = _SO + f".tmp{os.getpid()}"
+        tmp = so + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", *flags, "-o", tmp, _SRC, "-lm"])
-        os.replace(tmp, _SO)
-    return _SO
+        os.replace(tmp, so)
+    return so
 
 
 def _load():

@@ -177,8 +177,13 @@ float oracle_log(float x) { return log_spec(x); }
 
 /* ------------------------------------------------------------------ GEMM */
 
-static float b_at(const uint16_t* B, int b_nk, int N, int K, int k, int n) {
-    return b_nk ? bf(B[(size_t)n * K + k]) : bf(B[(size_t)k * N + n]);
+/* A [K,N] operand copied to [N,K] so that each output reads one contiguous
+   column; a pure data movement, the arithmetic order is untouched. */
+static uint16_t* transpose_kn(const uint16_t* B, int K, int N) {
+    uint16_t* t = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)K * (size_t)N);
+    for (int k = 0; k < K; ++k)
+        for (int n = 0; n < N; ++n) t[(size_t)n * K + k] = B[(size_t)k * N + n];
+    return t;
 }
 
 /*
@@ -200,12 +205,14 @@ int oracle_gemm_tree(const uint16_t* A, const uint16_t* B, int b_nk, int M, int 
     int Ls = L / T;
     float* P = (float*)malloc(sizeof(float) * (size_t)L);
     float* Q = (float*)malloc(sizeof(float) * (size_t)T);
+    const uint16_t* Bt = b_nk ? B : transpose_kn(B, K, N);
     for (int i = 0; i < M; ++i) {
         for (int n = 0; n < N; ++n) {
+            const uint16_t* bcol = Bt + (size_t)n * K;
             for (int j = 0; j < L; ++j) {
                 float acc = 0.0f;
                 for (int k = j * leaf; k < (j + 1) * leaf; ++k)
-                    acc = fmaf(bf(A[(size_t)i * K + k]), b_at(B, b_nk, N, K, k, n), acc);
+                    acc = fmaf(bf(A[(size_t)i * K + k]), bf(bcol[k]), acc);
                 P[j] = acc;
             }
             for (int t = 0; t < T; ++t) {
@@ -215,6 +222,7 @@ int oracle_gemm_tree(const uint16_t* A, const uint16_t* B, int b_nk, int M, int 
             C[(size_t)i * N + n] = tree_f32(Q, 0, T);
         }
     }
+    if (!b_nk) free((void*)Bt);
     free(P);
     free(Q);
     return 0;
@@ -230,31 +238,36 @@ int oracle_gemm_noninv(const uint16_t* A, const uint16_t* B, int b_nk, int M, in
     if (M < 0 || N < 0 || K <= 0 || T <= 0 || K % T) return -1;
     int Ks = K / T;
     float* Q = (float*)malloc(sizeof(float) * (size_t)T);
+    const uint16_t* Bt = b_nk ? B : transpose_kn(B, K, N);
     for (int i = 0; i < M; ++i) {
         for (int n = 0; n < N; ++n) {
+            const uint16_t* bcol = Bt + (size_t)n * K;
             for (int t = 0; t < T; ++t) {
                 float acc = 0.0f;
                 for (int k = t * Ks; k < (t + 1) * Ks; ++k)
-                    acc = fmaf(bf(A[(size_t)i * K + k]), b_at(B, b_nk, N, K, k, n), acc);
+                    acc = fmaf(bf(A[(size_t)i * K + k]), bf(bcol[k]), acc);
                 Q[t] = acc;
                 if (shard_out) shard_out[((size_t)t * M + i) * N + n] = acc;
             }
             C[(size_t)i * N + n] = seq_f32(Q, 0, T);
         }
     }
+    if (!b_nk) free((void*)Bt);
     free(Q);
     return 0;
 }
 
 /* Double-precision product for tolerance checks (sequential binary64 sum). */
 void oracle_gemm_f64(const uint16_t* A, const uint16_t* B, int b_nk, int M, int N, int K, double* C) {
+    const uint16_t* Bt = b_nk ? B : transpose_kn(B, K, N);
     for (int i = 0; i < M; ++i)
         for (int n = 0; n < N; ++n) {
+            const uint16_t* bcol = Bt + (size_t)n * K;
             double acc = 0.0;
-            for (int k = 0; k < K; ++k)
-                acc += (double)bf(A[(size_t)i * K + k]) * (double)b_at(B, b_nk, N, K, k, n);
+            for (int k = 0; k < K; ++k) acc += (double)bf(A[(size_t)i * K + k]) * (double)bf(bcol[k]);
             C[(size_t)i * N + n] = acc;
         }
+    if (!b_nk) free((void*)Bt);
 }
 
 /* ------------------------------------------------------- residual RMSNorm */
