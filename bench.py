@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the tree-ordered invariant hot path on B200.
+
+One step = one pass of every kernel of the path over one batch of M = 4096
+tokens, with the sizes of the lm_head / down_proj / reduction workloads:
+
+  residual RMSNorm   x, res bf16 [4096, 4096]          -> y, res_out
+  RoPE (fp32)        q, k bf16 [4096, 32, 128], pos     -> q', k'
+  SwiGLU (fp32)      g, u bf16 [4096, 14336]            -> A bf16
+  down_proj GEMM     A [4096, 14336] x B [14336, 4096], leaf 256, T = 1, tensor cores -> h bf16
+  lm_head logprob    h [4096, 4096] x W_lm [151936, 4096]^T, targets -> logprob fp32 [4096]
+
+``value`` is whole-job tokens/s (all ranks; each rank runs its own batch:
+weak scaling, no collective on the data path).  ``--impl reference`` times the
+CPU oracle on a bounded sample of the same step instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+M_TOK = 4096
+H = 4096
+F = 14336
+V = 151936
+HEADS, HEAD_DIM, MAX_POS = 32, 128, 32768
+LEAF = 256
+METRIC = "invariant GEMM TFLOP/s + logprob tokens/s, bitwise-stable over T/batch"
+WORKLOAD = ("tbik hot path, M=4096 tokens/step: residual RMSNorm H=4096 -> RoPE fp32 q,k [32x128] -> "
+            "SwiGLU fp32 [14336] -> down_proj tree GEMM [4096x14336]x[14336x4096] leaf 256 T=1 (tcgen05) -> "
+            "lm_head logprob V=151936 H=4096 leaf 256 (fused tcgen05 + tree log-softmax)")
+GEMM_FLOP = 2.0 * M_TOK * F * H
+LOGPROB_FLOP = 2.0 * M_TOK * V * H
+KERNELS_PER_STEP = 6  # rmsnorm, rope, swiglu, gemm, logprob gemm+stats, logprob row tree
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), src="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # pragma: no cover
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def start(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_step_sample(tokens: int):
+    """Time the CPU oracle on `tokens` tokens of the step (every kernel of the path)."""
+    import oracle
+    if tokens not in _ORACLE_INPUTS:
+        std = 0.02 * np.sqrt(H)
+        _ORACLE_INPUTS[tokens] = dict(
+            d=synth.reduction_inputs(tokens), g=synth.normal_bf16(11, (tokens, F), std=std),
+            u=synth.normal_bf16(12, (tokens, F), std=std), b=synth.down_proj_weight(F, H, "kn"),
+            w=synth.normal_bf16(31, (V, H), std=0.02), targets=synth.uniform_int32(32, tokens, 0, V),
+            table=oracle.rope_table(MAX_POS, HEAD_DIM, 1e6))
+    c_ = _ORACLE_INPUTS[tokens]
+    d, g, u, b, w, targets, table = (c_["d"], c_["g"], c_["u"], c_["b"], c_["w"], c_["targets"], c_["table"])
+    t0 = time.perf_counter()
+    oracle.rmsnorm_residual(d["x"], d["res"], d["gamma"], eps=1e-6)
+    oracle.rope(d["q"], d["pos"], table)
+    oracle.rope(d["k"], d["pos"], table)
+    a = oracle.swiglu(g, u)
+    c = oracle.gemm_tree(a, b, b_nk=False, T=1, leaf=LEAF)
+    hid = np.array([oracle.bf16_rne(float(v)) for v in c.ravel()], dtype=np.uint16).reshape(c.shape)
+    oracle.logprob(hid, w, targets, T=1, leaf=LEAF)
+    return time.perf_counter() - t0
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    tokens = 1
+    for _ in range(args.warmup):
+        oracle_step_sample(tokens)
+    times = [oracle_step_sample(tokens) for _ in range(args.steps)]
+    total = sum(times)
+    value = tokens * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16 inputs)",
+        "data": "synthetic (seeded SplitMix64/Box-Muller)",
+        "config": {"workload": WORKLOAD, "tokens_per_step": M_TOK, "sample_tokens_per_step": tokens,
+                   "T": 1, "leaf": LEAF},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{tokens} token(s) of the step per step: RMSNorm, RoPE q/k, SwiGLU, one "
+                                   f"down_proj row, one lm_head logprob row (single-threaded C oracle)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- GPU path
+
+def run_tbik(args):
+    import torch
+    import torch.distributed as dist
+
+    import invariant_tree_ordered_b200 as tbik
+    from invariant_tree_ordered_b200 import build as libbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not os.path.exists(libbuild.LIB):
+        libbuild.build_library()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def bf(a):
+        return synth.as_torch_bf16(a)
+
+    # ---- inputs (seeded, synthetic), resident in HBM
+    d = synth.reduction_inputs(M_TOK)
+    std = 0.02 * np.sqrt(H)
+    host = {
+        "x": bf(d["x"]), "res": bf(d["res"]), "q": bf(d["q"]), "k": bf(d["k"]),
+        "pos": torch.from_numpy(d["pos"]),
+        "g": bf(synth.normal_bf16(11, (M_TOK, F), std=std)), "u": bf(synth.normal_bf16(12, (M_TOK, F), std=std)),
+        "targets": torch.from_numpy(synth.uniform_int32(32, M_TOK, 0, V)),
+    }
+    gamma = bf(d["gamma"]).to(dev)
+    B = bf(synth.down_proj_weight(F, H, "kn")).to(dev)
+    W = bf(synth.normal_bf16(31, (V, H), std=0.02)).to(dev)
+    table = tbik.rope_table(MAX_POS, HEAD_DIM, 1e6, device=dev)
+    inp = {k: v.to(dev) for k, v in host.items()}
+    y = torch.empty_like(inp["x"])
+    res_out = torch.empty_like(inp["x"])
+    qo = torch.empty_like(inp["q"])
+    ko = torch.empty_like(inp["k"])
+    A = torch.empty((M_TOK, F), dtype=torch.bfloat16, device=dev)
+    hid = torch.empty((M_TOK, H), dtype=torch.bfloat16, device=dev)
+    out = torch.empty(M_TOK, dtype=torch.float32, device=dev)
+    gws = torch.empty(max(tbik.gemm_workspace(M_TOK, H, F, 1, LEAF, tbik.TC | tbik.OUT_BF16), 256),
+                      dtype=torch.uint8, device=dev)
+    lws = torch.empty(tbik.logprob_workspace(M_TOK, V, H, 1, LEAF, tbik.TC), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for k in ("rms", "rope", "swiglu", "gemm", "logprob")}
+    acc = {k: 0.0 for k in ev}
+
+    def step(src, timed=False, lp_events=None):
+        def mark(k, i):
+            if timed:
+                ev[k][i].record(stream)
+        mark("rms", 0)
+        tbik.rmsnorm_residual(src["x"], src["res"], gamma, eps=1e-6, T=1, y=y, res_out=res_out, stream=stream)
+        mark("rms", 1)
+        mark("rope", 0)
+        tbik.rope_swiglu(q=src["q"], k=src["k"], pos=src["pos"], table=table, q_out=qo, k_out=ko, stream=stream)
+        mark("rope", 1)
+        mark("swiglu", 0)
+        tbik.rope_swiglu(g=src["g"], u=src["u"], out=A, stream=stream)
+        mark("swiglu", 1)
+        mark("gemm", 0)
+        tbik.gemm(A, B, T=1, leaf=LEAF, tc=True, out_bf16=True, out=hid, workspace=gws, stream=stream)
+        mark("gemm", 1)
+        mark("logprob", 0)
+        if lp_events is not None:
+            lp_events[0].record(stream)
+        tbik.logprob(hid, W, src["targets"], T=1, leaf=LEAF, tc=True, out=out, workspace=lws, stream=stream)
+        if lp_events is not None:
+            lp_events[1].record(stream)
+        mark("logprob", 1)
+
+    for _ in range(args.warmup):
+        step(inp)
+    if tbik.get_error(stream) != tbik.TBIK_OK:
+        raise RuntimeError("device error during warm-up")
+
+    # ---- device-timed region: inputs resident in HBM
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    lp_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    t0.record(stream)
+    for i in range(args.steps):
+        step(inp, lp_events=lp_ev[i])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    # dominant kernel: average duration of the logprob call inside the timed region
+    lp_live_ms = float(np.mean([a.elapsed_time(b) for a, b in lp_ev]))
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    status = tbik.get_error(stream)
+    if status != tbik.TBIK_OK:
+        raise RuntimeError(f"device error in timed region: {status}")
+
+    # ---- per-kernel durations (same stream, events around each call, averaged)
+    comp = {k: [] for k in ev}
+    barrier()
+    for _ in range(min(args.steps, 20)):
+        step(inp, timed=True)
+        torch.cuda.synchronize()
+        for k, (a, b) in ev.items():
+            comp[k].append(a.elapsed_time(b))
+    comp_ms = {k: float(np.mean(v)) for k, v in comp.items()}
+
+    # ---- end to end: host buffers in pinned memory, copies inside the timed region
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    out_host = torch.empty(M_TOK, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+    dst = {k: torch.empty_like(v) for k, v in inp.items()}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dst[k].copy_(v, non_blocking=True)
+        step(dst)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+
+    # ---- overhead of the invariant path over the non-invariant baseline (T = 1)
+    def avg_ms(fn, n=10):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    nws = torch.empty(max(tbik.gemm_workspace(M_TOK, H, F, 1, LEAF, tbik.TC | tbik.NONINV | tbik.OUT_BF16), 256),
+                      dtype=torch.uint8, device=dev)
+    nlws = torch.empty(tbik.logprob_workspace(M_TOK, V, H, 1, LEAF, tbik.TC | tbik.NONINV), dtype=torch.uint8,
+                       device=dev)
+    hid2 = torch.empty_like(hid)
+    out2 = torch.empty_like(out)
+    g_inv = avg_ms(lambda: tbik.gemm(A, B, T=1, leaf=LEAF, tc=True, out_bf16=True, out=hid2, workspace=gws))
+    g_non = avg_ms(lambda: tbik.gemm(A, B, T=1, leaf=LEAF, tc=True, noninv=True, out_bf16=True, out=hid2,
+                                     workspace=nws))
+    l_inv = avg_ms(lambda: tbik.logprob(hid, W, inp["targets"], T=1, leaf=LEAF, tc=True, out=out2, workspace=lws), 5)
+    l_non = avg_ms(lambda: tbik.logprob(hid, W, inp["targets"], T=1, leaf=LEAF, tc=True, noninv=True, out=out2,
+                                        workspace=nlws), 5)
+    gws8 = torch.empty(tbik.gemm_workspace(M_TOK, H, F, 8, LEAF, tbik.TC | tbik.OUT_BF16), dtype=torch.uint8,
+                       device=dev)
+    g_t8 = avg_ms(lambda: tbik.gemm(A, B, T=8, leaf=LEAF, tc=True, out_bf16=True, out=hid2, workspace=gws8))
+    tbik.get_error(stream)
+
+    pk = peaks()
+    lp_ms = lp_live_ms
+    achieved = LOGPROB_FLOP / (lp_ms * 1e-3) / 1e12
+    ms_step = ms_total / args.steps
+    value = world * M_TOK * args.steps / (ms_total * 1e-3)
+    gb = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9  # noqa: E731
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, f32 accumulate/reduce",
+        "data": "synthetic (seeded SplitMix64/Box-Muller, shapes and distributions of the lm_head/down_proj/"
+                "reduction workloads)",
+        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": M_TOK, "T": 1, "leaf": LEAF,
+                   "parallelism": f"{world} independent batches (weak scaling, no data-path collective)",
+                   "l2": "inputs larger than L2: every step streams W_lm (1.24 GB) and B (117 MB)"},
+        "components": {
+            "down_proj_gemm_tflops": GEMM_FLOP / (comp_ms["gemm"] * 1e-3) / 1e12,
+            "down_proj_gemm_tflops_T8": GEMM_FLOP / (g_t8 * 1e-3) / 1e12,
+            "logprob_tokens_per_s": M_TOK / (lp_ms * 1e-3),
+            "logprob_tflops": achieved,
+            "rmsnorm_gbs": gb(4 * M_TOK * H * 2, comp_ms["rms"]),
+            "rope_gbs": gb(2 * 2 * M_TOK * HEADS * HEAD_DIM * 2 + M_TOK * (4 + HEAD_DIM * 4), comp_ms["rope"]),
+            "swiglu_gbs": gb(3 * M_TOK * F * 2, comp_ms["swiglu"]),
+            "ms": comp_ms,
+            "overhead_vs_noninv": {"gemm": g_inv / g_non - 1.0, "logprob": l_inv / l_non - 1.0,
+                                   "gemm_ms": [g_inv, g_non], "logprob_ms": [l_inv, l_non]},
+        },
+        "roofline": {"kernel": "tbik_logprob (fused tcgen05 GEMM + vocab stats, then row tree)",
+                     "bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
+                     "frac": achieved / pk["bf16_sus"], "traffic": None,
+                     "peak_source": f"{pk['src']} bf16 sustained"},
+        "e2e": {"value": world * M_TOK * args.steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok = 2
+        dt = oracle_step_sample(tok)
+        line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{tok} tokens of the step (RMSNorm, RoPE, SwiGLU, down_proj rows, "
+                                          f"lm_head logprob rows), single-threaded C oracle, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_tbik(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
