@@ -87,9 +87,9 @@ typedef enum {
 #define TBIK_OUT_BF16 0x100u /* C bf16 [M,N], rounded once (RNE) from the fp32 tree root */
 
 /* Vocabulary columns per logprob leaf, and the largest shard count the vocab
-   padding is sized for: V is padded to Vpad = ceil(V / (128*8)) * 128*8 with
+   padding is sized for: V is padded to Vpad = ceil(V / (64*8)) * 64*8 with
    identity leaves (max -inf, sum 0), independent of T. */
-#define TBIK_VOCAB_LEAF 128
+#define TBIK_VOCAB_LEAF 64
 #define TBIK_T_MAX 8
 
 TBIK_API const char* tbik_version(void);
@@ -194,12 +194,12 @@ TBIK_API size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, uns
  * without materialising the logits (TBIK_TC):
  *   z[i,v]  = tree-ordered dot product over H (leaves of `leaf`, TREE over
  *             all H/leaf leaves), kept fp32;
- *   vocab leaf j = columns [128j, 128j+128) cut at V: m_j = max in ascending
+ *   vocab leaf j = columns [64j, 64j+64) cut at V: m_j = max in ascending
  *             column order, s_j = sum in ascending order of exp(z - m_j);
  *   (m,s) combine: m = max(ma,mb); s = sa*exp(ma-m) + sb*exp(mb-m) (products
  *             rounded separately); identity (-inf, 0);
  *   shard t (of T) owns the vocab leaves [t*Lv/T, (t+1)*Lv/T) of the padded
- *             Lv = Vpad/128; shard summaries and then the T shards combine by TREE;
+ *             Lv = Vpad/64; shard summaries and then the T shards combine by TREE;
  *   out[i]  = (z[i,target] - m) - log(s)  (library log specification).
  * hidden bf16 [M,H]; W_lm bf16 [V,H] row-major; targets int32 [M]; out fp32 [M].
  * H % leaf == 0, leaf % 16 == 0, H % 8 == 0, T in {1,2,4,8}.  A target outside

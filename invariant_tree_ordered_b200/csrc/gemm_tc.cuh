@@ -10,10 +10,12 @@
 // never on M, N or T, so a row's bits are the same for every batch size and
 // every shard count.
 //
-// CTA layout (192 threads, one CTA per SM, persistent over work units):
+// CTA layout (320 threads, one CTA per SM, persistent over work units):
 //   warp 0     TMA producer: A and B k-blocks (64 deep) into a 6-stage ring
 //   warp 1     TMEM allocator + single-thread MMA issuer
-//   warps 2-5  epilogue: drain each leaf from TMEM and apply the tree
+//   warps 2-9  epilogue: drain each leaf from TMEM and apply the tree; warp w
+//              reads TMEM lanes 32*(w%4).. (its row quadrant) and the 64
+//              columns of half (w-2)/4 of the tile
 // TMEM (512 columns x 128 lanes, fp32): columns [0,256) hold two leaf
 // accumulators (double buffer); [256,512) hold two pending subtree results of
 // size <= 2 leaves.  Pending subtrees of >= 3 leaves (written once per 3+
@@ -34,7 +36,8 @@ constexpr int TC_BK = 64;
 constexpr int TC_STAGES = 6;
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
 constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each owning 64 columns
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_MAX_F = 64;
 constexpr int TC_SLOT_FLOATS = TC_BM * TC_BN;
@@ -58,11 +61,11 @@ struct TcParams {
     uint32_t b_lbo, b_sbo;
     // logprob epilogue
     const int32_t* targets;
-    float* stats;  // [tiles_n][M][2]  (max, sum-exp) per row and vocab leaf
+    float* stats;  // [vocab leaves][M][2]  (max, sum-exp) per row and 64-column vocab leaf
     float* zt;     // [M]  logit of the target
     int V;
     unsigned debug;
-    unsigned long long wait_ns;
+    unsigned long long wait_cycles;  // bound of every device-side wait, in SM cycles
     short lo[TC_MAX_F];
     short nl[TC_MAX_F];
 };
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const uint64_t wait_ns = p.wait_ns;
+    const uint64_t wait_lim = p.wait_cycles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 128);
+            mbar_init(&acc_empty[b], 32 * TC_EPI_WARPS);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -174,6 +177,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
+            const bool b_mn = p.b_mn != 0;
             uint32_t q = 0;
             for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
                 int tm, tn, f;
@@ -182,11 +186,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const int nkb = (p.nl[f] * p.leaf + TC_BK - 1) / TC_BK;
                 for (int kb = 0; kb < nkb; ++kb) {
                     const int s = q % TC_STAGES;
-                    if (!mbar_wait(&empty[s], ((q / TC_STAGES) & 1) ^ 1, abort_flag, wait_ns)) goto producer_out;
+                    if (!mbar_wait(&empty[s], ((q / TC_STAGES) & 1) ^ 1, abort_flag, wait_lim)) goto producer_out;
                     mbar_arrive_expect_tx(&full[s], TC_A_BYTES + TC_B_BYTES);
                     const int kx = k0 + kb * TC_BK;
                     tma_load_2d(sA + s * TC_A_BYTES, &tmA, &full[s], kx, tm * TC_BM);
-                    if (!p.b_mn) {
+                    if (!b_mn) {
                         tma_load_2d(sB + s * TC_B_BYTES, &tmB, &full[s], kx, tn * TC_BN);
                     } else {
                         tma_load_2d(sB + s * TC_B_BYTES, &tmB, &full[s], tn * TC_BN, kx);
@@ -198,59 +202,85 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         producer_out:
             // Let the copies this thread issued land before the CTA can exit.
             for (uint32_t i = (q > (uint32_t)TC_STAGES ? q - TC_STAGES : 0u); i < q; ++i)
-                mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_ns);
+                mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_lim);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // One k-block (4 MMAs of K = 16) per ring stage.  Descriptors are built
+        // once per stage and advanced by adding the byte offset >> 4 to the
+        // start-address field, so the issue path per MMA is a few instructions.
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN, 0, p.b_mn);
+            const bool b_mn = p.b_mn != 0;
+            const uint32_t b_lbo = p.b_lbo, b_sbo = p.b_sbo;
+            const uint32_t sA_u = smem_u32(sA), sB_u = smem_u32(sB);
+            const int spl = p.leaf / 16;  // MMAs per leaf
+            const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
+            const bool aligned = (spl % 4) == 0;  // leaf is a multiple of the 64-deep k-block
+            const int kb_per_leaf = spl / 4;
             uint32_t q = 0, a = 0;
             for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
-                const int nsteps = p.nl[f] * p.leaf / 16;
-                const int spl = p.leaf / 16;
+                const int nsteps = p.nl[f] * spl;
                 uint32_t buf = 0;
-                int in_leaf = 0;
-                for (int st = 0; st < nsteps; ++st) {
-                    const int ks = st & 3;
-                    if (in_leaf == 0) {
-                        buf = a & 1;
-                        if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_ns)) goto mma_out;
-                        tc_fence_after();
-                    }
+                int in_leaf = 0, kb_in_leaf = 0;
+                for (int st = 0; st < nsteps; st += 4) {
                     const int s = q % TC_STAGES;
-                    if (ks == 0) {
-                        if (!mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_ns)) goto mma_out;
-                        tc_fence_after();
+                    if (!mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_lim)) goto mma_out;
+                    tc_fence_after();
+                    const uint64_t adesc = smem_desc_sw128(sA_u + s * TC_A_BYTES, 16, 1024);
+                    const uint64_t bdesc = b_mn ? smem_desc_sw128(sB_u + s * TC_B_BYTES, b_lbo, b_sbo)
+                                                : smem_desc_sw128(sB_u + s * TC_B_BYTES, 16, 1024);
+                    if (aligned) {
+                        // The leaf is a whole number of k-blocks: straight-line burst.
+                        if (kb_in_leaf == 0) {
+                            buf = a & 1;
+                            if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_lim)) goto mma_out;
+                            tc_fence_after();
+                        }
+                        const uint32_t d = tmem_base + buf * TC_BN;
+                        tc_mma(d, adesc, bdesc, idesc, kb_in_leaf != 0 ? 1u : 0u);
+                        tc_mma(d, adesc + 2, bdesc + b_step, idesc, 1u);
+                        tc_mma(d, adesc + 4, bdesc + 2 * b_step, idesc, 1u);
+                        tc_mma(d, adesc + 6, bdesc + 3 * b_step, idesc, 1u);
+                        if (++kb_in_leaf == kb_per_leaf) {
+                            tc_commit(&acc_full[buf]);
+                            ++a;
+                            kb_in_leaf = 0;
+                        }
+                    } else {
+                        const int nk = min(4, nsteps - st);
+                        for (int ks = 0; ks < nk; ++ks) {
+                            if (in_leaf == 0) {
+                                buf = a & 1;
+                                if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_lim))
+                                    goto mma_out;
+                                tc_fence_after();
+                            }
+                            tc_mma(tmem_base + buf * TC_BN, adesc + (uint64_t)(ks * 2), bdesc + b_step * ks, idesc,
+                                   in_leaf != 0 ? 1u : 0u);
+                            if (++in_leaf == spl) {
+                                tc_commit(&acc_full[buf]);
+                                ++a;
+                                in_leaf = 0;
+                            }
+                        }
                     }
-                    const uint64_t adesc = smem_desc_sw128(smem_u32(sA + s * TC_A_BYTES) + ks * 32, 16, 1024);
-                    uint64_t bdesc;
-                    if (!p.b_mn)
-                        bdesc = smem_desc_sw128(smem_u32(sB + s * TC_B_BYTES) + ks * 32, 16, 1024);
-                    else
-                        bdesc = smem_desc_sw128(smem_u32(sB + s * TC_B_BYTES) + ks * 2048, p.b_lbo, p.b_sbo);
-                    tc_mma(tmem_base + buf * TC_BN, adesc, bdesc, idesc, in_leaf != 0 ? 1u : 0u);
-                    if (ks == 3 || st == nsteps - 1) {
-                        tc_commit(&empty[s]);
-                        ++q;
-                    }
-                    if (++in_leaf == spl) {
-                        tc_commit(&acc_full[buf]);
-                        ++a;
-                        in_leaf = 0;
-                    }
+                    tc_commit(&empty[s]);
+                    ++q;
                 }
             }
         mma_out:
             // Every MMA issued by this thread retires before TMEM is released.
             tc_commit(done);
-            mbar_drain(done, 0, wait_ns);
+            mbar_drain(done, 0, wait_lim);
         }
     } else {
         // ------------------------------------------------ epilogue
-        const int ew = warp & 3;
-        const int rt = ew * 32 + lane;  // row within the tile
+        const int ew = warp & 3;           // TMEM lane quadrant = rows 32*ew .. 32*ew+31
+        const int half = (warp - 2) >> 2;  // columns [64*half, 64*half+64)
+        const int rt = ew * 32 + lane;     // row within the tile
         const uint32_t tl = tmem_base + ((uint32_t)(ew * 32) << 16);
         uint32_t a = 0;
         for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
@@ -258,30 +288,45 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tc_decode(p, u, tm, tn, f);
             const int n = p.nl[f];
             const int row = tm * TC_BM + rt;
-            int tsp = 0, gsp = 0;
+            int tsp = 0, gsp = 0;  // pending subtrees in TMEM slots / in the global scratch
             for (int j = 0; j < n; ++j) {
                 const uint32_t buf = a & 1;
-                if (!mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_ns)) goto epi_out;
+                if (!mbar_wait_sleepy(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim)) goto epi_out;
                 tc_fence_after();
                 __syncwarp();
                 LeafOps ops;
                 leaf_ops(n, j, ops);
-                int pop_slot[24];
-                int t2 = tsp, g2 = gsp;
-                for (int i = 0; i < ops.npop; ++i) pop_slot[i] = (ops.pop_size[i] <= 2) ? --t2 : -(--g2) - 1;
+                // Pops come deepest first: the small subtrees (<= 2 leaves, TMEM
+                // slots) precede the large ones (global scratch).
+                int ns = 0;
+                while (ns < ops.npop && ops.pop_size[ns] <= 2) ++ns;
+                const int nb = ops.npop - ns;
                 const bool push_small = ops.push_size <= 2;
-                int push_slot = 0;
-                if (!ops.final_) push_slot = push_small ? t2++ : g2++;
+                const int t_after = tsp - ns, g_after = gsp - nb;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = half * 2 + cc;
+                    uint32_t r0[32], r1[32], r2[32];
+                    tmem_ld32_nowait(tl + buf * TC_BN + c * 32, r0);
+                    if (ns >= 1) tmem_ld32_nowait(tl + 256 + (tsp - 1) * TC_BN + c * 32, r1);
+                    if (ns >= 2) tmem_ld32_nowait(tl + 256 + (tsp - 2) * TC_BN + c * 32, r2);
+                    tmem_wait_ld(r0);
                     float v[32];
-                    tmem_ld32(tl + buf * TC_BN + c * 32, v);
-                    for (int i = 0; i < ops.npop; ++i) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r0[k]);
+                    if (ns >= 1) {
+                        tie32(r1);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r1[k]), v[k]);
+                    }
+                    if (ns >= 2) {
+                        tie32(r2);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r2[k]), v[k]);
+                    }
+                    for (int i = 0; i < nb; ++i) {
                         float w[32];
-                        if (pop_slot[i] >= 0)
-                            tmem_ld32(tl + 256 + pop_slot[i] * TC_BN + c * 32, w);
-                        else
-                            scratch_ld(scratch_slot(p, -pop_slot[i] - 1), c, rt, w);
+                        scratch_ld(scratch_slot(p, gsp - 1 - i), c, rt, w);
 #pragma unroll
                         for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(w[k], v[k]);
                     }
@@ -293,61 +338,64 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                 store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row,
                                             tn * TC_BN + c * 32, v);
                         } else {
-                            tmem_st32(tl + 256 + c * 32, v);  // stage the logits in slot 0
+                            tmem_st32_nowait(tl + 256 + c * 32, v);  // logits of this vocab leaf, slot 0
                         }
                     } else if (push_small) {
-                        tmem_st32(tl + 256 + push_slot * TC_BN + c * 32, v);
+                        tmem_st32_nowait(tl + 256 + t_after * TC_BN + c * 32, v);
                     } else {
-                        scratch_st(scratch_slot(p, push_slot), c, rt, v);
+                        scratch_st(scratch_slot(p, g_after), c, rt, v);
                     }
-                    __syncwarp();
                 }
-                tsp = t2;
-                gsp = g2;
+                tmem_wait_st();
+                tsp = t_after + ((!ops.final_ && push_small) ? 1 : 0);
+                gsp = g_after + ((!ops.final_ && !push_small) ? 1 : 0);
                 tc_fence_before();
                 if (!(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) mbar_arrive(&acc_empty[buf]);
                 ++a;
             }
             if (EPI == EPI_LOGPROB) {
-                // Vocab leaf = this tile's 128 columns: running max in ascending
-                // column order, then the ascending sum of exp(z - max).
-                const int n0 = tn * TC_BN;
-                const int tgt = (row < p.M) ? p.targets[row] : -1;
-                float m = 0.0f, zval = 0.0f;
-                bool have_t = false;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float v[32];
-                    tmem_ld32(tl + 256 + c * 32, v);
+                // This warp's 64 columns are one vocab leaf: running max in
+                // ascending column order, then the ascending sum of exp(z - max).
+                const int c0 = tn * TC_BN + half * 64;
+                const int vleaf = 2 * tn + half;
+                if (c0 < p.V) {
+                    const int tgt = (row < p.M) ? p.targets[row] : -1;
+                    float z[64];
+                    {
+                        uint32_t r0[32], r1[32];
+                        tmem_ld32_nowait(tl + 256 + (half * 2) * 32, r0);
+                        tmem_ld32_nowait(tl + 256 + (half * 2 + 1) * 32, r1);
+                        tmem_wait_ld(r0);
+                        tie32(r1);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int col = n0 + c * 32 + k;
-                        if (col < p.V) {
-                            if (c == 0 && k == 0)
-                                m = v[k];
-                            else if (v[k] > m)
-                                m = v[k];
-                            if (col == tgt) {
-                                zval = v[k];
+                        for (int k = 0; k < 32; ++k) {
+                            z[k] = __uint_as_float(r0[k]);
+                            z[32 + k] = __uint_as_float(r1[k]);
+                        }
+                    }
+                    const int ncol = min(64, p.V - c0);
+                    float m = z[0];
+                    float zval = 0.0f;
+                    bool have_t = (tgt == c0);
+                    if (have_t) zval = z[0];
+#pragma unroll
+                    for (int k = 1; k < 64; ++k) {
+                        if (k < ncol) {
+                            if (z[k] > m) m = z[k];
+                            if (c0 + k == tgt) {
+                                zval = z[k];
                                 have_t = true;
                             }
                         }
                     }
-                }
-                float s = 0.0f;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float v[32];
-                    tmem_ld32(tl + 256 + c * 32, v);
+                    float s = 0.0f;
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int col = n0 + c * 32 + k;
-                        if (col < p.V) s = __fadd_rn(s, exp_spec(__fsub_rn(v[k], m)));
+                    for (int k = 0; k < 64; ++k)
+                        if (k < ncol) s = __fadd_rn(s, exp_spec(__fsub_rn(z[k], m)));
+                    if (row < p.M) {
+                        *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
+                        if (have_t) p.zt[row] = zval;
                     }
-                }
-                if (row < p.M) {
-                    *reinterpret_cast<float2*>(p.stats + ((size_t)tn * p.M + row) * 2) = make_float2(m, s);
-                    if (have_t) p.zt[row] = zval;
                 }
                 __syncwarp();
             }

@@ -2,7 +2,7 @@
 // vocabulary reduction in tree order (TBIK summary page, 技术框架) and the
 // per-token logprob as the compared quantity (IsoExec brief, 壹/叁).
 //
-//  * vocab_stats_kernel (exact mode only): per (row, vocab leaf of 128
+//  * vocab_stats_kernel (exact mode only): per (row, vocab leaf of 64
 //    columns) the running max in ascending column order and the ascending sum
 //    of exp(z - max), from materialised fp32 logits.  The tensor-core mode
 //    computes the same summaries inside the GEMM epilogue instead.
@@ -18,7 +18,7 @@
 
 namespace tbik {
 
-constexpr int VLEAF = 128;
+constexpr int VLEAF = 64;  // vocabulary columns per leaf
 
 __global__ void vocab_stats_kernel(const float* __restrict__ z, const int32_t* __restrict__ targets,
                                    float* __restrict__ stats, float* __restrict__ zt, int M, int V, int nvt) {

@@ -32,6 +32,7 @@ struct DeviceInfo {
     bool init = false;
     bool ok = false;
     int sms = 0;
+    int clock_khz = 0;
     bool attrs_set = false;
 };
 DeviceInfo g_dev[kMaxDevices];
@@ -45,6 +46,8 @@ tbik_status device_info(int& dev, DeviceInfo*& info) {
         int major = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return TBIK_ERR_CUDA;
         if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return TBIK_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.clock_khz, cudaDevAttrClockRate, dev) != cudaSuccess || d.clock_khz <= 0)
+            d.clock_khz = 2000000;
         d.ok = (major == 10);
         d.init = true;
     }
@@ -265,8 +268,15 @@ tbik_status finish_gemm(const GemmPlan& p, uint8_t* ws, void* C, cudaStream_t s,
     return tree_combine(Q, MN, p.T, 1, C, p.out_bf16, s, sms);
 }
 
+// Wait bound in SM cycles at the device's maximum clock (a slower clock only
+// lengthens the bound in wall time).
+unsigned long long wait_cycles(const DeviceInfo* d) {
+    return (unsigned long long)((double)g_wait_ns * (double)d->clock_khz * 1e-6);
+}
+
 tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, void* C, uint8_t* ws,
-                     cudaStream_t s, int sms) {
+                     cudaStream_t s, const DeviceInfo* info) {
+    const int sms = info->sms;
     if (p.M == 0) return TBIK_OK;
     if (p.tc) {
         CUtensorMap ta, tb;
@@ -292,7 +302,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.b_lbo = swap ? 1024u : (uint32_t)(TC_B_BYTES / 2);
         prm.b_sbo = swap ? (uint32_t)(TC_B_BYTES / 2) : 1024u;
         prm.debug = g_debug_flags;
-        prm.wait_ns = g_wait_ns;
+        prm.wait_cycles = wait_cycles(info);
         for (int f = 0; f < p.F; ++f) {
             prm.lo[f] = (short)p.nodes[f].first;
             prm.nl[f] = (short)p.nodes[f].second;
@@ -331,7 +341,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
 struct LogprobPlan {
     int M = 0, V = 0, H = 0, T = 1, leaf = 256;
     bool tc = false, noninv = false;
-    int Vpad = 0, Lv = 0, nvt = 0, Lk = 0, tiles_m = 0, units = 0, grid = 0, gs = 0;
+    int Vpad = 0, Lv = 0, nvl = 0, nvt = 0, Lk = 0, tiles_m = 0, units = 0, grid = 0, gs = 0;
     size_t off_stats = 0, off_zt = 0, off_shard = 0, off_scratch = 0, off_z = 0, off_zgemm = 0, total = 0;
     GemmPlan zplan;  // exact mode: the logits GEMM
 };
@@ -348,7 +358,8 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
     const int step = VLEAF * TBIK_T_MAX;
     p.Vpad = (int)(((long long)V + step - 1) / step * step);
     p.Lv = p.Vpad / VLEAF;
-    p.nvt = (V + VLEAF - 1) / VLEAF;
+    p.nvl = (V + VLEAF - 1) / VLEAF;        // vocab leaves holding columns
+    p.nvt = (V + TC_BN - 1) / TC_BN;        // 128-column GEMM tiles (two vocab leaves each)
     p.Lk = H / leaf;
     if (p.Lk > 32767) return TBIK_ERR_SHAPE;
     p.tiles_m = (M + TC_BM - 1) / TC_BM;
@@ -360,7 +371,7 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
     p.gs = (tc && !p.noninv) ? max_big_pending(p.Lk) : 0;
     size_t off = 0;
     p.off_stats = off;
-    off = align256(off + (size_t)p.nvt * M * 2 * sizeof(float));
+    off = align256(off + (size_t)p.nvl * M * 2 * sizeof(float));
     p.off_zt = off;
     off = align256(off + (size_t)M * sizeof(float));
     p.off_shard = off;
@@ -430,7 +441,7 @@ tbik_status tbik_gemm(const uint16_t* A, const uint16_t* B, void* C, int M, int 
     if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return TBIK_ERR_ALIGN;
     if (p.total > 0 && (!ws || ws_bytes < p.total)) return TBIK_ERR_WORKSPACE;
     if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return TBIK_ERR_ALIGN;
-    return run_gemm(p, A, B, C, reinterpret_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream), info->sms);
+    return run_gemm(p, A, B, C, reinterpret_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream), info);
 }
 
 tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16_t* gamma, uint16_t* y,
@@ -568,7 +579,7 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         prm.zt = zt;
         prm.V = V;
         prm.debug = g_debug_flags & ~TBIK_DEBUG_WITHHOLD_ACC_ARRIVE;
-        prm.wait_ns = g_wait_ns;
+        prm.wait_cycles = wait_cycles(info);
         prm.lo[0] = 0;
         prm.nl[0] = (short)(p.noninv ? 1 : p.Lk);
         gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
@@ -579,16 +590,16 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         st = plan_gemm(M, V, H, 1, p.noninv ? H : leaf, TBIK_EXACT | TBIK_B_NK, info->sms, zp);
         if (st != TBIK_OK) return st;
         if (zp.total > p.zplan.total) return TBIK_ERR_WORKSPACE;
-        st = run_gemm(zp, hidden, W, z, w8 + p.off_zgemm, s, info->sms);
+        st = run_gemm(zp, hidden, W, z, w8 + p.off_zgemm, s, info);
         if (st != TBIK_OK) return st;
-        const size_t work = (size_t)M * p.nvt;
+        const size_t work = (size_t)M * p.nvl;
         int blocks = (int)((work + 255) / 256);
         if (blocks > info->sms * 16) blocks = info->sms * 16;
-        vocab_stats_kernel<<<blocks, 256, 0, s>>>(z, targets, stats, zt, M, V, p.nvt);
+        vocab_stats_kernel<<<blocks, 256, 0, s>>>(z, targets, stats, zt, M, V, p.nvl);
         if ((st = launch_status()) != TBIK_OK) return st;
     }
     logprob_row_kernel<<<(M + ROW_WARPS - 1) / ROW_WARPS, ROW_WARPS * 32, 0, s>>>(stats, zt, targets, out, shard, M,
-                                                                                V, p.nvt, p.Lv, T, p.noninv);
+                                                                                V, p.nvl, p.Lv, T, p.noninv);
     return launch_status();
 }
 

@@ -26,7 +26,7 @@ def _so_path() -> str:
 _lock = threading.Lock()
 _lib = None
 
-VLEAF = 128  # vocabulary columns per logprob leaf
+VLEAF = 64  # vocabulary columns per logprob leaf
 
 
 def _cpu_has_fma() -> bool:
