@@ -210,6 +210,36 @@ TBIK_API tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W_lm, 
                          float* out, int M, int V, int H, int T, int leaf, unsigned mode, void* ws,
                          size_t ws_bytes, void* stream);
 
+/*
+ * tbik_logprob_noalloc -- the pages have no counterpart for this entry point.
+ *
+ * For callers that cannot allocate device memory (code that must not call
+ * cudaMalloc, for example while its stream is being captured or under an
+ * allocator that forbids side allocations, and plain C callers with no device
+ * allocator of their own).  Same arguments and results as tbik_logprob in
+ * tensor-core mode (mode = TBIK_TC, optionally | TBIK_NONINV), minus the
+ * workspace: the scratch comes from one fixed device array of
+ * TBIK_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits.  The caller still passes inputs and
+ * outputs.  Nothing is allocated or freed.
+ *  - Returns TBIK_ERR_WORKSPACE, and launches nothing, when the arguments need
+ *    more scratch than TBIK_NOALLOC_SCRATCH_BYTES (that is, when
+ *    tbik_logprob_workspace() for the same arguments is larger).  For the
+ *    151936 x 4096 lm_head with leaf 256 this allows up to 742 rows per call.
+ *  - Returns TBIK_ERR_ARG for any mode without TBIK_TC or with TBIK_EXACT.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents.
+ *    Nothing in it needs clearing (every value read is written earlier in the
+ *    same call), but calls that overlap on the GPU (two streams, or two host
+ *    threads on one device) race on it: serialise them.
+ */
+#define TBIK_NOALLOC_SCRATCH_BYTES (32u << 20)
+TBIK_API tbik_status tbik_logprob_noalloc(const uint16_t* hidden, const uint16_t* W_lm, const int32_t* targets,
+                                          float* out, int M, int V, int H, int T, int leaf, unsigned mode,
+                                          void* stream);
+
 /* ---- errors -------------------------------------------------------------- */
 
 /*

@@ -262,3 +262,33 @@ def get_error(stream=None) -> int:
 
 def debug_set(flags: int = 0, wait_limit_ns: int = 0):
     _check(load_library().tbik_debug_set(flags, wait_limit_ns), "tbik_debug_set")
+
+
+_noalloc_ready = False
+
+
+def logprob_noalloc(hidden, W, targets, *, T: int = 1, leaf: int = 256, noninv: bool = False, out=None,
+                    stream=None):
+    """tbik_logprob_noalloc: tensor-core logprob whose scratch is the library's
+    fixed device array, for callers that cannot allocate a workspace.  Only the
+    output (when not given) is allocated here, by torch."""
+    global _noalloc_ready
+    torch = _torch()
+    lib = load_library()
+    if not _noalloc_ready:
+        vp, i32, u32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+        lib.tbik_logprob_noalloc.restype = i32
+        lib.tbik_logprob_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32, vp]
+        _noalloc_ready = True
+    _need(hidden, torch.bfloat16, "hidden")
+    _need(W, torch.bfloat16, "W_lm")
+    _need(targets, torch.int32, "targets")
+    M, H = hidden.shape
+    V = W.shape[0]
+    mode = TC | (NONINV if noninv else 0)
+    if out is None:
+        out = torch.empty(M, dtype=torch.float32, device=hidden.device)
+    _check(lib.tbik_logprob_noalloc(_ptr(hidden), _ptr(W), _ptr(targets), _ptr(out), M, V, H, T, leaf, mode,
+                                    _stream_handle(stream)), "tbik_logprob_noalloc")
+    return out
+

@@ -52,7 +52,7 @@ def build_library(force: bool = False, verbose: bool = False, extra=None) -> str
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "tbik_api.cu"), "-o", tmp]
+           *sorted(glob.glob(os.path.join(CSRC, "*.cu"))), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)

@@ -1,0 +1,74 @@
+"""tbik_logprob_noalloc, the entry point for callers that cannot allocate
+device memory (for example code that must not call cudaMalloc while its stream
+is being captured, or plain C callers without a device allocator).
+
+It must give the same logprobs as the allocating entry point tbik_logprob on
+consecutive calls (the scratch array it shares between calls keeps the previous
+call's contents), and refuse, without launching anything, arguments whose
+scratch would not fit its fixed array.  This file is collected last so a run
+that stops at the first failure has already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+from tests.gpu_util import dev_bf16, dev_i32, host_f32, u32  # noqa: E402
+
+import invariant_tree_ordered_b200 as tbik  # noqa: E402
+
+SCRATCH_BYTES = 32 << 20
+
+
+def _entry():
+    lib = tbik.load_library()
+    fn = lib.tbik_logprob_noalloc
+    vp, i32, u32_ = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+    fn.restype = i32
+    fn.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32_, vp]
+    return lib, fn
+
+
+def test_noalloc_logprob_matches_allocating_entry_point_on_two_calls():
+    lib, noalloc = _entry()
+    stream = torch.cuda.current_stream().cuda_stream
+    V, H, leaf = 20000, 2048, 256  # 8 K leaves: the kernels use the scratch's global stack
+    w = dev_bf16(synth.normal_bf16(500, (V, H), std=0.05))
+    for M, T, seed in ((300, 2, 501), (200, 8, 503)):
+        h = dev_bf16(synth.normal_bf16(seed, (M, H)))
+        t = dev_i32(synth.uniform_int32(seed + 1, M, 0, V))
+        ref = host_f32(tbik.logprob(h, w, t, T=T, leaf=leaf, tc=True))
+        assert tbik.get_error() == tbik.TBIK_OK
+        out = torch.full((M,), float("nan"), dtype=torch.float32, device="cuda")
+        status = noalloc(h.data_ptr(), w.data_ptr(), t.data_ptr(), out.data_ptr(), M, V, H, T, leaf, tbik.TC, stream)
+        assert status == tbik.TBIK_OK
+        assert tbik.get_error() == tbik.TBIK_OK
+        got = host_f32(out)
+        assert np.all(np.isfinite(got))
+        assert np.max(np.abs(got - ref)) <= 1e-4
+        assert np.array_equal(u32(got), u32(ref))
+
+
+def test_noalloc_refuses_arguments_beyond_its_scratch():
+    lib, noalloc = _entry()
+    stream = torch.cuda.current_stream().cuda_stream
+    V, H, leaf, T = 151936, 4096, 256, 8
+    assert lib.tbik_logprob_workspace(742, V, H, T, leaf, tbik.TC) <= SCRATCH_BYTES
+    assert lib.tbik_logprob_workspace(800, V, H, T, leaf, tbik.TC) > SCRATCH_BYTES
+    # The size check comes before any pointer is used: small stand-in buffers.
+    dummy = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    tg = torch.zeros(800, dtype=torch.int32, device="cuda")
+    out = torch.full((800,), float("nan"), dtype=torch.float32, device="cuda")
+    status = noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 800, V, H, T, leaf, tbik.TC,
+                     stream)
+    assert status == tbik.TBIK_ERR_WORKSPACE
+    assert noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 4, V, H, T, leaf, tbik.EXACT,
+                   stream) == tbik.TBIK_ERR_ARG
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all()
+    assert tbik.get_error() == tbik.TBIK_OK
