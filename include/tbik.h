@@ -225,7 +225,8 @@ TBIK_API tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W_lm, 
  *  - Returns TBIK_ERR_WORKSPACE, and launches nothing, when the arguments need
  *    more scratch than TBIK_NOALLOC_SCRATCH_BYTES (that is, when
  *    tbik_logprob_workspace() for the same arguments is larger).  For the
- *    151936 x 4096 lm_head with leaf 256 this allows up to 742 rows per call.
+ *    151936 x 4096 lm_head with leaf 256 on a 148-SM B200 this allows up to
+ *    1251 rows per call.
  *  - Returns TBIK_ERR_ARG for any mode without TBIK_TC or with TBIK_EXACT.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call

@@ -54,17 +54,30 @@ def test_noalloc_logprob_matches_allocating_entry_point_on_two_calls():
         assert np.array_equal(u32(got), u32(ref))
 
 
+def _largest_fitting_rows(lib, V, H, T, leaf):
+    lo, hi = 1, 1 << 20
+    while lo < hi:  # largest M whose scratch fits the fixed array
+        mid = (lo + hi + 1) // 2
+        if lib.tbik_logprob_workspace(mid, V, H, T, leaf, tbik.TC) <= SCRATCH_BYTES:
+            lo = mid
+        else:
+            hi = mid - 1
+    return lo
+
+
 def test_noalloc_refuses_arguments_beyond_its_scratch():
     lib, noalloc = _entry()
     stream = torch.cuda.current_stream().cuda_stream
     V, H, leaf, T = 151936, 4096, 256, 8
-    assert lib.tbik_logprob_workspace(742, V, H, T, leaf, tbik.TC) <= SCRATCH_BYTES
-    assert lib.tbik_logprob_workspace(800, V, H, T, leaf, tbik.TC) > SCRATCH_BYTES
+    m_max = _largest_fitting_rows(lib, V, H, T, leaf)
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert m_max == 1251  # the limit stated in tbik.h for the 151936 x 4096 lm_head
+    big = m_max + 1
     # The size check comes before any pointer is used: small stand-in buffers.
     dummy = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
-    tg = torch.zeros(800, dtype=torch.int32, device="cuda")
-    out = torch.full((800,), float("nan"), dtype=torch.float32, device="cuda")
-    status = noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 800, V, H, T, leaf, tbik.TC,
+    tg = torch.zeros(big, dtype=torch.int32, device="cuda")
+    out = torch.full((big,), float("nan"), dtype=torch.float32, device="cuda")
+    status = noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), big, V, H, T, leaf, tbik.TC,
                      stream)
     assert status == tbik.TBIK_ERR_WORKSPACE
     assert noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 4, V, H, T, leaf, tbik.EXACT,
