@@ -123,26 +123,42 @@ __device__ __forceinline__ MS ms_combine(MS a, MS b) {
 
 // ------------------------------------------------------------- tree walk
 
-// Streaming (post-order) evaluation of TREE over n leaves: after leaf j arrives,
-// the nodes whose last leaf is j close, deepest first; each close adds the
-// pending result of that node's left child (size pop_size[i]).  The shallowest
-// closed node (or the leaf itself) is then pushed, unless it is the root.
+// Streaming (post-order) evaluation of TREE over n leaves.  After leaf j
+// arrives, the nodes whose last leaf is j close, deepest first; each close adds
+// the pending result of that node's left child.  The closing nodes form the
+// deepest part of j's root path, and their left children shrink with depth, so
+// the pending values with <= 2 leaves are popped first, then the larger ones.
+// The shallowest closed node (or the leaf itself) is then pushed, unless it is
+// the root.  Computed in registers only.
 struct LeafOps {
-    int npop;
-    int pop_size[24];
-    int push_size;
-    bool final_;
+    int ns;          // pops of pending subtrees with <= 2 leaves
+    int nm;          // pops of pending subtrees with 3..4 leaves (at most one)
+    int nb;          // pops of pending subtrees with >= 5 leaves
+    int push_size;   // leaves of the value left after the pops
+    bool final_;     // that value is the root of the tree over n leaves
 };
 
-__device__ __forceinline__ void leaf_ops(int n, int j, LeafOps& o) {
-    int lo = 0, sz = n, depth = 0;
-    int plo[24], psz[24], ph[24];
+__device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
+    LeafOps o;
+    o.ns = 0;
+    o.nm = 0;
+    o.nb = 0;
+    int lo = 0, sz = n, top = 1;
+    bool closing = false;
     while (sz > 1) {
-        int h = (sz + 1) >> 1;
-        plo[depth] = lo;
-        psz[depth] = sz;
-        ph[depth] = h;
-        ++depth;
+        const int h = (sz + 1) >> 1;
+        if (!closing && lo + sz - 1 == j) {
+            closing = true;
+            top = sz;
+        }
+        if (closing) {
+            if (h <= 2)
+                ++o.ns;
+            else if (h <= 4)
+                ++o.nm;
+            else
+                ++o.nb;
+        }
         if (j < lo + h) {
             sz = h;
         } else {
@@ -150,15 +166,9 @@ __device__ __forceinline__ void leaf_ops(int n, int j, LeafOps& o) {
             sz -= h;
         }
     }
-    o.npop = 0;
-    int top = 1;
-    for (int d = depth - 1; d >= 0; --d) {
-        if (plo[d] + psz[d] - 1 != j) break;
-        o.pop_size[o.npop++] = ph[d];
-        top = psz[d];
-    }
     o.push_size = top;
     o.final_ = (top == n);
+    return o;
 }
 
 // ------------------------------------------------------------ PTX: misc
@@ -167,10 +177,47 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ------------------------------------------------------ PTX: CTA pairs
+// Thread-block clusters of two CTAs run one 256-row MMA tile (cta_group::2):
+// rank 0 (the leader) issues the MMAs; each CTA holds its own 128 rows of A
+// and 64 of the 128 B rows/columns in shared memory at the same offsets.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Arrive once on an mbarrier anywhere in the cluster (default semantics; the
+// tcgen05 reads it publishes are ordered by tcgen05.fence::before_thread_sync).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+
 // ---------------------------------------------------------- PTX: mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Named hardware barrier over `count` threads (ids 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void fence_barrier_init() {
@@ -219,25 +266,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// Same contract for waits that are long and off the critical issue path (the
-// epilogue waiting for a whole leaf): between polls the warp sleeps, so it
-// does not compete with the tensor core for the shared-memory pipe.
-__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                                 uint64_t limit_cycles) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        __nanosleep(128);
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if ((uint64_t)(clock64() - t0) > limit_cycles) {
-            *abort_flag = 1;
-            set_error(TBIK_ERR_TIMEOUT);
-            return false;
-        }
-    }
-}
-
 // Bounded wait used on the way out: no abort check, only the cycle limit.
 __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_cycles) {
     const long long t0 = clock64();
@@ -251,6 +279,16 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint6
 }
 
 // --------------------------------------------------------------- PTX: TMA
+
+// Pair form: the copy lands in this CTA's shared memory and completes its bytes
+// on an mbarrier that may be in the peer CTA (cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tmap, uint32_t bar_cluster, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -267,6 +305,38 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
 }
 
 // ------------------------------------------------------------ PTX: tcgen05
+// (cta_group::2 forms: executed by one warp / thread per the PTX ISA rules;
+// alloc, relinquish and dealloc are collective over one warp of each CTA.)
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on the mbarrier at this offset in both CTAs of the pair when every
+// tcgen05 op issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),

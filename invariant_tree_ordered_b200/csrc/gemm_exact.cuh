@@ -114,9 +114,8 @@ __global__ void __launch_bounds__(EX_THREADS) gemm_exact_kernel(const __grid_con
                     for (int c = 0; c < 4; ++c) acc[i * 4 + c] = __fmaf_rn(a[i], b[c], acc[i * 4 + c]);
                 if (k0 + kk + 1 == next_b) {
                     // leaf j complete: apply the tree
-                    LeafOps ops;
-                    leaf_ops(n, j, ops);
-                    for (int i = 0; i < ops.npop; ++i) {
+                    const LeafOps ops = leaf_ops(n, j);
+                    for (int i = 0; i < ops.ns + ops.nm + ops.nb; ++i) {
                         --sp;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) acc[e] = __fadd_rn(stk[sp][e], acc[e]);

@@ -4,24 +4,30 @@
 // Sizes That Eliminates Training-Inference Mismatch" (TBIK summary page),
 // sections 核心思路 / 技术框架: the K reduction is one hierarchical binary
 // tree shared by the local and the cross-GPU steps.  Here each K leaf is a
-// chain of 128x128x16 bf16 MMAs into an fp32 TMEM accumulator that restarts
+// chain of 256x128x16 bf16 MMAs into an fp32 TMEM accumulator that restarts
 // from zero; the leaves are then combined by the halving tree in fp32 in the
 // epilogue.  The MMA sequence of a leaf depends only on the leaf's K range,
 // never on M, N or T, so a row's bits are the same for every batch size and
 // every shard count.
 //
-// CTA layout (320 threads, one CTA per SM, persistent over work units):
-//   warp 0     TMA producer: A and B k-blocks (64 deep) into a 6-stage ring
-//   warp 1     TMEM allocator + single-thread MMA issuer
+// CTA pairs (clusters of 2, cta_group::2): a pair computes a 256 x 128 tile;
+// CTA r holds rows [128r, 128r+128) of A and rows/columns [64r, 64r+64) of B
+// in its shared memory and its own 128 x 128 fp32 accumulators in TMEM.  The
+// leader (rank 0) issues the MMAs; commits arrive on both CTAs' barriers.
+// Each CTA (320 threads, one per SM, persistent over work units):
+//   warp 0     TMA producer: its A and B halves, 128 deep (two 64-wide
+//              128-byte-swizzle slices), into a 3-stage ring
+//   warp 1     TMEM allocator (both CTAs) + single-thread MMA issuer (leader)
 //   warps 2-9  epilogue: drain each leaf from TMEM and apply the tree; warp w
 //              reads TMEM lanes 32*(w%4).. (its row quadrant) and the 64
 //              columns of half (w-2)/4 of the tile
-// TMEM (512 columns x 128 lanes, fp32): columns [0,256) hold two leaf
-// accumulators (double buffer); [256,512) hold two pending subtree results of
-// size <= 2 leaves.  Pending subtrees of >= 3 leaves (written once per 3+
-// leaves) go to a per-CTA fp32 scratch in global memory that stays in L2.
+// Pending subtree results wait in one of three places by size: <= 2 leaves in
+// TMEM (columns [256,512): two slots; never more than two pending), 3-4 leaves
+// in one shared-memory slot (never more than one pending), >= 5 leaves in a
+// per-CTA fp32 scratch in global memory that stays in L2 (written once per 5+
+// leaves).
 // A work unit is (m tile, n tile, frontier node f): the node's subtree of
-// leaves is reduced by this CTA; with more than one frontier node per tile the
+// leaves is reduced by this pair; with more than one frontier node per tile the
 // subtree results go to fp32 partial buffers that a combine kernel reduces
 // with the upper levels of the same tree.
 #pragma once
@@ -30,18 +36,20 @@
 
 namespace tbik {
 
-constexpr int TC_BM = 128;
+constexpr int TC_BM = 128;        // rows per CTA
+constexpr int TC_PAIR_M = 256;    // rows per CTA pair (one MMA tile)
 constexpr int TC_BN = 128;
-constexpr int TC_BK = 64;
-constexpr int TC_STAGES = 6;
-constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;
-constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;
+constexpr int TC_BK = 128;  // two 64-wide swizzle slices per stage
+constexpr int TC_STAGES = 3;
+constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;        // this CTA's A rows
+constexpr int TC_B_BYTES = (TC_BN / 2) * TC_BK * 2;  // this CTA's half of B
 constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each owning 64 columns
 constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_MAX_F = 64;
 constexpr int TC_SLOT_FLOATS = TC_BM * TC_BN;
-constexpr size_t TC_SMEM_BYTES = (size_t)TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+constexpr size_t TC_SMEM_BYTES = (size_t)TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + TC_SLOT_FLOATS * 4 +
+                                 1024 /*align*/ + 256 /*barriers*/;
 
 enum { EPI_TREE = 0, EPI_LOGPROB = 1 };
 
@@ -56,7 +64,7 @@ struct TcParams {
     void* out;        // C [M,N]
     float* partials;  // [F][M][N]
     float* scratch;   // [gridDim.x][gs][128*128], layout per slot [col/4][row][4]
-    int gs;           // global stack slots per CTA
+    int gs;           // global stack slots per CTA (pending subtrees of >= 5 leaves)
     int b_mn;         // 1: B is [K,N] (MN-major operand)
     uint32_t b_lbo, b_sbo;
     // logprob epilogue
@@ -130,25 +138,28 @@ __device__ __forceinline__ void store_row32(void* out, int out_bf16, int M, int 
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* sA = smem;
     uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * TC_B_BYTES);
-    uint64_t* full = bars;                     // [STAGES] TMA landed
-    uint64_t* empty = bars + TC_STAGES;        // [STAGES] MMAs done reading
-    uint64_t* acc_full = bars + 2 * TC_STAGES; // [2] leaf accumulator ready
-    uint64_t* acc_empty = acc_full + 2;        // [2] leaf accumulator drained
-    uint64_t* done = acc_empty + 2;            // all MMAs retired
+    float* sSlot = reinterpret_cast<float*>(sB + TC_STAGES * TC_B_BYTES);  // pending 3-4 leaf subtree
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sSlot + TC_SLOT_FLOATS);
+    uint64_t* full = bars;                      // [STAGES] both CTAs' copies landed (leader's)
+    uint64_t* empty = bars + TC_STAGES;         // [STAGES] MMAs done reading (both CTAs)
+    uint64_t* acc_full = bars + 2 * TC_STAGES;  // [2] leaf accumulator ready (both CTAs)
+    uint64_t* acc_empty = acc_full + 2;         // [2] leaf accumulator drained by both CTAs (leader's)
+    uint64_t* done = acc_empty + 2;             // all MMAs retired (both CTAs)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint64_t wait_lim = p.wait_cycles;
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < TC_STAGES; ++s) {
@@ -157,100 +168,112 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 32 * TC_EPI_WARPS);
+            mbar_init(&acc_empty[b], 2 * TC_EPI_WARPS);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, TC_TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
             const bool b_mn = p.b_mn != 0;
             uint32_t q = 0;
-            for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+            for (int u = pair; u < p.total_units; u += npairs) {
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
                 const int k0 = p.lo[f] * p.leaf;
                 const int nkb = (p.nl[f] * p.leaf + TC_BK - 1) / TC_BK;
+                const int arow = tm * TC_PAIR_M + TC_BM * rank;
+                const int brow = tn * TC_BN + (TC_BN / 2) * rank;
                 for (int kb = 0; kb < nkb; ++kb) {
                     const int s = q % TC_STAGES;
                     if (!mbar_wait(&empty[s], ((q / TC_STAGES) & 1) ^ 1, abort_flag, wait_lim)) goto producer_out;
-                    mbar_arrive_expect_tx(&full[s], TC_A_BYTES + TC_B_BYTES);
+                    const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (TC_A_BYTES + TC_B_BYTES));
                     const int kx = k0 + kb * TC_BK;
-                    tma_load_2d(sA + s * TC_A_BYTES, &tmA, &full[s], kx, tm * TC_BM);
-                    if (!b_mn) {
-                        tma_load_2d(sB + s * TC_B_BYTES, &tmB, &full[s], kx, tn * TC_BN);
-                    } else {
-                        tma_load_2d(sB + s * TC_B_BYTES, &tmB, &full[s], tn * TC_BN, kx);
-                        tma_load_2d(sB + s * TC_B_BYTES + TC_B_BYTES / 2, &tmB, &full[s], tn * TC_BN + 64, kx);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tma_load_2d_pair(sA + s * TC_A_BYTES + h * (TC_A_BYTES / 2), &tmA, bar, kx + 64 * h, arow);
+                        if (!b_mn)
+                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / 2), &tmB, bar, kx + 64 * h, brow);
+                        else
+                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / 2), &tmB, bar, brow, kx + 64 * h);
                     }
                     ++q;
                 }
             }
         producer_out:
-            // Let the copies this thread issued land before the CTA can exit.
-            for (uint32_t i = (q > (uint32_t)TC_STAGES ? q - TC_STAGES : 0u); i < q; ++i)
-                mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_lim);
+            // The leader lets the copies of both CTAs land before the pair can exit.
+            if (rank == 0)
+                for (uint32_t i = (q > (uint32_t)TC_STAGES ? q - TC_STAGES : 0u); i < q; ++i)
+                    mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_lim);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        // One k-block (4 MMAs of K = 16) per ring stage.  Descriptors are built
-        // once per stage and advanced by adding the byte offset >> 4 to the
-        // start-address field, so the issue path per MMA is a few instructions.
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN, 0, p.b_mn);
+        // ------------------------------------------------ MMA issuer (leader)
+        // One 128-deep stage (8 MMAs of K = 16) per barrier round: the fixed cost
+        // of a round (wait, descriptors, commit) on this one thread is the
+        // throughput limit, so each round carries as many MMAs as fit.
+        // Descriptors are built once per stage and advanced by adding the byte
+        // offset >> 4 to the start-address field.
+        if (lane == 0 && rank == 0) {
+            const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, TC_BN, 0, p.b_mn);
             const bool b_mn = p.b_mn != 0;
             const uint32_t b_lbo = p.b_lbo, b_sbo = p.b_sbo;
             const uint32_t sA_u = smem_u32(sA), sB_u = smem_u32(sB);
             const int spl = p.leaf / 16;  // MMAs per leaf
             const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
-            const bool aligned = (spl % 4) == 0;  // leaf is a multiple of the 64-deep k-block
-            const int kb_per_leaf = spl / 4;
+            const bool aligned = (spl % 8) == 0;  // leaf is a multiple of the 128-deep stage
+            const int kb_per_leaf = spl / 8;
             uint32_t q = 0, a = 0;
-            for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+            for (int u = pair; u < p.total_units; u += npairs) {
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
                 const int nsteps = p.nl[f] * spl;
                 uint32_t buf = 0;
                 int in_leaf = 0, kb_in_leaf = 0;
-                for (int st = 0; st < nsteps; st += 4) {
+                for (int st = 0; st < nsteps; st += 8) {
                     const int s = q % TC_STAGES;
                     if (!mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_lim)) goto mma_out;
                     tc_fence_after();
                     const uint64_t adesc = smem_desc_sw128(sA_u + s * TC_A_BYTES, 16, 1024);
                     const uint64_t bdesc = b_mn ? smem_desc_sw128(sB_u + s * TC_B_BYTES, b_lbo, b_sbo)
                                                 : smem_desc_sw128(sB_u + s * TC_B_BYTES, 16, 1024);
+                    const uint64_t a2 = adesc + ((TC_A_BYTES / 2) >> 4), b2 = bdesc + ((TC_B_BYTES / 2) >> 4);
                     if (aligned) {
-                        // The leaf is a whole number of k-blocks: straight-line burst.
                         if (kb_in_leaf == 0) {
                             buf = a & 1;
                             if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_lim)) goto mma_out;
                             tc_fence_after();
                         }
                         const uint32_t d = tmem_base + buf * TC_BN;
-                        tc_mma(d, adesc, bdesc, idesc, kb_in_leaf != 0 ? 1u : 0u);
-                        tc_mma(d, adesc + 2, bdesc + b_step, idesc, 1u);
-                        tc_mma(d, adesc + 4, bdesc + 2 * b_step, idesc, 1u);
-                        tc_mma(d, adesc + 6, bdesc + 3 * b_step, idesc, 1u);
+                        tc_mma_pair(d, adesc, bdesc, idesc, kb_in_leaf != 0 ? 1u : 0u);
+                        tc_mma_pair(d, adesc + 2, bdesc + b_step, idesc, 1u);
+                        tc_mma_pair(d, adesc + 4, bdesc + 2 * b_step, idesc, 1u);
+                        tc_mma_pair(d, adesc + 6, bdesc + 3 * b_step, idesc, 1u);
+                        tc_mma_pair(d, a2, b2, idesc, 1u);
+                        tc_mma_pair(d, a2 + 2, b2 + b_step, idesc, 1u);
+                        tc_mma_pair(d, a2 + 4, b2 + 2 * b_step, idesc, 1u);
+                        tc_mma_pair(d, a2 + 6, b2 + 3 * b_step, idesc, 1u);
                         if (++kb_in_leaf == kb_per_leaf) {
-                            tc_commit(&acc_full[buf]);
+                            tc_commit_pair(&acc_full[buf]);
                             ++a;
                             kb_in_leaf = 0;
                         }
                     } else {
-                        const int nk = min(4, nsteps - st);
+                        const int nk = min(8, nsteps - st);
                         for (int ks = 0; ks < nk; ++ks) {
                             if (in_leaf == 0) {
                                 buf = a & 1;
@@ -258,50 +281,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                     goto mma_out;
                                 tc_fence_after();
                             }
-                            tc_mma(tmem_base + buf * TC_BN, adesc + (uint64_t)(ks * 2), bdesc + b_step * ks, idesc,
-                                   in_leaf != 0 ? 1u : 0u);
+                            const uint64_t ad = (ks < 4 ? adesc : a2) + (uint64_t)((ks & 3) * 2);
+                            const uint64_t bd = (ks < 4 ? bdesc : b2) + b_step * (ks & 3);
+                            tc_mma_pair(tmem_base + buf * TC_BN, ad, bd, idesc, in_leaf != 0 ? 1u : 0u);
                             if (++in_leaf == spl) {
-                                tc_commit(&acc_full[buf]);
+                                tc_commit_pair(&acc_full[buf]);
                                 ++a;
                                 in_leaf = 0;
                             }
                         }
                     }
-                    tc_commit(&empty[s]);
+                    tc_commit_pair(&empty[s]);
                     ++q;
                 }
             }
         mma_out:
-            // Every MMA issued by this thread retires before TMEM is released.
-            tc_commit(done);
-            mbar_drain(done, 0, wait_lim);
+            // Every MMA issued by this thread retires before TMEM is released (both CTAs).
+            tc_commit_pair(done);
         }
+        if (lane == 0) mbar_drain(done, 0, wait_lim);
     } else {
-        // ------------------------------------------------ epilogue
+        // ------------------------------------------------ epilogue (both CTAs)
         const int ew = warp & 3;           // TMEM lane quadrant = rows 32*ew .. 32*ew+31
         const int half = (warp - 2) >> 2;  // columns [64*half, 64*half+64)
-        const int rt = ew * 32 + lane;     // row within the tile
+        const int rt = ew * 32 + lane;     // row within this CTA's 128
         const uint32_t tl = tmem_base + ((uint32_t)(ew * 32) << 16);
         uint32_t a = 0;
-        for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
+        for (int u = pair; u < p.total_units; u += npairs) {
             int tm, tn, f;
             tc_decode(p, u, tm, tn, f);
             const int n = p.nl[f];
-            const int row = tm * TC_BM + rt;
+            const int row = tm * TC_PAIR_M + TC_BM * rank + rt;
             int tsp = 0, gsp = 0;  // pending subtrees in TMEM slots / in the global scratch
             for (int j = 0; j < n; ++j) {
                 const uint32_t buf = a & 1;
-                if (!mbar_wait_sleepy(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim)) goto epi_out;
+                // One warp polls the accumulator barrier; the other epilogue
+                // warps wait on a hardware barrier, so nothing else polls.
+                if (warp == 2) mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim);
+                named_barrier_sync(1, 32 * TC_EPI_WARPS);
+                if (*abort_flag) goto epi_out;
                 tc_fence_after();
-                __syncwarp();
-                LeafOps ops;
-                leaf_ops(n, j, ops);
-                // Pops come deepest first: the small subtrees (<= 2 leaves, TMEM
-                // slots) precede the large ones (global scratch).
-                int ns = 0;
-                while (ns < ops.npop && ops.pop_size[ns] <= 2) ++ns;
-                const int nb = ops.npop - ns;
-                const bool push_small = ops.push_size <= 2;
+                const LeafOps ops = leaf_ops(n, j);
+                const int ns = ops.ns, nm = ops.nm, nb = ops.nb;
+                const int cls = ops.push_size <= 2 ? 0 : (ops.push_size <= 4 ? 1 : 2);
                 const int t_after = tsp - ns, g_after = gsp - nb;
 #pragma unroll 1
                 for (int cc = 0; cc < 2; ++cc) {
@@ -324,6 +346,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                         for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r2[k]), v[k]);
                     }
+                    if (nm) {
+                        float w[32];
+                        scratch_ld(sSlot, c, rt, w);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(w[k], v[k]);
+                    }
                     for (int i = 0; i < nb; ++i) {
                         float w[32];
                         scratch_ld(scratch_slot(p, gsp - 1 - i), c, rt, w);
@@ -340,17 +368,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         } else {
                             tmem_st32_nowait(tl + 256 + c * 32, v);  // logits of this vocab leaf, slot 0
                         }
-                    } else if (push_small) {
+                    } else if (cls == 0) {
                         tmem_st32_nowait(tl + 256 + t_after * TC_BN + c * 32, v);
+                    } else if (cls == 1) {
+                        scratch_st(sSlot, c, rt, v);
                     } else {
                         scratch_st(scratch_slot(p, g_after), c, rt, v);
                     }
                 }
                 tmem_wait_st();
-                tsp = t_after + ((!ops.final_ && push_small) ? 1 : 0);
-                gsp = g_after + ((!ops.final_ && !push_small) ? 1 : 0);
+                tsp = t_after + ((!ops.final_ && cls == 0) ? 1 : 0);
+                gsp = g_after + ((!ops.final_ && cls == 2) ? 1 : 0);
                 tc_fence_before();
-                if (!(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) mbar_arrive(&acc_empty[buf]);
+                __syncwarp();
+                if (lane == 0 && !(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE))
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
                 ++a;
             }
             if (EPI == EPI_LOGPROB) {
@@ -403,11 +435,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     epi_out:;
     }
 
+    // A CTA that gave up tells its peer, so the peer's waits end too.
+    if (*abort_flag && threadIdx.x == 0) st_cluster_u32(mapa_shared(smem_u32((const void*)abort_flag), rank ^ 1), 1);
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TC_TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
     }
 }
 

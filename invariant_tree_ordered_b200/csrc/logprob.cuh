@@ -98,9 +98,8 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
             int sp = 0;
             for (int j = 0; j < n; ++j) {
                 MS cur = leaf_ms(stats, M, nvt, row, lo + j);
-                LeafOps ops;
-                leaf_ops(n, j, ops);
-                for (int i = 0; i < ops.npop; ++i) cur = ms_combine(stk[--sp], cur);
+                const LeafOps ops = leaf_ops(n, j);
+                for (int i = 0; i < ops.ns + ops.nm + ops.nb; ++i) cur = ms_combine(stk[--sp], cur);
                 if (!ops.final_) stk[sp++] = cur;
                 else v = cur;
             }

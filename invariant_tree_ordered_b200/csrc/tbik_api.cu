@@ -120,13 +120,13 @@ void frontier(int lo, int n, int D, std::vector<std::pair<int, int>>& out) {
     frontier(lo + h, n - h, D - 1, out);
 }
 
-// Largest number of simultaneously pending left subtrees of >= 3 leaves while
+// Largest number of simultaneously pending left subtrees of >= 5 leaves while
 // streaming the tree over n leaves (they live in the global scratch).
 int max_big_pending(int n) {
     if (n <= 1) return 0;
     int h = (n + 1) / 2;
     int l = max_big_pending(h);
-    int r = max_big_pending(n - h) + (h >= 3 ? 1 : 0);
+    int r = max_big_pending(n - h) + (h >= 5 ? 1 : 0);
     return l > r ? l : r;
 }
 int max_stack_depth(int n) {
@@ -161,7 +161,7 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
     p.M = M, p.N = N, p.K = K, p.T = T, p.leaf = leaf;
     p.L = K / leaf;
     if (p.L % T) return TBIK_ERR_SHAPE;
-    const int bm = tc ? TC_BM : EX_BM, bn = tc ? TC_BN : EX_BN;
+    const int bm = tc ? TC_PAIR_M : EX_BM, bn = tc ? TC_BN : EX_BN;
     if (tc) {
         if (N % 8 || K % 8) return TBIK_ERR_SHAPE;
         if (p.noninv ? (K / T) % 16 : leaf % 16) return TBIK_ERR_SHAPE;
@@ -181,7 +181,7 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
         int dmax = ilog2(p.L);
         if (dmax > 6) dmax = 6;
         if (tc ? false : (max_stack_depth(p.L) > EX_MAXD)) return TBIK_ERR_SHAPE;
-        const long long want = tc ? sms : 2LL * sms;
+        const long long want = tc ? sms / 2 : 2LL * sms;  // CTA pairs / CTAs
         int D = d0;
         while (D < dmax && tiles * (1LL << D) < want) ++D;
         p.D = D;
@@ -196,8 +196,13 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
     const long long units = tiles * p.F;
     if (units > 0x7fffffffLL) return TBIK_ERR_SHAPE;
     p.units = (int)units;
-    p.grid = p.units < sms ? p.units : sms;
-    if (p.grid < 1) p.grid = 1;
+    if (tc) {
+        const int pairs = p.units < sms / 2 ? p.units : sms / 2;
+        p.grid = 2 * (pairs > 0 ? pairs : 1);
+    } else {
+        p.grid = p.units < sms ? p.units : sms;
+        if (p.grid < 1) p.grid = 1;
+    }
     p.gs = 0;
     if (tc)
         for (auto& nd : p.nodes) {
@@ -280,9 +285,9 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
     if (p.M == 0) return TBIK_OK;
     if (p.tc) {
         CUtensorMap ta, tb;
-        if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, TC_BK, TC_BM)) return TBIK_ERR_CUDA;
-        bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, TC_BK, TC_BN)
-                          : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, 64, TC_BK);
+        if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, 64, TC_BM)) return TBIK_ERR_CUDA;
+        bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, 64, TC_BN / 2)
+                          : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, TC_BN / 2, 64);
         if (!okb) return TBIK_ERR_CUDA;
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
@@ -299,8 +304,8 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.gs = p.gs;
         prm.b_mn = p.b_nk ? 0 : 1;
         const bool swap = g_debug_flags & TBIK_DEBUG_SWAP_MN_STRIDES;
-        prm.b_lbo = swap ? 1024u : (uint32_t)(TC_B_BYTES / 2);
-        prm.b_sbo = swap ? (uint32_t)(TC_B_BYTES / 2) : 1024u;
+        prm.b_lbo = swap ? 1024u : (uint32_t)TC_B_BYTES;
+        prm.b_sbo = swap ? (uint32_t)TC_B_BYTES : 1024u;
         prm.debug = g_debug_flags;
         prm.wait_cycles = wait_cycles(info);
         for (int f = 0; f < p.F; ++f) {
@@ -362,12 +367,14 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
     p.nvt = (V + TC_BN - 1) / TC_BN;        // 128-column GEMM tiles (two vocab leaves each)
     p.Lk = H / leaf;
     if (p.Lk > 32767) return TBIK_ERR_SHAPE;
-    p.tiles_m = (M + TC_BM - 1) / TC_BM;
+    p.tiles_m = (M + TC_PAIR_M - 1) / TC_PAIR_M;
     const long long units = (long long)p.tiles_m * p.nvt;
     if (units > 0x7fffffffLL) return TBIK_ERR_SHAPE;
     p.units = (int)units;
-    p.grid = p.units < sms ? p.units : sms;
-    if (p.grid < 1) p.grid = 1;
+    {
+        const int pairs = p.units < sms / 2 ? p.units : sms / 2;
+        p.grid = 2 * (pairs > 0 ? pairs : 1);
+    }
     p.gs = (tc && !p.noninv) ? max_big_pending(p.Lk) : 0;
     size_t off = 0;
     p.off_stats = off;
@@ -560,8 +567,8 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
     float* shard = reinterpret_cast<float*>(w8 + p.off_shard);
     if (p.tc) {
         CUtensorMap ta, tb;
-        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, TC_BK, TC_BM)) return TBIK_ERR_CUDA;
-        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, TC_BK, TC_BN)) return TBIK_ERR_CUDA;
+        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, 64, TC_BM)) return TBIK_ERR_CUDA;
+        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, 64, TC_BN / 2)) return TBIK_ERR_CUDA;
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
         prm.M = M, prm.N = V, prm.K = H;
