@@ -117,6 +117,24 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+# ------------------------------------------------- multi-rank aggregation
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest `value` over all ranks (all-reduce MAX); the identity for one rank."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(ms_total_max: float, steps: int, world: int, tokens_per_rank: int = M_TOK) -> float:
+    """Weak scaling: every rank runs its own batch; the job's time is the slowest rank's."""
+    return world * tokens_per_rank * steps / (ms_total_max * 1e-3)
+
+
 # ------------------------------------------------------------- CPU oracle
 
 _ORACLE_INPUTS = {}
@@ -195,12 +213,6 @@ def run_tbik(args):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     def bf(a):
         return synth.as_torch_bf16(a)
@@ -279,7 +291,7 @@ def run_tbik(args):
     clk = clocks.stop()
     # dominant kernel: average duration of the logprob call inside the timed region
     lp_live_ms = float(np.mean([a.elapsed_time(b) for a, b in lp_ev]))
-    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, dev)
     status = tbik.get_error(stream)
     if status != tbik.TBIK_OK:
         raise RuntimeError(f"device error in timed region: {status}")
@@ -317,7 +329,7 @@ def run_tbik(args):
         e2e_step()
     e1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     # ---- overhead of the invariant path over the non-invariant baseline (T = 1)
     def avg_ms(fn, n=10):
@@ -353,7 +365,7 @@ def run_tbik(args):
     lp_ms = lp_live_ms
     achieved = LOGPROB_FLOP / (lp_ms * 1e-3) / 1e12
     ms_step = ms_total / args.steps
-    value = world * M_TOK * args.steps / (ms_total * 1e-3)
+    value = whole_job_tokens_per_s(ms_total, args.steps, world)
     gb = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9  # noqa: E731
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -380,7 +392,7 @@ def run_tbik(args):
                      "bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
                      "frac": achieved / pk["bf16_sus"], "traffic": None,
                      "peak_source": f"{pk['src']} bf16 sustained"},
-        "e2e": {"value": world * M_TOK * args.steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_tokens_per_s(e2e_ms, args.steps, world), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk,
