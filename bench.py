@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8"], default=None,
+                    help="run only one call of the path, `--steps` times, for ncu captures (no JSON line)")
+    ap.add_argument("--tokens", type=int, default=M_TOK, help="tokens per call in --profile-case")
     return ap.parse_args()
 
 
@@ -411,12 +414,48 @@ def run_tbik(args):
     return 0
 
 
+def run_profile_case(args):
+    """One call of the path, repeated: the launches an ncu capture selects from."""
+    import torch
+
+    import invariant_tree_ordered_b200 as tbik
+
+    dev = torch.device("cuda", 0)
+    M = args.tokens
+    if args.profile_case == "logprob":
+        h = synth.as_torch_bf16(synth.normal_bf16(30, (M, H))).to(dev)
+        w = synth.as_torch_bf16(synth.normal_bf16(31, (V, H), std=0.02)).to(dev)
+        t = torch.from_numpy(synth.uniform_int32(32, M, 0, V)).to(dev)
+        ws = torch.empty(tbik.logprob_workspace(M, V, H, 1, LEAF, tbik.TC), dtype=torch.uint8, device=dev)
+        out = torch.empty(M, dtype=torch.float32, device=dev)
+        call = lambda: tbik.logprob(h, w, t, T=1, leaf=LEAF, tc=True, out=out, workspace=ws)  # noqa: E731
+    else:
+        T = 8 if args.profile_case == "gemm-t8" else 1
+        std = 0.02 * np.sqrt(H)
+        g = synth.as_torch_bf16(synth.normal_bf16(11, (M, F), std=std)).to(dev)
+        u = synth.as_torch_bf16(synth.normal_bf16(12, (M, F), std=std)).to(dev)
+        a = tbik.rope_swiglu(g=g, u=u)[2]
+        b = synth.as_torch_bf16(synth.down_proj_weight(F, H, "kn")).to(dev)
+        mode = tbik.TC | tbik.OUT_BF16
+        ws = torch.empty(max(tbik.gemm_workspace(M, H, F, T, LEAF, mode), 256), dtype=torch.uint8, device=dev)
+        out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        call = lambda: tbik.gemm(a, b, T=T, leaf=LEAF, tc=True, out_bf16=True, out=out, workspace=ws)  # noqa: E731
+    for _ in range(args.steps):
+        call()
+    torch.cuda.synchronize()
+    status = tbik.get_error()
+    print(f"profile case {args.profile_case}: {args.steps} calls, status {status}", flush=True)
+    return 0 if status == tbik.TBIK_OK else 1
+
+
 def main():
     args = parse()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_case:
+        return run_profile_case(args)
     return run_tbik(args)
 
 

@@ -127,22 +127,20 @@ __device__ __forceinline__ MS ms_combine(MS a, MS b) {
 // arrives, the nodes whose last leaf is j close, deepest first; each close adds
 // the pending result of that node's left child.  The closing nodes form the
 // deepest part of j's root path, and their left children shrink with depth, so
-// the pending values with <= 2 leaves are popped first, then the larger ones.
-// The shallowest closed node (or the leaf itself) is then pushed, unless it is
-// the root.  Computed in registers only.
+// pending values are popped smallest first.  The shallowest closed node (or the
+// leaf itself) is then pushed, unless it is the root.  Pending values are
+// counted by size class: 1 leaf, 2 leaves, 3-4 leaves, >= 5 leaves (a pending
+// single leaf is always consumed by the very next leaf; at most one value of 2
+// and one of 3-4 leaves is ever pending).  Computed in registers only.
 struct LeafOps {
-    int ns;          // pops of pending subtrees with <= 2 leaves
-    int nm;          // pops of pending subtrees with 3..4 leaves (at most one)
-    int nb;          // pops of pending subtrees with >= 5 leaves
-    int push_size;   // leaves of the value left after the pops
-    bool final_;     // that value is the root of the tree over n leaves
+    int n1, n2, nm, nb;  // pops per size class (1, 2, 3-4, >= 5 leaves)
+    int push_size;       // leaves of the value left after the pops
+    bool final_;         // that value is the root of the tree over n leaves
 };
 
 __device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
     LeafOps o;
-    o.ns = 0;
-    o.nm = 0;
-    o.nb = 0;
+    o.n1 = o.n2 = o.nm = o.nb = 0;
     int lo = 0, sz = n, top = 1;
     bool closing = false;
     while (sz > 1) {
@@ -152,8 +150,10 @@ __device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
             top = sz;
         }
         if (closing) {
-            if (h <= 2)
-                ++o.ns;
+            if (h == 1)
+                ++o.n1;
+            else if (h == 2)
+                ++o.n2;
             else if (h <= 4)
                 ++o.nm;
             else
@@ -169,6 +169,22 @@ __device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
     o.push_size = top;
     o.final_ = (top == n);
     return o;
+}
+
+__device__ __forceinline__ int leaf_pops(const LeafOps& o) { return o.n1 + o.n2 + o.nm + o.nb; }
+
+// A leaf's operations packed in 16 bits, so a table built once per CTA replaces
+// the walk (which costs several hundred cycles of dependent branches):
+// bit 0 pop of a single leaf, bit 1 pop of a 2-leaf value, bit 2 pop of a 3-4
+// leaf value, bits 3-7 pops of >= 5 leaf values, bits 8-9 size class of the
+// pushed value (0: 1 leaf, 1: 2, 2: 3-4, 3: >= 5), bit 10 final.
+__device__ __forceinline__ uint16_t encode_leaf_ops(const LeafOps& o) {
+    const int cls = o.push_size == 1 ? 0 : (o.push_size == 2 ? 1 : (o.push_size <= 4 ? 2 : 3));
+    return (uint16_t)(o.n1 | (o.n2 << 1) | (o.nm << 2) | (o.nb << 3) | (cls << 8) | ((o.final_ ? 1 : 0) << 10));
+}
+
+__device__ __forceinline__ int code_pops(uint32_t code) {
+    return (code & 1) + ((code >> 1) & 1) + ((code >> 2) & 1) + ((code >> 3) & 31);
 }
 
 // ------------------------------------------------------------ PTX: misc

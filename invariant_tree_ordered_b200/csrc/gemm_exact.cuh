@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(EX_THREADS) gemm_exact_kernel(const __grid_con
                 if (k0 + kk + 1 == next_b) {
                     // leaf j complete: apply the tree
                     const LeafOps ops = leaf_ops(n, j);
-                    for (int i = 0; i < ops.ns + ops.nm + ops.nb; ++i) {
+                    for (int i = 0; i < leaf_pops(ops); ++i) {
                         --sp;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) acc[e] = __fadd_rn(stk[sp][e], acc[e]);

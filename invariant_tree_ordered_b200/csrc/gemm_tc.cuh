@@ -17,15 +17,23 @@
 // Each CTA (320 threads, one per SM, persistent over work units):
 //   warp 0     TMA producer: its A and B halves, 128 deep (two 64-wide
 //              128-byte-swizzle slices), into a 3-stage ring
-//   warp 1     TMEM allocator (both CTAs) + single-thread MMA issuer (leader)
+//   warp 1     TMEM allocator (both CTAs) + MMA issuer (leader, lane 0)
 //   warps 2-9  epilogue: drain each leaf from TMEM and apply the tree; warp w
 //              reads TMEM lanes 32*(w%4).. (its row quadrant) and the 64
 //              columns of half (w-2)/4 of the tile
-// Pending subtree results wait in one of three places by size: <= 2 leaves in
-// TMEM (columns [256,512): two slots; never more than two pending), 3-4 leaves
-// in one shared-memory slot (never more than one pending), >= 5 leaves in a
-// per-CTA fp32 scratch in global memory that stays in L2 (written once per 5+
-// leaves).
+//   warp 10    waiter (leader): performs every mbarrier wait the issuer needs
+//              (stage landed, accumulator drained), then meets the MMA warp on
+//              a named barrier.  A barrier wait in the issuing thread costs the
+//              tensor pipe a few hundred cycles even when the barrier is
+//              already complete; a named barrier between two warps costs
+//              nothing, so the issuer only issues MMAs and commits.
+// TMEM (512 columns): three leaf accumulators (columns 0, 128, 256), so the
+// epilogue has two leaf-times to drain one, and a slot at column 384.  Pending
+// subtree results wait by size: a single leaf stays in its own accumulator
+// (it is always consumed by the next leaf, which releases both buffers); 2
+// leaves in the TMEM slot; 3-4 leaves in one shared-memory slot; >= 5 leaves in
+// a per-CTA fp32 scratch in global memory that stays in L2.  At most one value
+// of each of the first three classes is pending at a time.
 // A work unit is (m tile, n tile, frontier node f): the node's subtree of
 // leaves is reduced by this pair; with more than one frontier node per tile the
 // subtree results go to fp32 partial buffers that a combine kernel reduces
@@ -39,17 +47,23 @@ namespace tbik {
 constexpr int TC_BM = 128;        // rows per CTA
 constexpr int TC_PAIR_M = 256;    // rows per CTA pair (one MMA tile)
 constexpr int TC_BN = 128;
-constexpr int TC_BK = 128;  // two 64-wide swizzle slices per stage
+constexpr int TC_BK = 128;                // K per ring stage
+constexpr int TC_KSLICES = TC_BK / 64;    // 64-wide (128-byte) swizzle slices per stage
+constexpr int TC_KSTEPS = TC_BK / 16;     // MMAs (K = 16) per stage
 constexpr int TC_STAGES = 3;
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;        // this CTA's A rows
 constexpr int TC_B_BYTES = (TC_BN / 2) * TC_BK * 2;  // this CTA's half of B
 constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each owning 64 columns
-constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
+constexpr int TC_WAITER_WARP = 2 + TC_EPI_WARPS;
+constexpr int TC_THREADS = 32 * (TC_WAITER_WARP + 1);
+constexpr int TC_BAR_EPI = 1;      // named barrier: the epilogue warps
+constexpr int TC_BAR_HANDOFF = 2;  // named barrier: waiter warp + MMA warp, lockstep
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_MAX_F = 64;
 constexpr int TC_SLOT_FLOATS = TC_BM * TC_BN;
+constexpr int TC_TAB_MAX = 1024;  // leaves per subtree covered by the shared-memory op table
 constexpr size_t TC_SMEM_BYTES = (size_t)TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + TC_SLOT_FLOATS * 4 +
-                                 1024 /*align*/ + 256 /*barriers*/;
+                                 2 * TC_TAB_MAX * 2 /*op tables*/ + 1024 /*align*/ + 256 /*barriers*/;
 
 enum { EPI_TREE = 0, EPI_LOGPROB = 1 };
 
@@ -74,6 +88,7 @@ struct TcParams {
     int V;
     unsigned debug;
     unsigned long long wait_cycles;  // bound of every device-side wait, in SM cycles
+    int tab_n[2];                    // the (at most two) subtree sizes of the frontier nodes
     short lo[TC_MAX_F];
     short nl[TC_MAX_F];
 };
@@ -146,14 +161,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
     float* sSlot = reinterpret_cast<float*>(sB + TC_STAGES * TC_B_BYTES);  // pending 3-4 leaf subtree
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sSlot + TC_SLOT_FLOATS);
+    uint16_t* leaf_tab = reinterpret_cast<uint16_t*>(sSlot + TC_SLOT_FLOATS);  // [2][TC_TAB_MAX]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(leaf_tab + 2 * TC_TAB_MAX);
     uint64_t* full = bars;                      // [STAGES] both CTAs' copies landed (leader's)
     uint64_t* empty = bars + TC_STAGES;         // [STAGES] MMAs done reading (both CTAs)
-    uint64_t* acc_full = bars + 2 * TC_STAGES;  // [2] leaf accumulator ready (both CTAs)
-    uint64_t* acc_empty = acc_full + 2;         // [2] leaf accumulator drained by both CTAs (leader's)
-    uint64_t* done = acc_empty + 2;             // all MMAs retired (both CTAs)
+    uint64_t* acc_full = bars + 2 * TC_STAGES;  // [3] leaf accumulator ready (both CTAs)
+    uint64_t* acc_empty = acc_full + 3;         // [3] leaf accumulator drained by both CTAs (leader's)
+    uint64_t* done = acc_empty + 3;             // all MMAs retired (both CTAs)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* handoff_go = abort_flag + 1;  // waiter's verdict for the step it hands off
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -166,7 +183,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < 3; ++b) {
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 2 * TC_EPI_WARPS);
         }
@@ -178,6 +195,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
         tmem_relinquish_pair();
     }
+    const bool use_tab = p.tab_n[0] <= TC_TAB_MAX && p.tab_n[1] <= TC_TAB_MAX;
+    if (use_tab)
+        for (int i = threadIdx.x; i < p.tab_n[0] + p.tab_n[1]; i += blockDim.x) {
+            const int t = i < p.tab_n[0] ? 0 : 1;
+            const int j = i - (t ? p.tab_n[0] : 0);
+            leaf_tab[t * TC_TAB_MAX + j] = encode_leaf_ops(leaf_ops(p.tab_n[t], j));
+        }
     tc_fence_before();
     __syncthreads();
     cluster_sync();
@@ -205,12 +229,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (TC_A_BYTES + TC_B_BYTES));
                     const int kx = k0 + kb * TC_BK;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_2d_pair(sA + s * TC_A_BYTES + h * (TC_A_BYTES / 2), &tmA, bar, kx + 64 * h, arow);
+                    for (int h = 0; h < TC_KSLICES; ++h) {
+                        tma_load_2d_pair(sA + s * TC_A_BYTES + h * (TC_A_BYTES / TC_KSLICES), &tmA, bar, kx + 64 * h,
+                                         arow);
                         if (!b_mn)
-                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / 2), &tmB, bar, kx + 64 * h, brow);
+                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar,
+                                             kx + 64 * h, brow);
                         else
-                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / 2), &tmB, bar, brow, kx + 64 * h);
+                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar, brow,
+                                             kx + 64 * h);
                     }
                     ++q;
                 }
@@ -221,85 +248,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 for (uint32_t i = (q > (uint32_t)TC_STAGES ? q - TC_STAGES : 0u); i < q; ++i)
                     mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_lim);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer (leader)
-        // One 128-deep stage (8 MMAs of K = 16) per barrier round: the fixed cost
-        // of a round (wait, descriptors, commit) on this one thread is the
-        // throughput limit, so each round carries as many MMAs as fit.
-        // Descriptors are built once per stage and advanced by adding the byte
-        // offset >> 4 to the start-address field.
-        if (lane == 0 && rank == 0) {
+    } else if (warp == 1 || warp == TC_WAITER_WARP) {
+        // ------------------------------------------------ MMA issuer + waiter (leader)
+        // Both warps walk the same sequence of k-steps.  A hand-off happens
+        // where the issuer needs a condition: a stage start (its copies landed)
+        // or a leaf start (its accumulator buffer drained).  The waiter checks
+        // the condition(s), stores its verdict, and both warps bar.sync; the
+        // issuer then reads the verdict, so the two always stop together.
+        // One 128-deep stage carries 8 MMAs of K = 16; descriptors are built
+        // once per stage and advanced through the start-address field.
+        const bool is_mma = warp == 1;
+        if (rank == 0) {
             const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, TC_BN, 0, p.b_mn);
             const bool b_mn = p.b_mn != 0;
             const uint32_t b_lbo = p.b_lbo, b_sbo = p.b_sbo;
             const uint32_t sA_u = smem_u32(sA), sB_u = smem_u32(sB);
             const int spl = p.leaf / 16;  // MMAs per leaf
             const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
-            const bool aligned = (spl % 8) == 0;  // leaf is a multiple of the 128-deep stage
-            const int kb_per_leaf = spl / 8;
+            const bool aligned = (spl % TC_KSTEPS) == 0;  // leaf is a whole number of stages
+            const int kb_per_leaf = spl / TC_KSTEPS;
             uint32_t q = 0, a = 0;
+            // The hand-off: waiter lane 0 waits (bounded) for what the issuer needs.
+            auto handoff = [&](bool need_full, bool need_acc, int s, uint32_t abuf, uint32_t acount) -> bool {
+                if (!is_mma) {
+                    if (lane == 0) {
+                        bool ok = true;
+                        if (need_full) ok = mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_lim);
+                        if (ok && need_acc)
+                            ok = mbar_wait(&acc_empty[abuf], ((acount / 3) & 1) ^ 1, abort_flag, wait_lim);
+                        *handoff_go = ok ? 1 : 0;
+                    }
+                    __syncwarp();
+                }
+                named_barrier_sync(TC_BAR_HANDOFF, 64);
+                const bool go = *handoff_go != 0;
+                if (is_mma) tc_fence_after();
+                return go;
+            };
             for (int u = pair; u < p.total_units; u += npairs) {
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
                 const int nsteps = p.nl[f] * spl;
                 uint32_t buf = 0;
                 int in_leaf = 0, kb_in_leaf = 0;
-                for (int st = 0; st < nsteps; st += 8) {
+                for (int st = 0; st < nsteps; st += TC_KSTEPS) {
                     const int s = q % TC_STAGES;
-                    if (!mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_lim)) goto mma_out;
-                    tc_fence_after();
                     const uint64_t adesc = smem_desc_sw128(sA_u + s * TC_A_BYTES, 16, 1024);
                     const uint64_t bdesc = b_mn ? smem_desc_sw128(sB_u + s * TC_B_BYTES, b_lbo, b_sbo)
                                                 : smem_desc_sw128(sB_u + s * TC_B_BYTES, 16, 1024);
-                    const uint64_t a2 = adesc + ((TC_A_BYTES / 2) >> 4), b2 = bdesc + ((TC_B_BYTES / 2) >> 4);
+                    // k-step ks: slice ks/4 (advance by a slice's bytes >> 4), step ks%4 within it
+                    auto a_at = [&](int ks) {
+                        return adesc + (uint64_t)((ks >> 2) * ((TC_A_BYTES / TC_KSLICES) >> 4) + (ks & 3) * 2);
+                    };
+                    auto b_at = [&](int ks) {
+                        return bdesc + (uint64_t)((ks >> 2) * ((TC_B_BYTES / TC_KSLICES) >> 4)) + b_step * (ks & 3);
+                    };
                     if (aligned) {
-                        if (kb_in_leaf == 0) {
-                            buf = a & 1;
-                            if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_lim)) goto mma_out;
-                            tc_fence_after();
+                        if (kb_in_leaf == 0) buf = a % 3;
+                        if (!handoff(true, kb_in_leaf == 0, s, buf, a)) goto mma_out;
+                        if (is_mma && lane == 0) {
+                            const uint32_t d = tmem_base + buf * TC_BN;
+                            tc_mma_pair(d, a_at(0), b_at(0), idesc, kb_in_leaf != 0 ? 1u : 0u);
+#pragma unroll
+                            for (int ks = 1; ks < TC_KSTEPS; ++ks) tc_mma_pair(d, a_at(ks), b_at(ks), idesc, 1u);
+                            if (kb_in_leaf + 1 == kb_per_leaf) tc_commit_pair(&acc_full[buf]);
                         }
-                        const uint32_t d = tmem_base + buf * TC_BN;
-                        tc_mma_pair(d, adesc, bdesc, idesc, kb_in_leaf != 0 ? 1u : 0u);
-                        tc_mma_pair(d, adesc + 2, bdesc + b_step, idesc, 1u);
-                        tc_mma_pair(d, adesc + 4, bdesc + 2 * b_step, idesc, 1u);
-                        tc_mma_pair(d, adesc + 6, bdesc + 3 * b_step, idesc, 1u);
-                        tc_mma_pair(d, a2, b2, idesc, 1u);
-                        tc_mma_pair(d, a2 + 2, b2 + b_step, idesc, 1u);
-                        tc_mma_pair(d, a2 + 4, b2 + 2 * b_step, idesc, 1u);
-                        tc_mma_pair(d, a2 + 6, b2 + 3 * b_step, idesc, 1u);
                         if (++kb_in_leaf == kb_per_leaf) {
-                            tc_commit_pair(&acc_full[buf]);
                             ++a;
                             kb_in_leaf = 0;
                         }
                     } else {
-                        const int nk = min(8, nsteps - st);
+                        const int nk = min(TC_KSTEPS, nsteps - st);
                         for (int ks = 0; ks < nk; ++ks) {
-                            if (in_leaf == 0) {
-                                buf = a & 1;
-                                if (!mbar_wait(&acc_empty[buf], ((a >> 1) & 1) ^ 1, abort_flag, wait_lim))
-                                    goto mma_out;
-                                tc_fence_after();
+                            if (in_leaf == 0) buf = a % 3;
+                            if (ks == 0 || in_leaf == 0)
+                                if (!handoff(ks == 0, in_leaf == 0, s, buf, a)) goto mma_out;
+                            if (is_mma && lane == 0) {
+                                tc_mma_pair(tmem_base + buf * TC_BN, a_at(ks), b_at(ks), idesc, in_leaf != 0 ? 1u : 0u);
+                                if (in_leaf + 1 == spl) tc_commit_pair(&acc_full[buf]);
                             }
-                            const uint64_t ad = (ks < 4 ? adesc : a2) + (uint64_t)((ks & 3) * 2);
-                            const uint64_t bd = (ks < 4 ? bdesc : b2) + b_step * (ks & 3);
-                            tc_mma_pair(tmem_base + buf * TC_BN, ad, bd, idesc, in_leaf != 0 ? 1u : 0u);
                             if (++in_leaf == spl) {
-                                tc_commit_pair(&acc_full[buf]);
                                 ++a;
                                 in_leaf = 0;
                             }
                         }
                     }
-                    tc_commit_pair(&empty[s]);
+                    if (is_mma && lane == 0) tc_commit_pair(&empty[s]);
+                    __syncwarp();
                     ++q;
                 }
             }
         mma_out:
             // Every MMA issued by this thread retires before TMEM is released (both CTAs).
-            tc_commit_pair(done);
+            if (is_mma && lane == 0) tc_commit_pair(done);
         }
-        if (lane == 0) mbar_drain(done, 0, wait_lim);
+        if (is_mma && lane == 0) mbar_drain(done, 0, wait_lim);
     } else {
         // ------------------------------------------------ epilogue (both CTAs)
         const int ew = warp & 3;           // TMEM lane quadrant = rows 32*ew .. 32*ew+31
@@ -312,41 +355,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             tc_decode(p, u, tm, tn, f);
             const int n = p.nl[f];
             const int row = tm * TC_PAIR_M + TC_BM * rank + rt;
-            int tsp = 0, gsp = 0;  // pending subtrees in TMEM slots / in the global scratch
+            const uint16_t* tab = leaf_tab + (n == p.tab_n[0] ? 0 : TC_TAB_MAX);
+            int gsp = 0;  // pending subtrees of >= 5 leaves in the global scratch
             for (int j = 0; j < n; ++j) {
-                const uint32_t buf = a & 1;
+                const uint32_t buf = a % 3;
+                const uint32_t prev = (a + 2) % 3;  // accumulator of leaf j-1 (a retained single leaf)
                 // One warp polls the accumulator barrier; the other epilogue
                 // warps wait on a hardware barrier, so nothing else polls.
-                if (warp == 2) mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim);
-                named_barrier_sync(1, 32 * TC_EPI_WARPS);
+                if (warp == 2) mbar_wait(&acc_full[buf], (a / 3) & 1, abort_flag, wait_lim);
+                named_barrier_sync(TC_BAR_EPI, 32 * TC_EPI_WARPS);
                 if (*abort_flag) goto epi_out;
                 tc_fence_after();
-                const LeafOps ops = leaf_ops(n, j);
-                const int ns = ops.ns, nm = ops.nm, nb = ops.nb;
-                const int cls = ops.push_size <= 2 ? 0 : (ops.push_size <= 4 ? 1 : 2);
-                const int t_after = tsp - ns, g_after = gsp - nb;
+                const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(leaf_ops(n, j));
+                const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
+                const int nb = (code >> 3) & 31;
+                const int cls = (code >> 8) & 3;
+                const bool final_ = (code >> 10) & 1;
+                const int g_after = gsp - nb;
 #pragma unroll 1
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = half * 2 + cc;
+                    if (!final_ && cls == 0) break;  // a single leaf waits in its accumulator
                     uint32_t r0[32], r1[32], r2[32];
                     tmem_ld32_nowait(tl + buf * TC_BN + c * 32, r0);
-                    if (ns >= 1) tmem_ld32_nowait(tl + 256 + (tsp - 1) * TC_BN + c * 32, r1);
-                    if (ns >= 2) tmem_ld32_nowait(tl + 256 + (tsp - 2) * TC_BN + c * 32, r2);
+                    if (p1) tmem_ld32_nowait(tl + prev * TC_BN + c * 32, r1);
+                    if (p2) tmem_ld32_nowait(tl + 384 + c * 32, r2);
                     tmem_wait_ld(r0);
                     float v[32];
 #pragma unroll
                     for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r0[k]);
-                    if (ns >= 1) {
+                    if (p1) {
                         tie32(r1);
 #pragma unroll
                         for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r1[k]), v[k]);
                     }
-                    if (ns >= 2) {
+                    if (p2) {
                         tie32(r2);
 #pragma unroll
                         for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r2[k]), v[k]);
                     }
-                    if (nm) {
+                    if (pm) {
                         float w[32];
                         scratch_ld(sSlot, c, rt, w);
 #pragma unroll
@@ -358,7 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                         for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(w[k], v[k]);
                     }
-                    if (ops.final_) {
+                    if (final_) {
                         if (EPI == EPI_TREE) {
                             if (p.direct)
                                 store_row32(p.out, p.out_bf16, p.M, p.N, row, tn * TC_BN + c * 32, v);
@@ -366,23 +414,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                                 store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row,
                                             tn * TC_BN + c * 32, v);
                         } else {
-                            tmem_st32_nowait(tl + 256 + c * 32, v);  // logits of this vocab leaf, slot 0
+                            tmem_st32_nowait(tl + 384 + c * 32, v);  // logits of this vocab leaf
                         }
-                    } else if (cls == 0) {
-                        tmem_st32_nowait(tl + 256 + t_after * TC_BN + c * 32, v);
                     } else if (cls == 1) {
+                        tmem_st32_nowait(tl + 384 + c * 32, v);
+                    } else if (cls == 2) {
                         scratch_st(sSlot, c, rt, v);
                     } else {
                         scratch_st(scratch_slot(p, g_after), c, rt, v);
                     }
                 }
                 tmem_wait_st();
-                tsp = t_after + ((!ops.final_ && cls == 0) ? 1 : 0);
-                gsp = g_after + ((!ops.final_ && cls == 2) ? 1 : 0);
+                gsp = g_after + ((!final_ && cls == 3) ? 1 : 0);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0 && !(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE))
-                    mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
+                if (lane == 0 && !(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) {
+                    // Release this leaf's accumulator unless it waits as a single
+                    // leaf; release the previous leaf's if it was consumed here.
+                    if (final_ || cls != 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
+                    if (p1) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[prev]), 0));
+                }
                 ++a;
             }
             if (EPI == EPI_LOGPROB) {
@@ -395,8 +446,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                     float z[64];
                     {
                         uint32_t r0[32], r1[32];
-                        tmem_ld32_nowait(tl + 256 + (half * 2) * 32, r0);
-                        tmem_ld32_nowait(tl + 256 + (half * 2 + 1) * 32, r1);
+                        tmem_ld32_nowait(tl + 384 + (half * 2) * 32, r0);
+                        tmem_ld32_nowait(tl + 384 + (half * 2 + 1) * 32, r1);
                         tmem_wait_ld(r0);
                         tie32(r1);
 #pragma unroll

@@ -72,14 +72,27 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
     logprob_row_kernel(const float* __restrict__ stats, const float* __restrict__ zt,
                        const int32_t* __restrict__ targets, float* __restrict__ out, float* shard_ms, int M, int V,
                        int nvt, int Lv, int T, int noninv) {
+    constexpr int TAB = 512;
+    __shared__ uint16_t tab[2][TAB];  // leaf operation codes for the two frontier subtree sizes
     const int lane = threadIdx.x & 31;
     const int row = blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+    int d = 0;
+    while (d < 5 && (2 << d) <= Lv) ++d;  // largest d <= 5 with 2^d <= Lv
+    const int nf = 1 << d;
+    // Nodes at depth d of the halving tree hold floor or ceil of Lv / 2^d leaves.
+    const int n_hi = (Lv + nf - 1) / nf, n_lo = Lv / nf;
+    const bool use_tab = !noninv && n_hi <= TAB;
+    if (use_tab) {
+        for (int i = threadIdx.x; i < n_hi + n_lo; i += blockDim.x) {
+            const int t = i < n_hi ? 0 : 1;
+            const int j = i - (t ? n_hi : 0);
+            tab[t][j] = encode_leaf_ops(leaf_ops(t ? n_lo : n_hi, j));
+        }
+    }
+    __syncthreads();
     if (row >= M) return;
     MS fin;
     if (!noninv) {
-        int d = 0;
-        while (d < 5 && (2 << d) <= Lv) ++d;  // largest d <= 5 with 2^d <= Lv
-        const int nf = 1 << d;
         MS v;
         v.m = -INFINITY;
         v.s = 0.0f;
@@ -96,11 +109,13 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
             }
             MS stk[24];
             int sp = 0;
+            const uint16_t* tb = tab[n == n_hi ? 0 : 1];
             for (int j = 0; j < n; ++j) {
                 MS cur = leaf_ms(stats, M, nvt, row, lo + j);
-                const LeafOps ops = leaf_ops(n, j);
-                for (int i = 0; i < ops.ns + ops.nm + ops.nb; ++i) cur = ms_combine(stk[--sp], cur);
-                if (!ops.final_) stk[sp++] = cur;
+                const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
+                const int npop = code_pops(code);
+                for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
+                if (!((code >> 10) & 1)) stk[sp++] = cur;
                 else v = cur;
             }
         }

@@ -308,9 +308,11 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.b_sbo = swap ? (uint32_t)TC_B_BYTES : 1024u;
         prm.debug = g_debug_flags;
         prm.wait_cycles = wait_cycles(info);
+        prm.tab_n[0] = prm.tab_n[1] = p.nodes[0].second;
         for (int f = 0; f < p.F; ++f) {
             prm.lo[f] = (short)p.nodes[f].first;
             prm.nl[f] = (short)p.nodes[f].second;
+            if (prm.nl[f] != prm.tab_n[0]) prm.tab_n[1] = prm.nl[f];
         }
         gemm_tc_kernel<EPI_TREE><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
     } else {
@@ -589,6 +591,7 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         prm.wait_cycles = wait_cycles(info);
         prm.lo[0] = 0;
         prm.nl[0] = (short)(p.noninv ? 1 : p.Lk);
+        prm.tab_n[0] = prm.tab_n[1] = prm.nl[0];
         gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
         if ((st = launch_status()) != TBIK_OK) return st;
     } else {
