@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -118,6 +119,39 @@ class ClockSampler:
             self._t.join()
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------- profile-backed traffic
+
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "logprob_tc_m4096.md")
+KERNEL_SOURCES = ["device_common.cuh", "gemm_tc.cuh", "logprob.cuh", "tbik_api.cu"]
+
+
+def kernel_source_hash() -> str:
+    """sha256 over the sources of the logprob kernels (changes invalidate old counters)."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "invariant_tree_ordered_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """DRAM bytes per logprob launch from the committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    try:
+        with open(TRAFFIC_PROFILE) as f:
+            text = f.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha256")):
+            k, v = line.strip().strip("`").split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != kernel_source_hash() or "traffic_bytes_per_launch" not in fields:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
 
 
 # ------------------------------------------------- multi-rank aggregation
@@ -286,10 +320,12 @@ def run_tbik(args):
     t1 = torch.cuda.Event(enable_timing=True)
     lp_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(args.steps)]
+    torch.cuda.nvtx.range_push("tbik_timed_steps")
     t0.record(stream)
     for i in range(args.steps):
         step(inp, lp_events=lp_ev[i])
     t1.record(stream)
+    torch.cuda.nvtx.range_pop()
     barrier()
     clk = clocks.stop()
     # dominant kernel: average duration of the logprob call inside the timed region
@@ -303,6 +339,10 @@ def run_tbik(args):
     comp = {k: [] for k in ev}
     barrier()
     for _ in range(min(args.steps, 20)):
+        # a ~0.5 ms device-side spin first, so the host has queued every launch
+        # of the step before its first kernel starts: the events then bracket
+        # kernel time only, not Python launch latency
+        torch.cuda._sleep(1_000_000)
         step(inp, timed=True)
         torch.cuda.synchronize()
         for k, (a, b) in ev.items():
@@ -393,7 +433,7 @@ def run_tbik(args):
         },
         "roofline": {"kernel": "tbik_logprob (fused tcgen05 GEMM + vocab stats, then row tree)",
                      "bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_sus"], "traffic": None,
+                     "frac": achieved / pk["bf16_sus"], "traffic": profiled_traffic(),
                      "peak_source": f"{pk['src']} bf16 sustained"},
         "e2e": {"value": whole_job_tokens_per_s(e2e_ms, args.steps, world), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},

@@ -195,7 +195,9 @@ TBIK_API size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, uns
  *   z[i,v]  = tree-ordered dot product over H (leaves of `leaf`, TREE over
  *             all H/leaf leaves), kept fp32;
  *   vocab leaf j = columns [64j, 64j+64) cut at V: m_j = max in ascending
- *             column order, s_j = sum in ascending order of exp(z - m_j);
+ *             column order, s_j = sum in ascending order of exp(z - m_j)
+ *             (TBIK_EXACT: the library's exp specification, bit-exact to the
+ *             definition; TBIK_TC: the hardware base-2 exponential, a few ulp);
  *   (m,s) combine: m = max(ma,mb); s = sa*exp(ma-m) + sb*exp(mb-m) (products
  *             rounded separately); identity (-inf, 0);
  *   shard t (of T) owns the vocab leaves [t*Lv/T, (t+1)*Lv/T) of the padded

@@ -66,6 +66,16 @@ __device__ __forceinline__ float exp_spec(float x) {
     return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));
 }
 
+// e^x through the hardware base-2 exponential (ex2.approx): x is scaled by the
+// nearest float to log2(e) first.  A few ulp from e^x; used where results are
+// compared by tolerance (the tensor-core logprob's per-leaf sums), never in
+// the exact-order path.
+__device__ __forceinline__ float exp_hw(float x) {
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(__fmul_rn(x, 0x1.715476p+0f)));
+    return y;
+}
+
 // log x for x > 0: x = 2^e * m, m in [sqrt(1/2), sqrt 2]; t = f/(2+f), f = m-1;
 // log m = s + s*w*(1/3 + w/5 + w^2/7 + w^3/9 + w^4/11), s = 2t, w = t^2;
 // result = e*ln2hi + (e*ln2lo + log m).

@@ -438,7 +438,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             }
             if (EPI == EPI_LOGPROB) {
                 // This warp's 64 columns are one vocab leaf: running max in
-                // ascending column order, then the ascending sum of exp(z - max).
+                // ascending column order, then the ascending sum of exp(z - max)
+                // (hardware exponential: this mode is checked by tolerance).
                 const int c0 = tn * TC_BN + half * 64;
                 const int vleaf = 2 * tn + half;
                 if (c0 < p.V) {
@@ -474,7 +475,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                     float s = 0.0f;
 #pragma unroll
                     for (int k = 0; k < 64; ++k)
-                        if (k < ncol) s = __fadd_rn(s, exp_spec(__fsub_rn(z[k], m)));
+                        if (k < ncol) s = __fadd_rn(s, exp_hw(__fsub_rn(z[k], m)));
                     if (row < p.M) {
                         *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
                         if (have_t) p.zt[row] = zval;

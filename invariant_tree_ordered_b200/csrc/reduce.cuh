@@ -34,14 +34,16 @@ __device__ __forceinline__ float pairwise_inplace(float* v, int n) {
     return v[0];
 }
 
-// One CTA per token, NT = H/8 threads; thread t owns leaf t = elements [8t, 8t+8).
-// The leaf sums form a power-of-two pairwise tree: xor-shuffle levels inside a
+// One CTA per token with NT = H/(8*LPT) threads; thread t owns the LPT
+// consecutive leaves [LPT*t, LPT*t + LPT) (leaf = 8 elements, one 16-byte
+// vector per tensor).  The leaf sums form a power-of-two pairwise tree: the
+// lowest log2(LPT) levels inside the thread, then xor-shuffle levels inside a
 // warp (both lanes of a pair add the same two values, and fp32 addition is
 // commutative, so they hold the same bits), then shared-memory levels.  With T
-// shards, shard t's partial (a whole subtree of NT/T leaves) is taken at its
+// shards, shard t's partial (a whole subtree of (H/8)/T leaves) is taken at its
 // own level, written to the shard buffer, and the T partials are combined by
-// the same tree.
-template <int NT>
+// the same tree.  All of a thread's loads are issued before any arithmetic.
+template <int NT, int LPT>
 __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ res,
                                                               const uint16_t* __restrict__ gamma, uint16_t* y,
@@ -51,20 +53,34 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
     __shared__ float ss_sh;
     const int tid = threadIdx.x;
     const size_t base = (size_t)blockIdx.x * H;
-    const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + base) + tid);
-    const uint4 rv = __ldg(reinterpret_cast<const uint4*>(res + base) + tid);
-    const uint4 gv = __ldg(reinterpret_cast<const uint4*>(gamma) + tid);
-    float xf[8], rf[8], gf[8], r[8];
-    unpack8(xv, xf);
-    unpack8(rv, rf);
-    unpack8(gv, gf);
-    float acc = 0.0f;
+    uint4 xv[LPT], rv[LPT], gv[LPT];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        r[e] = __fadd_rn(xf[e], rf[e]);
-        acc = __fmaf_rn(r[e], r[e], acc);
+    for (int l = 0; l < LPT; ++l) {
+        xv[l] = __ldg(reinterpret_cast<const uint4*>(x + base) + LPT * tid + l);
+        rv[l] = __ldg(reinterpret_cast<const uint4*>(res + base) + LPT * tid + l);
+        gv[l] = __ldg(reinterpret_cast<const uint4*>(gamma) + LPT * tid + l);
     }
-    const int S = NT / T;  // leaves per shard (power of two)
+    float r[LPT][8], leafsum[LPT];
+#pragma unroll
+    for (int l = 0; l < LPT; ++l) {
+        float xf[8], rf[8];
+        unpack8(xv[l], xf);
+        unpack8(rv[l], rf);
+        float acc = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            r[l][e] = __fadd_rn(xf[e], rf[e]);
+            acc = __fmaf_rn(r[l][e], r[l][e], acc);
+        }
+        leafsum[l] = acc;
+    }
+    // in-thread levels of the pairwise tree
+#pragma unroll
+    for (int w = 1; w < LPT; w <<= 1)
+#pragma unroll
+        for (int l = 0; l < LPT; l += 2 * w) leafsum[l] = __fadd_rn(leafsum[l], leafsum[l + w]);
+    float acc = leafsum[0];
+    const int S = NT / T;  // threads per shard (power of two)
     const int lim = S < 32 ? S : 32;
     for (int w = 1; w < lim; w <<= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, w));
     if (S <= 32) {
@@ -80,11 +96,15 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
     const float ss = ss_sh;
     const float ms = __fdiv_rn(ss, (float)H);
     const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
-    float o[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(__fmul_rn(r[e], inv), gf[e]);
-    reinterpret_cast<uint4*>(y + base)[tid] = pack8(o);
-    if (res_out) reinterpret_cast<uint4*>(res_out + base)[tid] = pack8(r);
+    for (int l = 0; l < LPT; ++l) {
+        float gf[8], o[8];
+        unpack8(gv[l], gf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(__fmul_rn(r[l][e], inv), gf[e]);
+        reinterpret_cast<uint4*>(y + base)[LPT * tid + l] = pack8(o);
+        if (res_out) reinterpret_cast<uint4*>(res_out + base)[LPT * tid + l] = pack8(r[l]);
+    }
 }
 
 // Rotate-half RoPE: thread = (tensor, token, head, group of 8 pairs).  Each
@@ -136,28 +156,43 @@ __device__ __forceinline__ float swiglu1(float g, float u) {
     return __fmul_rn(sg, u);
 }
 
-// out = bf16((g / (1 + exp(-g))) * u), 8 elements per thread.
+// out = bf16((g / (1 + exp(-g))) * u), two 8-element vectors per thread per
+// iteration with all loads issued before the arithmetic.
+template <int IN_F32>
+__device__ __forceinline__ void load8(const void* p, long long i, float (&f)[8]) {
+    if (IN_F32) {
+        const float4* q = reinterpret_cast<const float4*>(p) + 2 * i;
+        const float4 a = __ldg(q), b = __ldg(q + 1);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    } else {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(p) + i), f);
+    }
+}
+
 template <int IN_F32>
 __global__ void swiglu_kernel(const void* __restrict__ g, const void* __restrict__ u, uint16_t* out, long long n) {
     const long long nv = n >> 3;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nv;
-         i += (long long)gridDim.x * blockDim.x) {
-        float gf[8], uf[8], o[8];
-        if (IN_F32) {
-            const float4* gp = reinterpret_cast<const float4*>(g) + 2 * i;
-            const float4* up = reinterpret_cast<const float4*>(u) + 2 * i;
-            const float4 g0 = __ldg(gp), g1 = __ldg(gp + 1), u0 = __ldg(up), u1 = __ldg(up + 1);
-            gf[0] = g0.x; gf[1] = g0.y; gf[2] = g0.z; gf[3] = g0.w;
-            gf[4] = g1.x; gf[5] = g1.y; gf[6] = g1.z; gf[7] = g1.w;
-            uf[0] = u0.x; uf[1] = u0.y; uf[2] = u0.z; uf[3] = u0.w;
-            uf[4] = u1.x; uf[5] = u1.y; uf[6] = u1.z; uf[7] = u1.w;
-        } else {
-            unpack8(__ldg(reinterpret_cast<const uint4*>(g) + i), gf);
-            unpack8(__ldg(reinterpret_cast<const uint4*>(u) + i), uf);
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nv; i += 2 * stride) {
+        const long long i2 = i + stride;
+        const bool two = i2 < nv;
+        float g0[8], u0[8], g1[8], u1[8];
+        load8<IN_F32>(g, i, g0);
+        load8<IN_F32>(u, i, u0);
+        if (two) {
+            load8<IN_F32>(g, i2, g1);
+            load8<IN_F32>(u, i2, u1);
         }
+        float o[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = swiglu1(gf[e], uf[e]);
+        for (int e = 0; e < 8; ++e) o[e] = swiglu1(g0[e], u0[e]);
         reinterpret_cast<uint4*>(out)[i] = pack8(o);
+        if (two) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = swiglu1(g1[e], u1[e]);
+            reinterpret_cast<uint4*>(out)[i2] = pack8(o);
+        }
     }
 }
 

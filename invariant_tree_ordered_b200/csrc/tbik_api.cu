@@ -468,13 +468,15 @@ tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const 
     if (!aligned16(x) || !aligned16(res) || !aligned16(gamma) || !aligned16(y) || (res_out && !aligned16(res_out)))
         return TBIK_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // Four leaves (32 elements) per thread when the width allows it: more
+    // bytes in flight per thread; the tree is the same.
     switch (nt) {
-        case 32: rmsnorm_residual_kernel<32><<<tokens, 32, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 64: rmsnorm_residual_kernel<64><<<tokens, 64, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 128: rmsnorm_residual_kernel<128><<<tokens, 128, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 256: rmsnorm_residual_kernel<256><<<tokens, 256, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 512: rmsnorm_residual_kernel<512><<<tokens, 512, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 1024: rmsnorm_residual_kernel<1024><<<tokens, 1024, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 32: rmsnorm_residual_kernel<32, 1><<<tokens, 32, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 64: rmsnorm_residual_kernel<64, 1><<<tokens, 64, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 128: rmsnorm_residual_kernel<32, 4><<<tokens, 32, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 256: rmsnorm_residual_kernel<64, 4><<<tokens, 64, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 512: rmsnorm_residual_kernel<128, 4><<<tokens, 128, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 1024: rmsnorm_residual_kernel<256, 4><<<tokens, 256, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
     }
     return launch_status();
 }
@@ -528,8 +530,8 @@ tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) 
     }
     if (a->g && a->n > 0) {
         const long long nv = a->n / 8;
-        long long blocks = (nv + 255) / 256;
-        if (blocks > (long long)info->sms * 16) blocks = (long long)info->sms * 16;
+        long long blocks = (nv + 511) / 512;  // two vectors per thread
+        if (blocks > (long long)info->sms * 8) blocks = (long long)info->sms * 8;
         if (a->in_f32)
             swiglu_kernel<1><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
         else
