@@ -66,14 +66,15 @@ __device__ __forceinline__ float exp_spec(float x) {
     return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));
 }
 
-// e^x through the hardware base-2 exponential (ex2.approx): x is scaled by the
-// nearest float to log2(e) first.  A few ulp from e^x; used where results are
-// compared by tolerance (the tensor-core logprob's per-leaf sums), never in
-// the exact-order path.
-__device__ __forceinline__ float exp_hw(float x) {
-    float y;
-    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(__fmul_rn(x, 0x1.715476p+0f)));
-    return y;
+// 2^y through the hardware base-2 exponential (ex2.approx, denormal results
+// flushed to zero).  Used where results are compared by tolerance (the
+// tensor-core logprob's per-leaf sums of exp(z - max), whose terms are at
+// most 1 and whose sum is at least 1, so a flushed term below 2^-126 never
+// changes the sum), never in the exact-order path.
+__device__ __forceinline__ float ex2_hw(float y) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(y));
+    return r;
 }
 
 // log x for x > 0: x = 2^e * m, m in [sqrt(1/2), sqrt 2]; t = f/(2+f), f = m-1;

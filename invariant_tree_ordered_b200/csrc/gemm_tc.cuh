@@ -170,7 +170,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     uint64_t* done = acc_empty + 3;             // all MMAs retired (both CTAs)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* handoff_go = abort_flag + 1;  // waiter's verdict for the step it hands off
+    // Waiter's verdicts, two slots by hand-off parity: the waiter writes the
+    // verdict of hand-off h+1 only after hand-off h's barrier, and it reaches
+    // hand-off h+2 (same slot as h) only after the issuer has passed hand-off
+    // h+1's barrier, so the issuer always reads the verdict of its own step.
+    volatile int* handoff_go = abort_flag + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -267,21 +271,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
             const bool aligned = (spl % TC_KSTEPS) == 0;  // leaf is a whole number of stages
             const int kb_per_leaf = spl / TC_KSTEPS;
-            uint32_t q = 0, a = 0;
+            uint32_t q = 0, a = 0, hc = 0;
             // The hand-off: waiter lane 0 waits (bounded) for what the issuer needs.
             auto handoff = [&](bool need_full, bool need_acc, int s, uint32_t abuf, uint32_t acount) -> bool {
+                volatile int* verdict = handoff_go + (hc & 1);
+                ++hc;
                 if (!is_mma) {
                     if (lane == 0) {
                         bool ok = true;
                         if (need_full) ok = mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_lim);
                         if (ok && need_acc)
                             ok = mbar_wait(&acc_empty[abuf], ((acount / 3) & 1) ^ 1, abort_flag, wait_lim);
-                        *handoff_go = ok ? 1 : 0;
+                        *verdict = ok ? 1 : 0;
                     }
                     __syncwarp();
                 }
                 named_barrier_sync(TC_BAR_HANDOFF, 64);
-                const bool go = *handoff_go != 0;
+                const bool go = *verdict != 0;
                 if (is_mma) tc_fence_after();
                 return go;
             };
@@ -365,123 +371,145 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 if (warp == 2) mbar_wait(&acc_full[buf], (a / 3) & 1, abort_flag, wait_lim);
                 named_barrier_sync(TC_BAR_EPI, 32 * TC_EPI_WARPS);
                 if (*abort_flag) goto epi_out;
-                tc_fence_after();
+                ++a;
                 const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(leaf_ops(n, j));
                 const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
                 const int nb = (code >> 3) & 31;
                 const int cls = (code >> 8) & 3;
                 const bool final_ = (code >> 10) & 1;
-                const int g_after = gsp - nb;
-#pragma unroll 1
+                if (!final_ && cls == 0) continue;  // a single leaf waits in its accumulator
+                tc_fence_after();
+                // Phase 1: this leaf plus the single leaf it pops, into registers;
+                // both accumulators are released before any other tree work, so
+                // the MMA never waits on the pops and pushes below.
+                float v[2][32];
+#pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = half * 2 + cc;
-                    if (!final_ && cls == 0) break;  // a single leaf waits in its accumulator
-                    uint32_t r0[32], r1[32], r2[32];
+                    uint32_t r0[32], r1[32];
                     tmem_ld32_nowait(tl + buf * TC_BN + c * 32, r0);
                     if (p1) tmem_ld32_nowait(tl + prev * TC_BN + c * 32, r1);
-                    if (p2) tmem_ld32_nowait(tl + 384 + c * 32, r2);
                     tmem_wait_ld(r0);
-                    float v[32];
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(r0[k]);
                     if (p1) {
                         tie32(r1);
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r1[k]), v[k]);
-                    }
-                    if (p2) {
-                        tie32(r2);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(__uint_as_float(r2[k]), v[k]);
-                    }
-                    if (pm) {
-                        float w[32];
-                        scratch_ld(sSlot, c, rt, w);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(w[k], v[k]);
-                    }
-                    for (int i = 0; i < nb; ++i) {
-                        float w[32];
-                        scratch_ld(scratch_slot(p, gsp - 1 - i), c, rt, w);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) v[k] = __fadd_rn(w[k], v[k]);
-                    }
-                    if (final_) {
-                        if (EPI == EPI_TREE) {
-                            if (p.direct)
-                                store_row32(p.out, p.out_bf16, p.M, p.N, row, tn * TC_BN + c * 32, v);
-                            else
-                                store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row,
-                                            tn * TC_BN + c * 32, v);
-                        } else {
-                            tmem_st32_nowait(tl + 384 + c * 32, v);  // logits of this vocab leaf
-                        }
-                    } else if (cls == 1) {
-                        tmem_st32_nowait(tl + 384 + c * 32, v);
-                    } else if (cls == 2) {
-                        scratch_st(sSlot, c, rt, v);
+                        for (int k = 0; k < 32; ++k) v[cc][k] = __fadd_rn(__uint_as_float(r1[k]), __uint_as_float(r0[k]));
                     } else {
-                        scratch_st(scratch_slot(p, g_after), c, rt, v);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[cc][k] = __uint_as_float(r0[k]);
                     }
                 }
-                tmem_wait_st();
-                gsp = g_after + ((!final_ && cls == 3) ? 1 : 0);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0 && !(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) {
-                    // Release this leaf's accumulator unless it waits as a single
-                    // leaf; release the previous leaf's if it was consumed here.
-                    if (final_ || cls != 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
                     if (p1) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[prev]), 0));
                 }
-                ++a;
-            }
-            if (EPI == EPI_LOGPROB) {
-                // This warp's 64 columns are one vocab leaf: running max in
-                // ascending column order, then the ascending sum of exp(z - max)
-                // (hardware exponential: this mode is checked by tolerance).
-                const int c0 = tn * TC_BN + half * 64;
-                const int vleaf = 2 * tn + half;
-                if (c0 < p.V) {
-                    const int tgt = (row < p.M) ? p.targets[row] : -1;
-                    float z[64];
-                    {
-                        uint32_t r0[32], r1[32];
-                        tmem_ld32_nowait(tl + 384 + (half * 2) * 32, r0);
-                        tmem_ld32_nowait(tl + 384 + (half * 2 + 1) * 32, r1);
-                        tmem_wait_ld(r0);
-                        tie32(r1);
+                // Phase 2: the other pops, deepest (smallest) first, both chunks
+                // at once, then the push of the result (or the output).
+                if (p2) {
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) {
-                            z[k] = __uint_as_float(r0[k]);
-                            z[32 + k] = __uint_as_float(r1[k]);
-                        }
-                    }
-                    const int ncol = min(64, p.V - c0);
-                    float m = z[0];
-                    float zval = 0.0f;
-                    bool have_t = (tgt == c0);
-                    if (have_t) zval = z[0];
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t r2[32];
+                        tmem_ld32_nowait(tl + 384 + (half * 2 + cc) * 32, r2);
+                        tmem_wait_ld(r2);
 #pragma unroll
-                    for (int k = 1; k < 64; ++k) {
-                        if (k < ncol) {
-                            if (z[k] > m) m = z[k];
-                            if (c0 + k == tgt) {
-                                zval = z[k];
-                                have_t = true;
-                            }
-                        }
-                    }
-                    float s = 0.0f;
-#pragma unroll
-                    for (int k = 0; k < 64; ++k)
-                        if (k < ncol) s = __fadd_rn(s, exp_hw(__fsub_rn(z[k], m)));
-                    if (row < p.M) {
-                        *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
-                        if (have_t) p.zt[row] = zval;
+                        for (int k = 0; k < 32; ++k) v[cc][k] = __fadd_rn(__uint_as_float(r2[k]), v[cc][k]);
                     }
                 }
-                __syncwarp();
+                if (pm) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float w[32];
+                        scratch_ld(sSlot, half * 2 + cc, rt, w);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[cc][k] = __fadd_rn(w[k], v[cc][k]);
+                    }
+                }
+                for (int i = 0; i < nb; ++i) {
+                    const float* sl = scratch_slot(p, gsp - 1 - i);
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float w[32];
+                        scratch_ld(sl, half * 2 + cc, rt, w);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) v[cc][k] = __fadd_rn(w[k], v[cc][k]);
+                    }
+                }
+                const int g_after = gsp - nb;
+                gsp = g_after + ((!final_ && cls == 3) ? 1 : 0);
+                if (!final_) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = half * 2 + cc;
+                        if (cls == 1)
+                            tmem_st32_nowait(tl + 384 + c * 32, v[cc]);
+                        else if (cls == 2)
+                            scratch_st(sSlot, c, rt, v[cc]);
+                        else
+                            scratch_st(scratch_slot(p, g_after), c, rt, v[cc]);
+                    }
+                    if (cls == 1) tmem_wait_st();
+                } else if (EPI == EPI_TREE) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int col = tn * TC_BN + (half * 2 + cc) * 32;
+                        if (p.direct)
+                            store_row32(p.out, p.out_bf16, p.M, p.N, row, col, v[cc]);
+                        else
+                            store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row, col, v[cc]);
+                    }
+                } else {
+                    // Logprob: this warp's 64 columns are one vocab leaf.  The
+                    // max, then the sum of exp(z - max) = 2^(z*log2e - max*log2e)
+                    // as two interleaved partial sums (even and odd columns, each
+                    // ascending) added at the end.  Hardware exponential: this
+                    // mode is checked by tolerance; the order is fixed, so the
+                    // bits are the same for every T and M.
+                    const int c0 = tn * TC_BN + half * 64;
+                    const int vleaf = 2 * tn + half;
+                    if (c0 < p.V) {
+                        const int tgt = (row < p.M) ? p.targets[row] : -1;
+                        const int ncol = min(64, p.V - c0);
+                        const int kt = tgt - c0;  // target column within this leaf
+                        const bool have_t = (unsigned)kt < (unsigned)ncol;
+                        float zval = 0.0f;
+                        if (have_t) {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) {
+                                if (k == kt) zval = v[0][k];
+                                if (k + 32 == kt) zval = v[1][k];
+                            }
+                        }
+                        if (ncol < 64) {  // the last vocab leaf: columns past V add nothing
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) {
+                                if (k >= ncol) v[0][k] = -INFINITY;
+                                if (k + 32 >= ncol) v[1][k] = -INFINITY;
+                            }
+                        }
+                        float m = v[0][0];
+#pragma unroll
+                        for (int k = 1; k < 32; ++k) m = fmaxf(m, v[0][k]);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) m = fmaxf(m, v[1][k]);
+                        const float log2e = 0x1.715476p+0f;
+                        const float ml = -__fmul_rn(m, log2e);
+                        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                            for (int k = 0; k < 32; k += 2) {
+                                s0 = __fadd_rn(s0, ex2_hw(__fmaf_rn(v[cc][k], log2e, ml)));
+                                s1 = __fadd_rn(s1, ex2_hw(__fmaf_rn(v[cc][k + 1], log2e, ml)));
+                            }
+                        const float s = __fadd_rn(s0, s1);
+                        if (row < p.M) {
+                            *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
+                            if (have_t) p.zt[row] = zval;
+                        }
+                    }
+                }
             }
         }
     epi_out:;
