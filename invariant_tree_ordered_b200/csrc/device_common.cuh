@@ -30,8 +30,10 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
     return *reinterpret_cast<uint16_t*>(&b);
 }
 
+// Two values in one instruction (cvt.rn.bf16x2.f32): the same rounding as f2bf.
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
-    return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&b);
 }
 
 // ----------------------------------------------------- exp / log specs
@@ -45,11 +47,18 @@ __device__ __forceinline__ float pow2i(int n) { return __uint_as_float((uint32_t
 // e^x: clamp to [-104, 89]; k = rint(x*log2e); r = (x - k*ln2hi) - k*ln2lo;
 // degree-7 Taylor polynomial of e^r (coefficients: nearest floats to 1/n!);
 // scale by 2^(k/2) exactly, then by 2^(k-k/2) (one rounding).
+// Instruction choices that keep those bits: rint of y = x*log2e (|y| < 151)
+// is (y + 1.5*2^23) - 1.5*2^23 in round-to-nearest-even, and the integer k
+// sits in the low bits of that sum; when 2^k is a normal float (k in
+// [-126, 127]) the product p*2^k is rounded once, exactly as the two-step
+// scaling rounds it (its first step, by 2^(k/2), is exact).
 __device__ __forceinline__ float exp_spec(float x) {
     if (x != x) return __fadd_rn(x, x);
     x = fminf(fmaxf(x, -104.0f), 89.0f);
     const float log2e = 0x1.715476p+0f, ln2hi = 0x1.62e4p-1f, ln2lo = 0x1.7f7d1cp-20f;
-    float kf = rintf(__fmul_rn(x, log2e));
+    const float t = __fadd_rn(__fmul_rn(x, log2e), 0x1.8p23f);
+    const float kf = __fsub_rn(t, 0x1.8p23f);
+    const int k = __float_as_int(t) - 0x4b400000;
     float r = __fmaf_rn(-kf, ln2hi, x);
     r = __fmaf_rn(-kf, ln2lo, r);
     float p = 0x1.a01a02p-13f;
@@ -60,9 +69,9 @@ __device__ __forceinline__ float exp_spec(float x) {
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
-    int k = (int)kf;
-    int k1 = k / 2;
-    int k2 = k - k1;
+    if (k >= -126 && k <= 127) return __fmul_rn(p, pow2i(k));
+    const int k1 = k / 2;
+    const int k2 = k - k1;
     return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));
 }
 

@@ -27,102 +27,118 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
     return w;
 }
 
-// Pairwise (power-of-two) tree over v[0..n) in place; returns v[0].
-__device__ __forceinline__ float pairwise_inplace(float* v, int n) {
-    for (int w = 1; w < n; w <<= 1)
-        for (int i = 0; i < n; i += 2 * w) v[i] = __fadd_rn(v[i], v[i + w]);
-    return v[0];
-}
-
-// One CTA per token with NT = H/(8*LPT) threads; thread t owns the LPT
-// consecutive leaves [LPT*t, LPT*t + LPT) (leaf = 8 elements, one 16-byte
-// vector per tensor).  The leaf sums form a power-of-two pairwise tree: the
-// lowest log2(LPT) levels inside the thread, then xor-shuffle levels inside a
-// warp (both lanes of a pair add the same two values, and fp32 addition is
-// commutative, so they hold the same bits), then shared-memory levels.  With T
-// shards, shard t's partial (a whole subtree of (H/8)/T leaves) is taken at its
-// own level, written to the shard buffer, and the T partials are combined by
-// the same tree.  All of a thread's loads are issued before any arithmetic.
+// NT = H/(8*LPT) threads per token; thread t owns the LPT consecutive leaves
+// [LPT*t, LPT*t + LPT) (leaf = 8 elements, one 16-byte vector per tensor).
+// The leaf sums form a power-of-two pairwise tree: the lowest log2(LPT)
+// levels inside the thread, then xor-shuffle levels inside groups of
+// L = min(NT/T, 32) lanes (both lanes of a pair add the same two values, and
+// fp32 addition is commutative, so they hold the same bits), then the
+// remaining levels over the NT/L group values through shared memory.  With T
+// shards each shard (a whole subtree of (H/8)/T leaves) ends at or above the
+// group level, so these are the same levels as a per-shard tree followed by
+// the tree over the T shard partials.  A CTA loops over tokens and loads the
+// next token while it reduces and writes the current one; gamma is loaded once.
 template <int NT, int LPT>
 __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ res,
                                                               const uint16_t* __restrict__ gamma, uint16_t* y,
-                                                              uint16_t* res_out, int H, float eps, int T) {
-    __shared__ float warp_part[NT / 32 > 0 ? NT / 32 : 1];
-    __shared__ float shard[8];
-    __shared__ float ss_sh;
+                                                              uint16_t* res_out, int tokens, int H, float eps,
+                                                              int T) {
+    __shared__ float part[2][32];
     const int tid = threadIdx.x;
-    const size_t base = (size_t)blockIdx.x * H;
-    uint4 xv[LPT], rv[LPT], gv[LPT];
+    int t = blockIdx.x;
+    if (t >= tokens) return;
+    const int S = NT / T;            // threads per shard (a power of two)
+    const int L = S < 32 ? S : 32;   // lanes per shuffle group
+    const int G = NT / L;            // group values combined through shared memory
+    uint4 gv[LPT], xv[LPT], rv[LPT];
 #pragma unroll
     for (int l = 0; l < LPT; ++l) {
-        xv[l] = __ldg(reinterpret_cast<const uint4*>(x + base) + LPT * tid + l);
-        rv[l] = __ldg(reinterpret_cast<const uint4*>(res + base) + LPT * tid + l);
         gv[l] = __ldg(reinterpret_cast<const uint4*>(gamma) + LPT * tid + l);
+        xv[l] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H) + LPT * tid + l);
+        rv[l] = __ldg(reinterpret_cast<const uint4*>(res + (size_t)t * H) + LPT * tid + l);
     }
-    float r[LPT][8], leafsum[LPT];
+    for (int it = 0;; ++it) {
+        const int tn = t + gridDim.x;
+        const bool more = tn < tokens;
+        uint4 xn[LPT], rn[LPT];
+        if (more) {
 #pragma unroll
-    for (int l = 0; l < LPT; ++l) {
-        float xf[8], rf[8];
-        unpack8(xv[l], xf);
-        unpack8(rv[l], rf);
-        float acc = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            r[l][e] = __fadd_rn(xf[e], rf[e]);
-            acc = __fmaf_rn(r[l][e], r[l][e], acc);
+            for (int l = 0; l < LPT; ++l) {
+                xn[l] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)tn * H) + LPT * tid + l);
+                rn[l] = __ldg(reinterpret_cast<const uint4*>(res + (size_t)tn * H) + LPT * tid + l);
+            }
         }
-        leafsum[l] = acc;
-    }
-    // in-thread levels of the pairwise tree
+        float leafsum[LPT];
 #pragma unroll
-    for (int w = 1; w < LPT; w <<= 1)
+        for (int l = 0; l < LPT; ++l) {
+            float xf[8], rf[8];
+            unpack8(xv[l], xf);
+            unpack8(rv[l], rf);
+            float acc = 0.0f;
 #pragma unroll
-        for (int l = 0; l < LPT; l += 2 * w) leafsum[l] = __fadd_rn(leafsum[l], leafsum[l + w]);
-    float acc = leafsum[0];
-    const int S = NT / T;  // threads per shard (power of two)
-    const int lim = S < 32 ? S : 32;
-    for (int w = 1; w < lim; w <<= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, w));
-    if (S <= 32) {
-        if ((tid % S) == 0) shard[tid / S] = acc;
-    } else {
-        if ((tid & 31) == 0) warp_part[tid >> 5] = acc;
+            for (int e = 0; e < 8; ++e) {
+                const float r = __fadd_rn(xf[e], rf[e]);
+                acc = __fmaf_rn(r, r, acc);
+            }
+            leafsum[l] = acc;
+        }
+#pragma unroll
+        for (int w = 1; w < LPT; w <<= 1)
+#pragma unroll
+            for (int l = 0; l < LPT; l += 2 * w) leafsum[l] = __fadd_rn(leafsum[l], leafsum[l + w]);
+        float acc = leafsum[0];
+        for (int w = 1; w < L; w <<= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, w));
+        if ((tid % L) == 0) part[it & 1][tid / L] = acc;
         __syncthreads();
-        if (tid < T) shard[tid] = pairwise_inplace(&warp_part[tid * (S / 32)], S / 32);
-    }
-    __syncthreads();
-    if (tid == 0) ss_sh = pairwise_inplace(shard, T);
-    __syncthreads();
-    const float ss = ss_sh;
-    const float ms = __fdiv_rn(ss, (float)H);
-    const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+        // every warp applies the remaining levels to the G group values itself
+        float pv = (tid & 31) < G ? part[it & 1][tid & 31] : 0.0f;
+        for (int w = 1; w < G; w <<= 1) pv = __fadd_rn(pv, __shfl_xor_sync(0xffffffffu, pv, w));
+        const float ss = __shfl_sync(0xffffffffu, pv, 0);
+        const float ms = __fdiv_rn(ss, (float)H);
+        const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 #pragma unroll
-    for (int l = 0; l < LPT; ++l) {
-        float gf[8], o[8];
-        unpack8(gv[l], gf);
+        for (int l = 0; l < LPT; ++l) {
+            float xf[8], rf[8], gf[8], r[8], o[8];
+            unpack8(xv[l], xf);
+            unpack8(rv[l], rf);
+            unpack8(gv[l], gf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(__fmul_rn(r[l][e], inv), gf[e]);
-        reinterpret_cast<uint4*>(y + base)[LPT * tid + l] = pack8(o);
-        if (res_out) reinterpret_cast<uint4*>(res_out + base)[LPT * tid + l] = pack8(r[l]);
+            for (int e = 0; e < 8; ++e) {
+                r[e] = __fadd_rn(xf[e], rf[e]);
+                o[e] = __fmul_rn(__fmul_rn(r[e], inv), gf[e]);
+            }
+            reinterpret_cast<uint4*>(y + (size_t)t * H)[LPT * tid + l] = pack8(o);
+            if (res_out) reinterpret_cast<uint4*>(res_out + (size_t)t * H)[LPT * tid + l] = pack8(r);
+        }
+        if (!more) break;
+        t = tn;
+#pragma unroll
+        for (int l = 0; l < LPT; ++l) {
+            xv[l] = xn[l];
+            rv[l] = rn[l];
+        }
     }
 }
 
-// Rotate-half RoPE: thread = (tensor, token, head, group of 8 pairs).  Each
-// product is rounded on its own (no fma), then one bf16 rounding.
+// Rotate-half RoPE: thread = (tensor, token, head, group of 8 pairs), grid-
+// stride loop; item indices in IDX (32-bit when they fit, for cheap division).
+// Each product is rounded on its own (no fma), then one bf16 rounding.
+template <typename IDX>
 __global__ void rope_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, uint16_t* q_out,
                             uint16_t* k_out, const int32_t* __restrict__ pos, const float* __restrict__ table,
                             int tokens, int heads, int head_dim, int max_pos) {
     const uint16_t* x = blockIdx.y == 0 ? q : k;
     uint16_t* o = blockIdx.y == 0 ? q_out : k_out;
     if (x == nullptr) return;
-    const int half = head_dim >> 1;
-    const int gph = half >> 3;
-    const size_t total = (size_t)tokens * heads * gph;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const int g = (int)(i % gph);
-        const size_t th = i / gph;
-        const int token = (int)(th / heads);
-        const size_t hb = th * head_dim;
+    const IDX half = (IDX)(head_dim >> 1);
+    const IDX gph = half >> 3;
+    const IDX total = (IDX)tokens * (IDX)heads * gph;
+    for (IDX i = blockIdx.x * (IDX)blockDim.x + threadIdx.x; i < total; i += (IDX)gridDim.x * blockDim.x) {
+        const IDX th = i / gph;
+        const int g = (int)(i - th * gph);
+        const int token = (int)(th / (IDX)heads);
+        const size_t hb = (size_t)th * head_dim;
         const int p = __ldg(pos + token);
         float x1[8], x2[8], o1[8], o2[8];
         unpack8(__ldg(reinterpret_cast<const uint4*>(x + hb + 8 * g)), x1);
@@ -156,17 +172,41 @@ __device__ __forceinline__ float swiglu1(float g, float u) {
     return __fmul_rn(sg, u);
 }
 
-// out = bf16((g / (1 + exp(-g))) * u), two 8-element vectors per thread per
-// iteration with all loads issued before the arithmetic.
+// out = bf16((g / (1 + exp(-g))) * u), one 8-element vector per thread per
+// iteration of a grid-stride loop; the next iteration's inputs are loaded
+// before this one's arithmetic, so loads stay in flight during the (ALU-heavy)
+// exp and division.
 template <int IN_F32>
-__device__ __forceinline__ void load8(const void* p, long long i, float (&f)[8]) {
-    if (IN_F32) {
+struct Vec8;
+template <>
+struct Vec8<0> {
+    uint4 a;
+};
+template <>
+struct Vec8<1> {
+    float4 a, b;
+};
+
+template <int IN_F32>
+__device__ __forceinline__ Vec8<IN_F32> load_vec8(const void* p, long long i) {
+    Vec8<IN_F32> r;
+    if constexpr (IN_F32) {
         const float4* q = reinterpret_cast<const float4*>(p) + 2 * i;
-        const float4 a = __ldg(q), b = __ldg(q + 1);
-        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        r.a = __ldg(q);
+        r.b = __ldg(q + 1);
     } else {
-        unpack8(__ldg(reinterpret_cast<const uint4*>(p) + i), f);
+        r.a = __ldg(reinterpret_cast<const uint4*>(p) + i);
+    }
+    return r;
+}
+
+template <int IN_F32>
+__device__ __forceinline__ void unpack_vec8(const Vec8<IN_F32>& r, float (&f)[8]) {
+    if constexpr (IN_F32) {
+        f[0] = r.a.x, f[1] = r.a.y, f[2] = r.a.z, f[3] = r.a.w;
+        f[4] = r.b.x, f[5] = r.b.y, f[6] = r.b.z, f[7] = r.b.w;
+    } else {
+        unpack8(r.a, f);
     }
 }
 
@@ -174,25 +214,27 @@ template <int IN_F32>
 __global__ void swiglu_kernel(const void* __restrict__ g, const void* __restrict__ u, uint16_t* out, long long n) {
     const long long nv = n >> 3;
     const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < nv; i += 2 * stride) {
-        const long long i2 = i + stride;
-        const bool two = i2 < nv;
-        float g0[8], u0[8], g1[8], u1[8];
-        load8<IN_F32>(g, i, g0);
-        load8<IN_F32>(u, i, u0);
-        if (two) {
-            load8<IN_F32>(g, i2, g1);
-            load8<IN_F32>(u, i2, u1);
+    long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (i >= nv) return;
+    Vec8<IN_F32> cg = load_vec8<IN_F32>(g, i), cu = load_vec8<IN_F32>(u, i);
+    while (true) {
+        const long long inext = i + stride;
+        const bool more = inext < nv;
+        Vec8<IN_F32> ng, nu;
+        if (more) {
+            ng = load_vec8<IN_F32>(g, inext);
+            nu = load_vec8<IN_F32>(u, inext);
         }
-        float o[8];
+        float gf[8], uf[8], o[8];
+        unpack_vec8<IN_F32>(cg, gf);
+        unpack_vec8<IN_F32>(cu, uf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = swiglu1(g0[e], u0[e]);
+        for (int e = 0; e < 8; ++e) o[e] = swiglu1(gf[e], uf[e]);
         reinterpret_cast<uint4*>(out)[i] = pack8(o);
-        if (two) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[e] = swiglu1(g1[e], u1[e]);
-            reinterpret_cast<uint4*>(out)[i2] = pack8(o);
-        }
+        if (!more) break;
+        i = inext;
+        cg = ng;
+        cu = nu;
     }
 }
 

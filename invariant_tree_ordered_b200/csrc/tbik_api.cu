@@ -100,6 +100,36 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 
 // ------------------------------------------------------------- tree plan
 
+// Grid for a kernel that loops over work items (tokens): as many CTAs as are
+// resident on the device at once, at most one per item.
+template <typename Kernel, typename... Args>
+void launch_token_loop(Kernel kernel, int threads, int items, const DeviceInfo* info, cudaStream_t s, Args... args) {
+    // resident CTAs per SM, looked up once per (kernel, device)
+    struct Entry {
+        const void* fn;
+        int dev, per_sm;
+    };
+    static Entry cache[64];
+    static int used = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int per_sm = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].fn == reinterpret_cast<const void*>(kernel) && cache[i].dev == dev) per_sm = cache[i].per_sm;
+    }
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (used < 64) cache[used++] = Entry{reinterpret_cast<const void*>(kernel), dev, per_sm};
+    }
+    const long long resident = (long long)per_sm * info->sms;
+    const int grid = (int)(items < resident ? items : resident);
+    kernel<<<grid, threads, 0, s>>>(args...);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 int ilog2(int x) {
@@ -471,12 +501,12 @@ tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const 
     // Four leaves (32 elements) per thread when the width allows it: more
     // bytes in flight per thread; the tree is the same.
     switch (nt) {
-        case 32: rmsnorm_residual_kernel<32, 1><<<tokens, 32, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 64: rmsnorm_residual_kernel<64, 1><<<tokens, 64, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 128: rmsnorm_residual_kernel<32, 4><<<tokens, 32, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 256: rmsnorm_residual_kernel<64, 4><<<tokens, 64, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 512: rmsnorm_residual_kernel<128, 4><<<tokens, 128, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
-        case 1024: rmsnorm_residual_kernel<256, 4><<<tokens, 256, 0, s>>>(x, res, gamma, y, res_out, H, eps, T); break;
+        case 32: launch_token_loop(rmsnorm_residual_kernel<32, 1>, 32, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 64: launch_token_loop(rmsnorm_residual_kernel<64, 1>, 64, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 128: launch_token_loop(rmsnorm_residual_kernel<32, 4>, 32, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 256: launch_token_loop(rmsnorm_residual_kernel<64, 4>, 64, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 512: launch_token_loop(rmsnorm_residual_kernel<128, 4>, 128, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 1024: launch_token_loop(rmsnorm_residual_kernel<256, 4>, 256, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
     }
     return launch_status();
 }
@@ -524,14 +554,19 @@ tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) 
         const size_t work = (size_t)a->tokens * a->heads * (a->head_dim / 16);
         int blocks = (int)((work + 255) / 256);
         if (blocks > info->sms * 16) blocks = info->sms * 16;
-        rope_kernel<<<dim3(blocks, 2), 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table, a->tokens,
-                                                    a->heads, a->head_dim, a->max_pos);
+        const size_t stride = (size_t)blocks * 256;
+        if (work + stride < (1ull << 32))  // every index the loop forms fits 32 bits
+            rope_kernel<uint32_t><<<dim3(blocks, 2), 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table,
+                                                                  a->tokens, a->heads, a->head_dim, a->max_pos);
+        else
+            rope_kernel<size_t><<<dim3(blocks, 2), 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table,
+                                                                a->tokens, a->heads, a->head_dim, a->max_pos);
         if ((st = launch_status()) != TBIK_OK) return st;
     }
     if (a->g && a->n > 0) {
         const long long nv = a->n / 8;
-        long long blocks = (nv + 511) / 512;  // two vectors per thread
-        if (blocks > (long long)info->sms * 8) blocks = (long long)info->sms * 8;
+        long long blocks = (nv + 255) / 256;
+        if (blocks > (long long)info->sms * 16) blocks = (long long)info->sms * 16;
         if (a->in_f32)
             swiglu_kernel<1><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
         else

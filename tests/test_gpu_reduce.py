@@ -14,7 +14,7 @@ from tests.gpu_util import dev_bf16, dev_f32, dev_i32, host_bits16, host_f32  # 
 import invariant_tree_ordered_b200 as tbik  # noqa: E402
 
 
-@pytest.mark.parametrize("tokens", [1, 16, 128, 1024])
+@pytest.mark.parametrize("tokens", [1, 16, 128, 1024, 3000])  # 3000: CTAs loop over several tokens
 def test_rmsnorm_bitwise_all_T(tokens):
     d = synth.reduction_inputs(tokens, F=8)
     y_ref, r_ref = oracle.rmsnorm_residual(d["x"], d["res"], d["gamma"], eps=1e-6)
