@@ -77,7 +77,9 @@ typedef enum {
                             fixed by the hardware and identical for every T and M. */
 /* Deliberately non-invariant baseline (with EXACT or TC): each shard
    accumulates its whole K range in one chain and the shard partials are summed
-   left to right, ((Q0+Q1)+Q2)+...; logprob also combines leaves left to right. */
+   left to right, ((Q0+Q1)+Q2)+...  In tbik_logprob this applies to the lm_head
+   logits (H split into T shards, requires H % T == 0, and (H/T) % 16 == 0 in
+   TC mode); the vocabulary reduction stays the tree. */
 #define TBIK_NONINV 0x4u
 /* Layout of B in tbik_gemm (row-major in both cases): */
 #define TBIK_B_KN 0x00u  /* B is [K,N] (N contiguous) */

@@ -191,6 +191,24 @@ __device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
     return o;
 }
 
+// The same operations for the left-to-right chain ((L0 + L1) + L2) + ... of
+// the non-invariant baseline: leaf j > 0 pops the running sum of j leaves.
+__device__ __forceinline__ LeafOps seq_leaf_ops(int n, int j) {
+    LeafOps o;
+    o.n1 = o.n2 = o.nm = o.nb = 0;
+    if (j == 1)
+        o.n1 = 1;
+    else if (j == 2)
+        o.n2 = 1;
+    else if (j == 3 || j == 4)
+        o.nm = 1;
+    else if (j >= 5)
+        o.nb = 1;
+    o.push_size = j + 1;
+    o.final_ = (j == n - 1);
+    return o;
+}
+
 __device__ __forceinline__ int leaf_pops(const LeafOps& o) { return o.n1 + o.n2 + o.nm + o.nb; }
 
 // A leaf's operations packed in 16 bits, so a table built once per CTA replaces

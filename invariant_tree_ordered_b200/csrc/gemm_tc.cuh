@@ -88,6 +88,7 @@ struct TcParams {
     int V;
     unsigned debug;
     unsigned long long wait_cycles;  // bound of every device-side wait, in SM cycles
+    int seq;                         // 1: the leaves form the left-to-right chain, not the tree
     int tab_n[2];                    // the (at most two) subtree sizes of the frontier nodes
     short lo[TC_MAX_F];
     short nl[TC_MAX_F];
@@ -204,7 +205,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         for (int i = threadIdx.x; i < p.tab_n[0] + p.tab_n[1]; i += blockDim.x) {
             const int t = i < p.tab_n[0] ? 0 : 1;
             const int j = i - (t ? p.tab_n[0] : 0);
-            leaf_tab[t * TC_TAB_MAX + j] = encode_leaf_ops(leaf_ops(p.tab_n[t], j));
+            leaf_tab[t * TC_TAB_MAX + j] = encode_leaf_ops(p.seq ? seq_leaf_ops(p.tab_n[t], j) : leaf_ops(p.tab_n[t], j));
         }
     tc_fence_before();
     __syncthreads();
@@ -372,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 named_barrier_sync(TC_BAR_EPI, 32 * TC_EPI_WARPS);
                 if (*abort_flag) goto epi_out;
                 ++a;
-                const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(leaf_ops(n, j));
+                const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(p.seq ? seq_leaf_ops(n, j) : leaf_ops(n, j));
                 const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
                 const int nb = (code >> 3) & 31;
                 const int cls = (code >> 8) & 3;

@@ -71,7 +71,7 @@ constexpr int ROW_WARPS = 8;
 __global__ void __launch_bounds__(ROW_WARPS * 32)
     logprob_row_kernel(const float* __restrict__ stats, const float* __restrict__ zt,
                        const int32_t* __restrict__ targets, float* __restrict__ out, float* shard_ms, int M, int V,
-                       int nvt, int Lv, int T, int noninv) {
+                       int nvt, int Lv, int T) {
     constexpr int TAB = 512;
     __shared__ uint16_t tab[2][TAB];  // leaf operation codes for the two frontier subtree sizes
     const int lane = threadIdx.x & 31;
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
     const int nf = 1 << d;
     // Nodes at depth d of the halving tree hold floor or ceil of Lv / 2^d leaves.
     const int n_hi = (Lv + nf - 1) / nf, n_lo = Lv / nf;
-    const bool use_tab = !noninv && n_hi <= TAB;
+    const bool use_tab = n_hi <= TAB;
     if (use_tab) {
         for (int i = threadIdx.x; i < n_hi + n_lo; i += blockDim.x) {
             const int t = i < n_hi ? 0 : 1;
@@ -91,75 +91,50 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
     }
     __syncthreads();
     if (row >= M) return;
-    MS fin;
-    if (!noninv) {
-        MS v;
-        v.m = -INFINITY;
-        v.s = 0.0f;
-        if (lane < nf) {
-            int lo = 0, n = Lv;
-            for (int lvl = 0; lvl < d; ++lvl) {
-                const int h = (n + 1) >> 1;
-                if ((lane >> (d - 1 - lvl)) & 1) {
-                    lo += h;
-                    n -= h;
-                } else {
-                    n = h;
-                }
-            }
-            MS stk[24];
-            int sp = 0;
-            const uint16_t* tb = tab[n == n_hi ? 0 : 1];
-            for (int j = 0; j < n; ++j) {
-                MS cur = leaf_ms(stats, M, nvt, row, lo + j);
-                const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
-                const int npop = code_pops(code);
-                for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
-                if (!((code >> 10) & 1)) stk[sp++] = cur;
-                else v = cur;
+    // Each shard's vocab leaves by the tree: the frontier subtrees in
+    // lanes, then butterflies inside each shard's lanes.
+    MS v;
+    v.m = -INFINITY;
+    v.s = 0.0f;
+    if (lane < nf) {
+        int lo = 0, n = Lv;
+        for (int lvl = 0; lvl < d; ++lvl) {
+            const int h = (n + 1) >> 1;
+            if ((lane >> (d - 1 - lvl)) & 1) {
+                lo += h;
+                n -= h;
+            } else {
+                n = h;
             }
         }
-        const int sl = nf / T;  // lanes per shard
-        for (int w = 1; w < sl; w <<= 1) v = butterfly_ms(v, lane, w);
-        if (lane < nf && (lane % sl) == 0)
-            *reinterpret_cast<float2*>(shard_ms + ((size_t)(lane / sl) * M + row) * 2) = make_float2(v.m, v.s);
-        __syncwarp();
-        MS sv;
-        sv.m = -INFINITY;
-        sv.s = 0.0f;
-        if (lane < T) {
-            const float2 t2 = *reinterpret_cast<const float2*>(shard_ms + ((size_t)lane * M + row) * 2);
-            sv.m = t2.x;
-            sv.s = t2.y;
+        MS stk[24];
+        int sp = 0;
+        const uint16_t* tb = tab[n == n_hi ? 0 : 1];
+        for (int j = 0; j < n; ++j) {
+            MS cur = leaf_ms(stats, M, nvt, row, lo + j);
+            const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
+            const int npop = code_pops(code);
+            for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
+            if (!((code >> 10) & 1)) stk[sp++] = cur;
+            else v = cur;
         }
-        for (int w = 1; w < T; w <<= 1) sv = butterfly_ms(sv, lane, w);
-        fin = sv;
-    } else {
-        // Non-invariant baseline: left-to-right inside each shard, then across shards.
-        const int Ls = Lv / T;
-        MS sv;
-        sv.m = -INFINITY;
-        sv.s = 0.0f;
-        if (lane < T) {
-            sv = leaf_ms(stats, M, nvt, row, lane * Ls);
-            for (int j = 1; j < Ls; ++j) sv = ms_combine(sv, leaf_ms(stats, M, nvt, row, lane * Ls + j));
-            *reinterpret_cast<float2*>(shard_ms + ((size_t)lane * M + row) * 2) = make_float2(sv.m, sv.s);
-        }
-        __syncwarp();
-        if (lane == 0) {
-            const float2 t0 = *reinterpret_cast<const float2*>(shard_ms + (size_t)row * 2);
-            sv.m = t0.x;
-            sv.s = t0.y;
-            for (int t = 1; t < T; ++t) {
-                const float2 tt = *reinterpret_cast<const float2*>(shard_ms + ((size_t)t * M + row) * 2);
-                MS b;
-                b.m = tt.x;
-                b.s = tt.y;
-                sv = ms_combine(sv, b);
-            }
-        }
-        fin = sv;
     }
+    const int sl = nf / T;  // lanes per shard
+    for (int w = 1; w < sl; w <<= 1) v = butterfly_ms(v, lane, w);
+    if (lane < nf && (lane % sl) == 0)
+        *reinterpret_cast<float2*>(shard_ms + ((size_t)(lane / sl) * M + row) * 2) = make_float2(v.m, v.s);
+    __syncwarp();
+    // The T shard partials (the emulated cross-GPU exchange), by the same tree.
+    MS sv;
+    sv.m = -INFINITY;
+    sv.s = 0.0f;
+    if (lane < T) {
+        const float2 t2 = *reinterpret_cast<const float2*>(shard_ms + ((size_t)lane * M + row) * 2);
+        sv.m = t2.x;
+        sv.s = t2.y;
+    }
+    for (int w = 1; w < T; w <<= 1) sv = butterfly_ms(sv, lane, w);
+    const MS fin = sv;
     if (lane == 0) {
         const int t = targets[row];
         if (t < 0 || t >= V) {

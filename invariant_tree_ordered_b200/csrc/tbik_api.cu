@@ -383,6 +383,12 @@ struct LogprobPlan {
     GemmPlan zplan;  // exact mode: the logits GEMM
 };
 
+tbik_status zgemm_plan(const LogprobPlan& p, int sms, GemmPlan& z) {
+    const int M = p.M > 0 ? p.M : 1;
+    if (p.noninv) return plan_gemm(M, p.V, p.H, p.T, p.H / p.T, TBIK_EXACT | TBIK_B_NK | TBIK_NONINV, sms, z);
+    return plan_gemm(M, p.V, p.H, 1, p.leaf, TBIK_EXACT | TBIK_B_NK, sms, z);
+}
+
 tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, int sms, LogprobPlan& p) {
     if (mode & ~(TBIK_EXACT | TBIK_TC | TBIK_NONINV)) return TBIK_ERR_ARG;
     const bool exact = mode & TBIK_EXACT, tc = mode & TBIK_TC;
@@ -397,7 +403,9 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
     p.Lv = p.Vpad / VLEAF;
     p.nvl = (V + VLEAF - 1) / VLEAF;        // vocab leaves holding columns
     p.nvt = (V + TC_BN - 1) / TC_BN;        // 128-column GEMM tiles (two vocab leaves each)
-    p.Lk = H / leaf;
+    // The baseline's logits: T chains over H/T each, summed left to right.
+    if (p.noninv && (H % T || (tc && (H / T) % 16))) return TBIK_ERR_SHAPE;
+    p.Lk = p.noninv ? T : H / leaf;
     if (p.Lk > 32767) return TBIK_ERR_SHAPE;
     p.tiles_m = (M + TC_PAIR_M - 1) / TC_PAIR_M;
     const long long units = (long long)p.tiles_m * p.nvt;
@@ -407,7 +415,8 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
         const int pairs = p.units < sms / 2 ? p.units : sms / 2;
         p.grid = 2 * (pairs > 0 ? pairs : 1);
     }
-    p.gs = (tc && !p.noninv) ? max_big_pending(p.Lk) : 0;
+    // pending results of >= 5 leaves: the tree's depth, or one for the chain
+    p.gs = tc ? (p.noninv ? (p.Lk >= 6 ? 1 : 0) : max_big_pending(p.Lk)) : 0;
     size_t off = 0;
     p.off_stats = off;
     off = align256(off + (size_t)p.nvl * M * 2 * sizeof(float));
@@ -420,8 +429,8 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
         off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
     }
     if (exact) {
-        // logits z fp32 [M][V] from the exact GEMM (one K tree, or one chain for the baseline)
-        tbik_status st = plan_gemm(M > 0 ? M : 1, V, H, 1, p.noninv ? H : leaf, TBIK_EXACT | TBIK_B_NK, sms, p.zplan);
+        // logits z fp32 [M][V] from the exact GEMM (the K tree, or the baseline's T chains summed in order)
+        tbik_status st = zgemm_plan(p, sms, p.zplan);
         if (st != TBIK_OK) return st;
         p.off_z = off;
         off = align256(off + (size_t)M * V * sizeof(float));
@@ -611,7 +620,8 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
         prm.M = M, prm.N = V, prm.K = H;
-        prm.leaf = p.noninv ? H : leaf;
+        prm.leaf = p.noninv ? H / T : leaf;
+        prm.seq = p.noninv ? 1 : 0;
         prm.F = 1;
         prm.tiles_m = p.tiles_m, prm.tiles_n = p.nvt;
         prm.group_m = p.tiles_m;  // all row tiles of a vocab tile run together: W_lm is read once
@@ -627,14 +637,14 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         prm.debug = g_debug_flags & ~TBIK_DEBUG_WITHHOLD_ACC_ARRIVE;
         prm.wait_cycles = wait_cycles(info);
         prm.lo[0] = 0;
-        prm.nl[0] = (short)(p.noninv ? 1 : p.Lk);
+        prm.nl[0] = (short)p.Lk;
         prm.tab_n[0] = prm.tab_n[1] = prm.nl[0];
         gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
         if ((st = launch_status()) != TBIK_OK) return st;
     } else {
         float* z = reinterpret_cast<float*>(w8 + p.off_z);
         GemmPlan zp;
-        st = plan_gemm(M, V, H, 1, p.noninv ? H : leaf, TBIK_EXACT | TBIK_B_NK, info->sms, zp);
+        st = zgemm_plan(p, info->sms, zp);
         if (st != TBIK_OK) return st;
         if (zp.total > p.zplan.total) return TBIK_ERR_WORKSPACE;
         st = run_gemm(zp, hidden, W, z, w8 + p.off_zgemm, s, info);
@@ -646,7 +656,7 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         if ((st = launch_status()) != TBIK_OK) return st;
     }
     logprob_row_kernel<<<(M + ROW_WARPS - 1) / ROW_WARPS, ROW_WARPS * 32, 0, s>>>(stats, zt, targets, out, shard, M,
-                                                                                V, p.nvl, p.Lv, T, p.noninv);
+                                                                                V, p.nvl, p.Lv, T);
     return launch_status();
 }
 

@@ -410,12 +410,6 @@ static ms_t tree_ms(const ms_t* P, int lo, int n) {
     return ms_combine(tree_ms(P, lo, h), tree_ms(P, lo + h, n - h));
 }
 
-static ms_t seq_ms(const ms_t* P, int lo, int n) {
-    ms_t acc = P[lo];
-    for (int i = 1; i < n; ++i) acc = ms_combine(acc, P[lo + i]);
-    return acc;
-}
-
 void oracle_tree_ms(const float* m, const float* s, int n, float* out_m, float* out_s) {
     ms_t* P = (ms_t*)malloc(sizeof(ms_t) * (size_t)n);
     for (int i = 0; i < n; ++i) {
@@ -440,8 +434,11 @@ void oracle_tree_ms(const float* m, const float* s, int n, float* out_m, float* 
  *   Lv = vpad/vleaf leaves; shard t owns leaves [t*Lv/T, (t+1)*Lv/T)
  *   (m_t, s_t) = TREE over its leaves; (m, s) = TREE over the T shards
  *   out[i]     = (z[target] - m) - log(s);  a target outside [0, V) gives NaN.
- * noninv != 0 is the non-invariant baseline: z is one fma chain over all H,
- * and both combines run left to right instead of by the tree.
+ * noninv != 0 is the non-invariant baseline applied to the lm_head GEMM:
+ * H is split into T contiguous shards, each logit is one fma chain per shard
+ * and the T partial logits are summed left to right ("per-shard GEMM, then a
+ * sequential sum of the partials"); the vocabulary reduction is the tree
+ * above, so the baseline differs from the method only in the logits.
  * row_m/row_s (nullable) receive the final (m, s) per row.
  */
 int oracle_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* targets, float* out,
@@ -452,7 +449,7 @@ int oracle_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* tar
         return -1;
     int Lk = H / leaf;
     int Lv = vpad / vleaf;
-    if (Lv % T) return -1;
+    if (Lv % T || (noninv && H % T)) return -1;
     int Ls = Lv / T;
     float* z = (float*)malloc(sizeof(float) * (size_t)V);
     float* P = (float*)malloc(sizeof(float) * (size_t)Lk);
@@ -463,9 +460,14 @@ int oracle_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* tar
         for (int v = 0; v < V; ++v) {
             const uint16_t* w = W + (size_t)v * H;
             if (noninv) {
-                float acc = 0.0f;
-                for (int k = 0; k < H; ++k) acc = fmaf(bf(h[k]), bf(w[k]), acc);
-                z[v] = acc;
+                int Hs = H / T;
+                float sum = 0.0f;
+                for (int t = 0; t < T; ++t) {
+                    float acc = 0.0f;
+                    for (int k = t * Hs; k < (t + 1) * Hs; ++k) acc = fmaf(bf(h[k]), bf(w[k]), acc);
+                    sum = t ? sum + acc : acc;
+                }
+                z[v] = sum;
             } else {
                 for (int j = 0; j < Lk; ++j) {
                     float acc = 0.0f;
@@ -491,8 +493,8 @@ int oracle_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* tar
             leaves[j].m = m;
             leaves[j].s = s;
         }
-        for (int t = 0; t < T; ++t) shards[t] = noninv ? seq_ms(leaves, t * Ls, Ls) : tree_ms(leaves, t * Ls, Ls);
-        ms_t fin = noninv ? seq_ms(shards, 0, T) : tree_ms(shards, 0, T);
+        for (int t = 0; t < T; ++t) shards[t] = tree_ms(leaves, t * Ls, Ls);
+        ms_t fin = tree_ms(shards, 0, T);
         if (row_m) row_m[i] = fin.m;
         if (row_s) row_s[i] = fin.s;
         int tg = targets[i];
