@@ -50,7 +50,8 @@ constexpr int TC_BN = 128;
 constexpr int TC_BK = 128;                // K per ring stage
 constexpr int TC_KSLICES = TC_BK / 64;    // 64-wide (128-byte) swizzle slices per stage
 constexpr int TC_KSTEPS = TC_BK / 16;     // MMAs (K = 16) per stage
-constexpr int TC_STAGES = 3;
+constexpr int TC_STAGES = 3;       // ring stages when A fills its 128 rows
+constexpr int TC_MAX_STAGES = 8;   // ring stages when the A copies are small (small M)
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;        // this CTA's A rows
 constexpr int TC_B_BYTES = (TC_BN / 2) * TC_BK * 2;  // this CTA's half of B
 constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each owning 64 columns
@@ -62,7 +63,8 @@ constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_MAX_F = 64;
 constexpr int TC_SLOT_FLOATS = TC_BM * TC_BN;
 constexpr int TC_TAB_MAX = 1024;  // leaves per subtree covered by the shared-memory op table
-constexpr size_t TC_SMEM_BYTES = (size_t)TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + TC_SLOT_FLOATS * 4 +
+constexpr int TC_RING_BYTES = TC_STAGES * (TC_A_BYTES + TC_B_BYTES);
+constexpr size_t TC_SMEM_BYTES = (size_t)TC_RING_BYTES + TC_SLOT_FLOATS * 4 +
                                  2 * TC_TAB_MAX * 2 /*op tables*/ + 1024 /*align*/ + 256 /*barriers*/;
 
 enum { EPI_TREE = 0, EPI_LOGPROB = 1 };
@@ -89,6 +91,12 @@ struct TcParams {
     unsigned debug;
     unsigned long long wait_cycles;  // bound of every device-side wait, in SM cycles
     int seq;                         // 1: the leaves form the left-to-right chain, not the tree
+    int a_box_rows;                  // rows per A copy: 128, or M rounded up to 8 when M <= 128
+    // Ring layout: stage s at s * stage_bytes holds two A slices of a_slice
+    // bytes (a_box_rows rows of 128 bytes) and then the two 8 KiB B slices;
+    // stages = TC_RING_BYTES / stage_bytes, at most TC_MAX_STAGES.
+    int stages;
+    uint32_t stage_bytes, a_slice;
     int tab_n[2];                    // the (at most two) subtree sizes of the frontier nodes
     short lo[TC_MAX_F];
     short nl[TC_MAX_F];
@@ -159,14 +167,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                    const __grid_constant__ TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
-    float* sSlot = reinterpret_cast<float*>(sB + TC_STAGES * TC_B_BYTES);  // pending 3-4 leaf subtree
+    uint8_t* ring = smem;
+    float* sSlot = reinterpret_cast<float*>(smem + TC_RING_BYTES);  // pending 3-4 leaf subtree
     uint16_t* leaf_tab = reinterpret_cast<uint16_t*>(sSlot + TC_SLOT_FLOATS);  // [2][TC_TAB_MAX]
     uint64_t* bars = reinterpret_cast<uint64_t*>(leaf_tab + 2 * TC_TAB_MAX);
-    uint64_t* full = bars;                      // [STAGES] both CTAs' copies landed (leader's)
-    uint64_t* empty = bars + TC_STAGES;         // [STAGES] MMAs done reading (both CTAs)
-    uint64_t* acc_full = bars + 2 * TC_STAGES;  // [3] leaf accumulator ready (both CTAs)
+    uint64_t* full = bars;                          // [stages] both CTAs' copies landed (leader's)
+    uint64_t* empty = bars + TC_MAX_STAGES;         // [stages] MMAs done reading (both CTAs)
+    uint64_t* acc_full = bars + 2 * TC_MAX_STAGES;  // [3] leaf accumulator ready (both CTAs)
     uint64_t* acc_empty = acc_full + 3;         // [3] leaf accumulator drained by both CTAs (leader's)
     uint64_t* done = acc_empty + 3;             // all MMAs retired (both CTAs)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
@@ -184,7 +191,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < TC_STAGES; ++s) {
+        for (int s = 0; s < TC_MAX_STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -219,7 +226,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
             const bool b_mn = p.b_mn != 0;
-            uint32_t q = 0;
+            const int stages = p.stages;
+            uint32_t q = 0, ph = 0;
+            int s = 0;
             for (int u = pair; u < p.total_units; u += npairs) {
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
@@ -227,31 +236,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 const int nkb = (p.nl[f] * p.leaf + TC_BK - 1) / TC_BK;
                 const int arow = tm * TC_PAIR_M + TC_BM * rank;
                 const int brow = tn * TC_BN + (TC_BN / 2) * rank;
+                // A CTA whose 128 rows are all past M copies no A: the MMA
+                // then reads stale shared memory for rows whose results are
+                // never stored (rows of an MMA are independent).  Small M also
+                // copies only a_box_rows rows.
+                const int rows_pair = p.M - tm * TC_PAIR_M;
+                const bool a_mine = rows_pair - TC_BM * (int)rank > 0;
+                const uint32_t a_copy = p.a_slice * TC_KSLICES;  // bytes per CTA and stage
+                const uint32_t tx = a_copy * (rows_pair > TC_BM ? 2u : 1u) + 2u * TC_B_BYTES;
                 for (int kb = 0; kb < nkb; ++kb) {
-                    const int s = q % TC_STAGES;
-                    if (!mbar_wait(&empty[s], ((q / TC_STAGES) & 1) ^ 1, abort_flag, wait_lim)) goto producer_out;
+                    if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, wait_lim)) goto producer_out;
                     const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (TC_A_BYTES + TC_B_BYTES));
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
                     const int kx = k0 + kb * TC_BK;
+                    uint8_t* sA = ring + (size_t)s * p.stage_bytes;
+                    uint8_t* sB = sA + a_copy;
 #pragma unroll
                     for (int h = 0; h < TC_KSLICES; ++h) {
-                        tma_load_2d_pair(sA + s * TC_A_BYTES + h * (TC_A_BYTES / TC_KSLICES), &tmA, bar, kx + 64 * h,
-                                         arow);
+                        if (a_mine) tma_load_2d_pair(sA + h * p.a_slice, &tmA, bar, kx + 64 * h, arow);
                         if (!b_mn)
-                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar,
-                                             kx + 64 * h, brow);
+                            tma_load_2d_pair(sB + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar, kx + 64 * h, brow);
                         else
-                            tma_load_2d_pair(sB + s * TC_B_BYTES + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar, brow,
-                                             kx + 64 * h);
+                            tma_load_2d_pair(sB + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar, brow, kx + 64 * h);
                     }
                     ++q;
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
             }
         producer_out:
             // The leader lets the copies of both CTAs land before the pair can exit.
             if (rank == 0)
-                for (uint32_t i = (q > (uint32_t)TC_STAGES ? q - TC_STAGES : 0u); i < q; ++i)
-                    mbar_drain(&full[i % TC_STAGES], (i / TC_STAGES) & 1, wait_lim);
+                for (uint32_t i = (q > (uint32_t)stages ? q - stages : 0u); i < q; ++i)
+                    mbar_drain(&full[i % stages], (i / stages) & 1, wait_lim);
         }
     } else if (warp == 1 || warp == TC_WAITER_WARP) {
         // ------------------------------------------------ MMA issuer + waiter (leader)
@@ -267,20 +286,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, TC_BN, 0, p.b_mn);
             const bool b_mn = p.b_mn != 0;
             const uint32_t b_lbo = p.b_lbo, b_sbo = p.b_sbo;
-            const uint32_t sA_u = smem_u32(sA), sB_u = smem_u32(sB);
+            const uint32_t ring_u = smem_u32(ring);
+            const uint32_t stage_bytes = p.stage_bytes, a_slice = p.a_slice;
+            const int stages = p.stages;
             const int spl = p.leaf / 16;  // MMAs per leaf
             const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
             const bool aligned = (spl % TC_KSTEPS) == 0;  // leaf is a whole number of stages
             const int kb_per_leaf = spl / TC_KSTEPS;
-            uint32_t q = 0, a = 0, hc = 0;
+            uint32_t a = 0, hc = 0, ph = 0;  // ph: phase of the ring (flips when stage 0 comes round)
+            int s = 0;
             // The hand-off: waiter lane 0 waits (bounded) for what the issuer needs.
-            auto handoff = [&](bool need_full, bool need_acc, int s, uint32_t abuf, uint32_t acount) -> bool {
+            auto handoff = [&](bool need_full, bool need_acc, uint32_t abuf, uint32_t acount) -> bool {
                 volatile int* verdict = handoff_go + (hc & 1);
                 ++hc;
                 if (!is_mma) {
                     if (lane == 0) {
                         bool ok = true;
-                        if (need_full) ok = mbar_wait(&full[s], (q / TC_STAGES) & 1, abort_flag, wait_lim);
+                        if (need_full) ok = mbar_wait(&full[s], ph, abort_flag, wait_lim);
                         if (ok && need_acc)
                             ok = mbar_wait(&acc_empty[abuf], ((acount / 3) & 1) ^ 1, abort_flag, wait_lim);
                         *verdict = ok ? 1 : 0;
@@ -299,20 +321,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 uint32_t buf = 0;
                 int in_leaf = 0, kb_in_leaf = 0;
                 for (int st = 0; st < nsteps; st += TC_KSTEPS) {
-                    const int s = q % TC_STAGES;
-                    const uint64_t adesc = smem_desc_sw128(sA_u + s * TC_A_BYTES, 16, 1024);
-                    const uint64_t bdesc = b_mn ? smem_desc_sw128(sB_u + s * TC_B_BYTES, b_lbo, b_sbo)
-                                                : smem_desc_sw128(sB_u + s * TC_B_BYTES, 16, 1024);
+                    // The A slices of a small-M stage are a_box_rows rows apart;
+                    // the MMA's other rows read whatever follows (results never
+                    // stored), always inside this CTA's shared memory.
+                    const uint32_t sa = ring_u + (uint32_t)s * stage_bytes;
+                    const uint32_t sb = sa + a_slice * TC_KSLICES;
+                    const uint64_t adesc = smem_desc_sw128(sa, 16, 1024);
+                    const uint64_t bdesc = b_mn ? smem_desc_sw128(sb, b_lbo, b_sbo) : smem_desc_sw128(sb, 16, 1024);
                     // k-step ks: slice ks/4 (advance by a slice's bytes >> 4), step ks%4 within it
                     auto a_at = [&](int ks) {
-                        return adesc + (uint64_t)((ks >> 2) * ((TC_A_BYTES / TC_KSLICES) >> 4) + (ks & 3) * 2);
+                        return adesc + (uint64_t)((ks >> 2) * (a_slice >> 4) + (ks & 3) * 2);
                     };
                     auto b_at = [&](int ks) {
                         return bdesc + (uint64_t)((ks >> 2) * ((TC_B_BYTES / TC_KSLICES) >> 4)) + b_step * (ks & 3);
                     };
                     if (aligned) {
                         if (kb_in_leaf == 0) buf = a % 3;
-                        if (!handoff(true, kb_in_leaf == 0, s, buf, a)) goto mma_out;
+                        if (!handoff(true, kb_in_leaf == 0, buf, a)) goto mma_out;
                         if (is_mma && lane == 0) {
                             const uint32_t d = tmem_base + buf * TC_BN;
                             tc_mma_pair(d, a_at(0), b_at(0), idesc, kb_in_leaf != 0 ? 1u : 0u);
@@ -329,7 +354,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                         for (int ks = 0; ks < nk; ++ks) {
                             if (in_leaf == 0) buf = a % 3;
                             if (ks == 0 || in_leaf == 0)
-                                if (!handoff(ks == 0, in_leaf == 0, s, buf, a)) goto mma_out;
+                                if (!handoff(ks == 0, in_leaf == 0, buf, a)) goto mma_out;
                             if (is_mma && lane == 0) {
                                 tc_mma_pair(tmem_base + buf * TC_BN, a_at(ks), b_at(ks), idesc, in_leaf != 0 ? 1u : 0u);
                                 if (in_leaf + 1 == spl) tc_commit_pair(&acc_full[buf]);
@@ -342,7 +367,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                     }
                     if (is_mma && lane == 0) tc_commit_pair(&empty[s]);
                     __syncwarp();
-                    ++q;
+                    if (++s == stages) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
             }
         mma_out:

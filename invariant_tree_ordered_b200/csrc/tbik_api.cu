@@ -130,6 +130,20 @@ void launch_token_loop(Kernel kernel, int threads, int items, const DeviceInfo* 
     kernel<<<grid, threads, 0, s>>>(args...);
 }
 
+// Rows of A per TMA copy in the tensor-core kernel: the whole 128-row half
+// tile, or only M rounded up to a whole 8-row swizzle atom when M <= 128.
+int a_box_rows(int M) { return M >= TC_BM ? TC_BM : ((M + 7) / 8) * 8; }
+
+// Ring of the tensor-core kernel: with a small A copy (small M) the same
+// shared memory holds more stages of B, i.e. more bytes in flight.
+void set_ring(TcParams& prm, int a_box) {
+    prm.a_box_rows = a_box;
+    prm.a_slice = (uint32_t)a_box * 128u;
+    prm.stage_bytes = 2u * prm.a_slice + (uint32_t)TC_B_BYTES;
+    const int st = (int)(TC_RING_BYTES / prm.stage_bytes);
+    prm.stages = st < TC_MAX_STAGES ? st : TC_MAX_STAGES;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 int ilog2(int x) {
@@ -315,12 +329,14 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
     if (p.M == 0) return TBIK_OK;
     if (p.tc) {
         CUtensorMap ta, tb;
-        if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, 64, TC_BM)) return TBIK_ERR_CUDA;
+        const int a_box = a_box_rows(p.M);
+        if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
         bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, 64, TC_BN / 2)
                           : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, TC_BN / 2, 64);
         if (!okb) return TBIK_ERR_CUDA;
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
+        set_ring(prm, a_box);
         prm.M = p.M, prm.N = p.N, prm.K = p.K;
         prm.leaf = p.leaf_eff;
         prm.F = p.F;
@@ -615,10 +631,12 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
     float* shard = reinterpret_cast<float*>(w8 + p.off_shard);
     if (p.tc) {
         CUtensorMap ta, tb;
-        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, 64, TC_BM)) return TBIK_ERR_CUDA;
+        const int a_box = a_box_rows(M);
+        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
         if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, 64, TC_BN / 2)) return TBIK_ERR_CUDA;
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
+        set_ring(prm, a_box);
         prm.M = M, prm.N = V, prm.K = H;
         prm.leaf = p.noninv ? H / T : leaf;
         prm.seq = p.noninv ? 1 : 0;
