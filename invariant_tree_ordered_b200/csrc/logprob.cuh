@@ -6,12 +6,9 @@
 //    columns) the running max in ascending column order and the ascending sum
 //    of exp(z - max), from materialised fp32 logits.  The tensor-core mode
 //    computes the same summaries inside the GEMM epilogue instead.
-//  * logprob_row_kernel: one warp per row.  Lane l reduces frontier node l of
-//    the halving tree over the Lv padded leaves (a whole subtree, streamed
-//    leaf by leaf with a small stack); the upper levels are xor-butterfly
-//    levels in which the left operand of every combine is the lower lane.  The
-//    T shard summaries are taken at their own level, written to the shard
-//    buffer, read back and combined by the top levels of the same tree.
+//  * logprob_row_kernel: the vocabulary tree per row over the Lv padded
+//    leaves: frontier subtrees streamed leaf by leaf with a small stack, then
+//    xor-butterfly levels, the T shard summaries taken at their own level.
 #pragma once
 
 #include "device_common.cuh"
@@ -66,16 +63,26 @@ __device__ __forceinline__ MS butterfly_ms(MS v, int lane, int w) {
     return (lane & w) ? ms_combine(o, v) : ms_combine(v, o);
 }
 
-constexpr int ROW_WARPS = 8;
+constexpr int ROW_BLOCK = 32;  // rows per CTA of the row kernel (one per lane), 32 warps
 
-__global__ void __launch_bounds__(ROW_WARPS * 32)
+// The vocabulary tree per row.  Frontier node f (depth d, nf = 2^d <= 32
+// whole subtrees) of row r is reduced by lane r of warp f, streaming its
+// leaves with a small stack, so a warp's loads of one leaf index cover 32
+// consecutive rows (coalesced).  The nf subtree results go through shared
+// memory to warp r, whose lane f then holds node f of row r, and the upper
+// levels are xor-butterfly levels in which the left operand of every combine
+// is the lower lane.  The T shard summaries are taken at their own level,
+// written to the shard buffer, read back and combined by the top levels.
+__global__ void __launch_bounds__(ROW_BLOCK * 32)
     logprob_row_kernel(const float* __restrict__ stats, const float* __restrict__ zt,
                        const int32_t* __restrict__ targets, float* __restrict__ out, float* shard_ms, int M, int V,
                        int nvt, int Lv, int T) {
     constexpr int TAB = 512;
-    __shared__ uint16_t tab[2][TAB];  // leaf operation codes for the two frontier subtree sizes
+    __shared__ uint16_t tab[2][TAB];        // leaf operation codes for the two frontier subtree sizes
+    __shared__ float2 part[32][ROW_BLOCK];  // [frontier node][row in block]
     const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+    const int warp = threadIdx.x >> 5;
+    const int row0 = blockIdx.x * ROW_BLOCK;
     int d = 0;
     while (d < 5 && (2 << d) <= Lv) ++d;  // largest d <= 5 with 2^d <= Lv
     const int nf = 1 << d;
@@ -90,34 +97,47 @@ __global__ void __launch_bounds__(ROW_WARPS * 32)
         }
     }
     __syncthreads();
+    // Frontier node `warp` of row row0 + lane.
+    if (warp < nf) {
+        const int row = row0 + lane;
+        MS v;
+        v.m = -INFINITY;
+        v.s = 0.0f;
+        if (row < M) {
+            int lo = 0, n = Lv;
+            for (int lvl = 0; lvl < d; ++lvl) {
+                const int h = (n + 1) >> 1;
+                if ((warp >> (d - 1 - lvl)) & 1) {
+                    lo += h;
+                    n -= h;
+                } else {
+                    n = h;
+                }
+            }
+            MS stk[24];
+            int sp = 0;
+            const uint16_t* tb = tab[n == n_hi ? 0 : 1];
+            for (int j = 0; j < n; ++j) {
+                MS cur = leaf_ms(stats, M, nvt, row, lo + j);
+                const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
+                const int npop = code_pops(code);
+                for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
+                if (!((code >> 10) & 1)) stk[sp++] = cur;
+                else v = cur;
+            }
+        }
+        part[warp][lane] = make_float2(v.m, v.s);
+    }
+    __syncthreads();
+    const int row = row0 + warp;
     if (row >= M) return;
-    // Each shard's vocab leaves by the tree: the frontier subtrees in
-    // lanes, then butterflies inside each shard's lanes.
     MS v;
     v.m = -INFINITY;
     v.s = 0.0f;
     if (lane < nf) {
-        int lo = 0, n = Lv;
-        for (int lvl = 0; lvl < d; ++lvl) {
-            const int h = (n + 1) >> 1;
-            if ((lane >> (d - 1 - lvl)) & 1) {
-                lo += h;
-                n -= h;
-            } else {
-                n = h;
-            }
-        }
-        MS stk[24];
-        int sp = 0;
-        const uint16_t* tb = tab[n == n_hi ? 0 : 1];
-        for (int j = 0; j < n; ++j) {
-            MS cur = leaf_ms(stats, M, nvt, row, lo + j);
-            const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
-            const int npop = code_pops(code);
-            for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
-            if (!((code >> 10) & 1)) stk[sp++] = cur;
-            else v = cur;
-        }
+        const float2 t2 = part[lane][warp];
+        v.m = t2.x;
+        v.s = t2.y;
     }
     const int sl = nf / T;  // lanes per shard
     for (int w = 1; w < sl; w <<= 1) v = butterfly_ms(v, lane, w);

@@ -673,7 +673,7 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
         vocab_stats_kernel<<<blocks, 256, 0, s>>>(z, targets, stats, zt, M, V, p.nvl);
         if ((st = launch_status()) != TBIK_OK) return st;
     }
-    logprob_row_kernel<<<(M + ROW_WARPS - 1) / ROW_WARPS, ROW_WARPS * 32, 0, s>>>(stats, zt, targets, out, shard, M,
+    logprob_row_kernel<<<(M + ROW_BLOCK - 1) / ROW_BLOCK, ROW_BLOCK * 32, 0, s>>>(stats, zt, targets, out, shard, M,
                                                                                 V, p.nvl, p.Lv, T);
     return launch_status();
 }
