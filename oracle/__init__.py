@@ -80,6 +80,8 @@ def _load():
                 "oracle_swiglu_f32": (None, [vp, vp, vp, i64]),
                 "oracle_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]),
                 "oracle_logprob_f64": (None, [vp, vp, vp, vp, i32, i32, i32]),
+                "oracle_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32]),
+                "oracle_attention_f64": (None, [vp, vp, vp, vp, i32, i32, i32, i32]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(lib, name)
@@ -252,3 +254,25 @@ def logprob_f64(hidden_bits, w_bits, targets):
     out = np.empty(M, dtype=np.float64)
     _load().oracle_logprob_f64(ph, pw, pt, out.ctypes.data, M, V, H)
     return out
+
+
+def attention(q_bits, k_bits, v_bits, *, chunk: int = 64):
+    """Causal attention, keys in chunks combined by the tree; bf16 [batch, seq, heads, head_dim] in and out."""
+    q, pq = _c(q_bits, np.uint16)
+    k, pk = _c(k_bits, np.uint16)
+    v, pv = _c(v_bits, np.uint16)
+    B, S, NH, D = q.shape
+    out = np.empty_like(q)
+    _check(_load().oracle_attention(pq, pk, pv, out.ctypes.data, B, S, NH, D, chunk), "attention")
+    return out
+
+
+def attention_f64(q_bits, k_bits, v_bits):
+    q, pq = _c(q_bits, np.uint16)
+    k, pk = _c(k_bits, np.uint16)
+    v, pv = _c(v_bits, np.uint16)
+    B, S, NH, D = q.shape
+    out = np.empty(q.shape, dtype=np.float64)
+    _load().oracle_attention_f64(pq, pk, pv, out.ctypes.data, B, S, NH, D)
+    return out
+

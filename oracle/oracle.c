@@ -533,3 +533,146 @@ void oracle_logprob_f64(const uint16_t* hidden, const uint16_t* W, const int32_t
     }
     free(z);
 }
+
+/* ------------------------------------------------------------- attention */
+/*
+ * Causal attention with the keys in fixed chunks combined by TREE (the
+ * end-to-end decoder row; the pages' tree order applied to the reduction over
+ * keys).  Readings (listed in the design notes as A1-A4):
+ *  A1 score s_j = fl(dot(q_i, k_j) * scale): dot accumulated over the head
+ *     dimension in ascending order with fmaf from +0, scale = the binary32
+ *     nearest to 1/sqrt(head_dim).  Keys j <= i only.
+ *  A2 keys form chunks of `chunk` consecutive positions; chunk c holds keys
+ *     [c*chunk, c*chunk + chunk) that are <= i.  Per chunk: m = max of its
+ *     scores; p_j = exp(s_j - m) (exp_spec), 0 for a slot past i;
+ *     s = TREE over the chunk's `chunk` slots of p; o[d] = ascending sum over
+ *     the chunk's keys of p_j * v_j[d] by fmaf from +0.
+ *  A3 chunk results combine as (m,s,o) (+) (m',s',o'): M = max(m, m'),
+ *     e = exp(m - M), e' = exp(m' - M), s = s*e + s'*e', o[d] = o[d]*e + o'[d]*e'
+ *     (products rounded separately); the chunks 0..floor(i/chunk) by TREE.
+ *  A4 out[d] = bf16(o[d] / s).
+ * Layout: q, k, v, out bf16 [batch][seq][heads][head_dim]; head_dim <= 256.
+ */
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int seq, heads, hd, chunk, i;
+    size_t b_off;  /* element offset of this sequence */
+    int h;
+    float scale;
+} att_ctx;
+
+static size_t att_at(const att_ctx* c, int pos) {
+    return c->b_off + ((size_t)pos * c->heads + c->h) * c->hd;
+}
+
+/* one chunk: (m, s, o) */
+static void att_chunk(const att_ctx* c, int ci, float* m_out, float* s_out, float* o) {
+    int j0 = ci * c->chunk;
+    int j1 = j0 + c->chunk - 1;
+    if (j1 > c->i) j1 = c->i;
+    int n = j1 - j0 + 1;
+    float* sc = (float*)malloc(sizeof(float) * (size_t)c->chunk);
+    float* p = (float*)malloc(sizeof(float) * (size_t)c->chunk);
+    const uint16_t* q = c->q + att_at(c, c->i);
+    for (int t = 0; t < n; ++t) {
+        const uint16_t* k = c->k + att_at(c, j0 + t);
+        float dot = 0.0f;
+        for (int d = 0; d < c->hd; ++d) dot = fmaf(bf(q[d]), bf(k[d]), dot);
+        sc[t] = dot * c->scale;
+    }
+    float m = sc[0];
+    for (int t = 1; t < n; ++t)
+        if (sc[t] > m) m = sc[t];
+    for (int t = 0; t < c->chunk; ++t) p[t] = (t < n) ? exp_spec(sc[t] - m) : 0.0f;
+    float s = tree_f32(p, 0, c->chunk);
+    for (int d = 0; d < c->hd; ++d) {
+        float acc = 0.0f;
+        for (int t = 0; t < n; ++t) acc = fmaf(p[t], bf(c->v[att_at(c, j0 + t) + d]), acc);
+        o[d] = acc;
+    }
+    *m_out = m;
+    *s_out = s;
+    free(sc);
+    free(p);
+}
+
+/* TREE over chunks [lo, lo+n) */
+static void att_tree(const att_ctx* c, int lo, int n, float* m_out, float* s_out, float* o) {
+    if (n == 1) {
+        att_chunk(c, lo, m_out, s_out, o);
+        return;
+    }
+    int h = (n + 1) / 2;
+    float ma, sa, mb, sb, ob[256];
+    att_tree(c, lo, h, &ma, &sa, o);
+    att_tree(c, lo + h, n - h, &mb, &sb, ob);
+    float M = (mb > ma) ? mb : ma;
+    float ea = exp_spec(ma - M), eb = exp_spec(mb - M);
+    float pa = sa * ea, pb = sb * eb;
+    *m_out = M;
+    *s_out = pa + pb;
+    for (int d = 0; d < c->hd; ++d) {
+        float xa = o[d] * ea, xb = ob[d] * eb;
+        o[d] = xa + xb;
+    }
+}
+
+int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int batch, int seq,
+                     int heads, int head_dim, int chunk) {
+    if (batch < 0 || seq < 0 || heads <= 0 || head_dim <= 0 || head_dim > 256 || chunk <= 0) return -1;
+    att_ctx c;
+    c.q = q;
+    c.k = k;
+    c.v = v;
+    c.seq = seq;
+    c.heads = heads;
+    c.hd = head_dim;
+    c.chunk = chunk;
+    c.scale = (float)(1.0 / sqrt((double)head_dim));
+    float o[256];
+    for (int b = 0; b < batch; ++b) {
+        c.b_off = (size_t)b * seq * heads * head_dim;
+        for (int h = 0; h < heads; ++h) {
+            c.h = h;
+            for (int i = 0; i < seq; ++i) {
+                c.i = i;
+                float m, s;
+                att_tree(&c, 0, i / chunk + 1, &m, &s, o);
+                uint16_t* dst = out + att_at(&c, i);
+                for (int d = 0; d < head_dim; ++d) dst[d] = bf16_rne(o[d] / s);
+            }
+        }
+    }
+    return 0;
+}
+
+/* Binary64 causal softmax attention (no chunks), for tolerance checks. */
+void oracle_attention_f64(const uint16_t* q, const uint16_t* k, const uint16_t* v, double* out, int batch, int seq,
+                          int heads, int head_dim) {
+    double* sc = (double*)malloc(sizeof(double) * (size_t)(seq > 0 ? seq : 1));
+    double scale = 1.0 / sqrt((double)head_dim);
+    for (int b = 0; b < batch; ++b)
+        for (int h = 0; h < heads; ++h)
+            for (int i = 0; i < seq; ++i) {
+                size_t qi = (((size_t)b * seq + i) * heads + h) * head_dim;
+                double mx = -INFINITY;
+                for (int j = 0; j <= i; ++j) {
+                    size_t kj = (((size_t)b * seq + j) * heads + h) * head_dim;
+                    double dot = 0.0;
+                    for (int d = 0; d < head_dim; ++d) dot += (double)bf(q[qi + d]) * (double)bf(k[kj + d]);
+                    sc[j] = dot * scale;
+                    if (sc[j] > mx) mx = sc[j];
+                }
+                double s = 0.0;
+                for (int j = 0; j <= i; ++j) s += exp(sc[j] - mx);
+                for (int d = 0; d < head_dim; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= i; ++j) {
+                        size_t vj = (((size_t)b * seq + j) * heads + h) * head_dim;
+                        acc += exp(sc[j] - mx) * (double)bf(v[vj + d]);
+                    }
+                    out[qi + d] = acc / s;
+                }
+            }
+    free(sc);
+}

@@ -413,3 +413,62 @@ def test_logprob_noninv_diverges_over_T():
     t = synth.uniform_int32(40, M, 0, V)
     outs = [oracle.logprob(h, w, t, T=T, leaf=128, noninv=True) for T in (1, 2, 4, 8)]
     assert any(not np.array_equal(bits(outs[0]), bits(o)) for o in outs[1:])
+
+
+# ------------------------------------------------------------- attention
+
+def _bf16_of(x):
+    """bf16 bits of values that bf16 represents exactly (checked)."""
+    f = np.asarray(x, dtype=np.float32)
+    b = (f.view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(synth.bf16_bits_to_f32(b), f)
+    return b
+
+
+def test_attention_single_key_is_v():
+    q = synth.normal_bf16(60, (2, 1, 3, 128))
+    k = synth.normal_bf16(61, (2, 1, 3, 128))
+    v = synth.normal_bf16(62, (2, 1, 3, 128))
+    assert np.array_equal(oracle.attention(q, k, v), v)  # p = exp(0) = 1, s = 1, o = v
+
+
+def test_attention_chunk_tree_grouping_and_causality():
+    # equal scores (identical keys) make every p = 1 and every combine factor
+    # exp(0) = 1, so o is a plain fp32 sum of v in the chunk tree's grouping:
+    # keys [1, 2^27, -2^27] as three 1-key chunks: TREE(3) = (c0 + c1) + c2 = 0
+    # (2^27 + 1 rounds to 2^27); the other grouping would give 1.
+    S = 3
+    q = synth.normal_bf16(63, (1, S, 1, 128))
+    k = np.tile(synth.normal_bf16(64, (1, 1, 1, 128)), (1, S, 1, 1))
+    vals = np.array([1.0, 2.0**27, -2.0**27], dtype=np.float32)
+    v = np.zeros((1, S, 1, 128), dtype=np.float32)
+    v[0, :, 0, 0] = vals
+    v[0, :, 0, 1] = 2.0  # mean 2 exactly
+    vb = _bf16_of(v)
+    out = synth.bf16_bits_to_f32(oracle.attention(q, k, vb, chunk=1))
+    assert out[0, 2, 0, 0] == 0.0
+    assert out[0, 1, 0, 0] == np.float32(np.float32(1.0 + 2.0**27) / 2)  # (1 + 2^27) / 2 over keys 0..1
+    assert np.all(out[0, :, 0, 1] == 2.0)
+    # one 3-key chunk: o accumulates keys in ascending order by fma, same grouping here
+    out3 = synth.bf16_bits_to_f32(oracle.attention(q, k, vb, chunk=4))
+    assert out3[0, 2, 0, 0] == 0.0
+    # causality: keys and values after position i never change output i
+    k2, v2 = k.copy(), vb.copy()
+    k2[0, 2] = synth.normal_bf16(65, (1, 128))
+    v2[0, 2] = synth.normal_bf16(66, (1, 128))
+    o1 = oracle.attention(q, k, vb, chunk=1)
+    o2 = oracle.attention(q, k2, v2, chunk=1)
+    assert np.array_equal(o1[0, :2], o2[0, :2])
+
+
+@pytest.mark.parametrize("chunk", [1, 7, 64])
+def test_attention_within_binary64_softmax(chunk):
+    B, S, NH, D = 2, 150, 2, 128
+    q = synth.normal_bf16(67, (B, S, NH, D))
+    k = synth.normal_bf16(68, (B, S, NH, D))
+    v = synth.normal_bf16(69, (B, S, NH, D))
+    got = synth.bf16_bits_to_f32(oracle.attention(q, k, v, chunk=chunk)).astype(np.float64)
+    ref = oracle.attention_f64(q, k, v)
+    # one bf16 rounding (half an ulp of 2^-7 relative) plus fp32 reduction error
+    tol = np.abs(ref) * (2.0**-8 + 2e-5) + 1e-6
+    assert np.all(np.abs(got - ref) <= tol)
