@@ -186,6 +186,39 @@ typedef struct {
 
 TBIK_API tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* args, void* stream);
 
+/* ---- causal attention with the key reduction in tree order --------------- */
+
+/*
+ * Attention of each query position over the keys at positions <= its own,
+ * with the reduction over keys in the same halving tree as every other
+ * reduction here (TBIK summary page, 技术框架), so the output does not depend
+ * on the batch composition or on how heads are split across devices:
+ *   s_j = fl(dot(q_i, k_j) * scale), dot ascending over the head dimension by
+ *         fma from +0, scale = binary32 nearest to 1/sqrt(head_dim);
+ *   keys in chunks of `chunk` = 64 positions; per chunk m = max of its scores,
+ *   p_j = exp(s_j - m) (the library's exp specification), s = TREE over the
+ *   chunk's 64 slots of p (0 past position i), o[d] = ascending sum of
+ *   p_j * v_j[d] by fma from +0;
+ *   chunk summaries combined by TREE: M = max, e = exp(m - M),
+ *   s = s*e + s'*e', o = o*e + o'*e' (products rounded separately);
+ *   out[d] = bf16(o[d] / s).
+ * q, k, v, out: bf16 [batch][seq][heads][head_dim] in device memory, 16-byte
+ * aligned; out may alias q but not k or v.  head_dim in {64, 128};
+ * chunk == 64; seq <= 16384.  Returns TBIK_ERR_SHAPE / _ARG / _ALIGN for
+ * violations, without launching.
+ */
+TBIK_API tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int batch,
+                                    int seq, int heads, int head_dim, int chunk, void* stream);
+
+/*
+ * Embedding rows: out[t] = table[ids[t]] for t < tokens (bf16 rows of d
+ * elements, d % 8 == 0, 16-byte aligned).  An id outside [0, V) gives a zero
+ * row and records TBIK_ERR_TARGET in the device error word.  Data movement
+ * only (the decoder's first step); no counterpart on the pages.
+ */
+TBIK_API tbik_status tbik_embedding(const int32_t* ids, const uint16_t* table, uint16_t* out, int tokens, int V,
+                                    int d, void* stream);
+
 /* ---- fused lm_head -> log-softmax -> target logprob ---------------------- */
 
 TBIK_API size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, unsigned mode);

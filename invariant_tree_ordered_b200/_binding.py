@@ -81,6 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "tbik_rope_swiglu_fp32": (i32, [ctypes.POINTER(RopeSwigluArgs), vp]),
             "tbik_logprob_workspace": (sz, [i32, i32, i32, i32, i32, u32]),
             "tbik_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
+            "tbik_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
+            "tbik_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp]),
             "tbik_get_error": (i32, [vp]),
             "tbik_debug_set": (i32, [u32, ull]),
         }
@@ -232,6 +234,37 @@ def rope_swiglu(*, q=None, k=None, pos=None, table=None, q_out=None, k_out=None,
         a.g, a.u, a.out, a.n, a.in_f32 = _ptr(g), _ptr(u), _ptr(out), g.numel(), int(g.dtype == torch.float32)
     _check(lib.tbik_rope_swiglu_fp32(ctypes.byref(a), _stream_handle(stream)), "tbik_rope_swiglu_fp32")
     return q_out, k_out, out
+
+
+def attention(q, k, v, *, out=None, chunk: int = 64, stream=None):
+    """Causal attention with the key reduction in tree order (see tbik_attention);
+    q, k, v bf16 [batch, seq, heads, head_dim]."""
+    torch = _torch()
+    lib = load_library()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share the shape [batch, seq, heads, head_dim]")
+    B, S, NH, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib.tbik_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, NH, D, chunk, _stream_handle(stream)),
+           "tbik_attention")
+    return out
+
+
+def embedding(ids, table, *, out=None, stream=None):
+    """Rows of ``table`` (bf16 [V, d]) at ``ids`` (int32 [tokens]) (see tbik_embedding)."""
+    torch = _torch()
+    lib = load_library()
+    _need(ids, torch.int32, "ids")
+    _need(table, torch.bfloat16, "table")
+    V, d = table.shape
+    if out is None:
+        out = torch.empty((ids.numel(), d), dtype=torch.bfloat16, device=table.device)
+    _check(lib.tbik_embedding(_ptr(ids), _ptr(table), _ptr(out), ids.numel(), V, d, _stream_handle(stream)),
+           "tbik_embedding")
+    return out
 
 
 def logprob_workspace(M, V, H, T, leaf, mode) -> int:

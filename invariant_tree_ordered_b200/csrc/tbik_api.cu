@@ -15,6 +15,7 @@
 #include "gemm_exact.cuh"
 #include "gemm_tc.cuh"
 #include "logprob.cuh"
+#include "attention.cuh"
 #include "reduce.cuh"
 #include "tbik.h"
 
@@ -553,6 +554,46 @@ tbik_status tbik_rope_table(float* table, int max_pos, int head_dim, double base
         return TBIK_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return TBIK_ERR_CUDA;
     return TBIK_OK;
+}
+
+tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int batch,
+                           int seq, int heads, int head_dim, int chunk, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (batch < 0 || seq < 0 || heads <= 0) return TBIK_ERR_ARG;
+    if ((head_dim != 64 && head_dim != 128) || chunk != ATT_CHUNK || seq > 256 * ATT_CHUNK) return TBIK_ERR_SHAPE;
+    if (batch == 0 || seq == 0) return TBIK_OK;
+    if (!q || !k || !v || !out) return TBIK_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TBIK_ERR_ALIGN;
+    const long long blocks = (long long)batch * heads * ((seq + ATT_WARPS - 1) / ATT_WARPS);
+    if (blocks > 0x7fffffffLL) return TBIK_ERR_SHAPE;
+    const float scale = (float)(1.0 / std::sqrt((double)head_dim));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 128)
+        attention_kernel<4><<<(int)blocks, ATT_WARPS * 32, 0, s>>>(q, k, v, out, batch, seq, heads, scale);
+    else
+        attention_kernel<2><<<(int)blocks, ATT_WARPS * 32, 0, s>>>(q, k, v, out, batch, seq, heads, scale);
+    return launch_status();
+}
+
+tbik_status tbik_embedding(const int32_t* ids, const uint16_t* table, uint16_t* out, int tokens, int V, int d,
+                           void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (tokens < 0 || V <= 0 || d <= 0) return TBIK_ERR_ARG;
+    if (d % 8) return TBIK_ERR_SHAPE;
+    if (tokens == 0) return TBIK_OK;
+    if (!ids || !table || !out) return TBIK_ERR_ARG;
+    if (!aligned16(table) || !aligned16(out)) return TBIK_ERR_ALIGN;
+    const long long work = (long long)tokens * (d / 8);
+    long long blocks = (work + 255) / 256;
+    if (blocks > (long long)info->sms * 16) blocks = (long long)info->sms * 16;
+    embedding_kernel<<<(int)blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ids, table, out, tokens, V, d);
+    return launch_status();
 }
 
 tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) {

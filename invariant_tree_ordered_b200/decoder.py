@@ -1,0 +1,91 @@
+"""A Llama-style pre-norm decoder forward pass built from the library's calls,
+returning the per-token logprob of given targets.  Every step runs in the
+library's kernels; this module only allocates the activations (torch) and
+sequences the calls.
+
+Per layer: y = RMSNorm(h); q, k, v = y Wq, y Wk, y Wv (column-parallel: each
+device holds whole output columns, so the K reduction is the full tree and the
+same for every T); RoPE on q, k; causal attention with the keys in chunks of
+64 combined by the tree (heads split across devices: per-head, so the same
+for every T); o Wo (row-parallel: K = d split into T shards, combined by the
+tree, or by the non-invariant chain-and-sum baseline); residual + RMSNorm;
+gate, up (column-parallel); SwiGLU; down (row-parallel); residual.  Then the
+final RMSNorm and the lm_head logprob (T splits the vocabulary).  GEMM outputs
+are rounded to bf16 once; gammas come with the weights; eps 1e-6; RoPE base
+1e6; positions 0..seq-1 in every sequence.
+"""
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import _binding as tb
+
+
+@dataclass
+class DecoderConfig:
+    d: int
+    heads: int
+    head_dim: int
+    ffn: int
+    vocab: int
+    layers: int
+    leaf: int = 256       # K leaf of the d-wide GEMMs
+    leaf_ffn: int = 176   # K leaf of the down projection (ffn wide)
+
+
+class Decoder:
+    """Weights are device bf16 tensors: ``emb`` and ``lm_head`` [vocab, d],
+    ``gamma`` [d], and per layer ``wq wk wv wo`` [d, d], ``wg wu`` [d, ffn],
+    ``wd`` [ffn, d] ([in, out] row-major)."""
+
+    def __init__(self, cfg: DecoderConfig, emb, lm_head, gamma, layers):
+        self.cfg, self.emb, self.lm_head, self.gamma, self.layers = cfg, emb, lm_head, gamma, layers
+        self._tables = {}
+
+    def _table(self, seq, device):
+        key = (seq, str(device))
+        if key not in self._tables:
+            self._tables[key] = tb.rope_table(seq, self.cfg.head_dim, 1e6, device=device)
+        return self._tables[key]
+
+    def forward(self, ids, targets, pos, *, T: int = 1, tc: bool = True, noninv: bool = False, stream=None):
+        """ids, targets: device int32 [batch, seq]; pos: device int32 [batch*seq]
+        (the position of each token).  Returns fp32 logprobs [batch, seq]."""
+        torch = tb._torch()
+        c = self.cfg
+        B, S = ids.shape
+        n = B * S
+        dev = ids.device
+        bf = torch.bfloat16
+
+        def dense(a, w, leaf, shards=1, baseline=False):
+            out = torch.empty((a.shape[0], w.shape[1]), dtype=bf, device=dev)
+            tb.gemm(a, w, T=shards, leaf=leaf, tc=tc, noninv=baseline, out_bf16=True, out=out, stream=stream)
+            return out
+
+        x = tb.embedding(ids.reshape(-1), self.emb, stream=stream)
+        res = torch.zeros((n, c.d), dtype=bf, device=dev)
+        table = self._table(S, dev)
+        y, res = tb.rmsnorm_residual(x, res, self.gamma, eps=1e-6, T=1, stream=stream)
+        for L in self.layers:
+            q = dense(y, L["wq"], c.leaf)
+            k = dense(y, L["wk"], c.leaf)
+            v = dense(y, L["wv"], c.leaf)
+            q3, k3 = q.view(n, c.heads, c.head_dim), k.view(n, c.heads, c.head_dim)
+            tb.rope_swiglu(q=q3, k=k3, pos=pos, table=table, q_out=q3, k_out=k3, stream=stream)
+            o = tb.attention(q.view(B, S, c.heads, c.head_dim), k.view(B, S, c.heads, c.head_dim),
+                             v.view(B, S, c.heads, c.head_dim), stream=stream)
+            a = dense(o.view(n, c.d), L["wo"], c.leaf, T, noninv)
+            y, res = tb.rmsnorm_residual(a, res, self.gamma, eps=1e-6, T=1, stream=stream)
+            g = dense(y, L["wg"], c.leaf)
+            u = dense(y, L["wu"], c.leaf)
+            _, _, act = tb.rope_swiglu(g=g, u=u, stream=stream)
+            m = dense(act, L["wd"], c.leaf_ffn, T, noninv)
+            y, res = tb.rmsnorm_residual(m, res, self.gamma, eps=1e-6, T=1, stream=stream)
+        lp = tb.logprob(y, self.lm_head, targets.reshape(-1), T=T, leaf=c.leaf, tc=tc, noninv=noninv, stream=stream)
+        return lp.view(B, S)
+
+
+def positions(batch: int, seq: int) -> np.ndarray:
+    """Position of each token of a [batch, seq] block (0..seq-1 per sequence)."""
+    return np.tile(np.arange(seq, dtype=np.int32), batch)

@@ -66,6 +66,7 @@ def _load():
                                       ctypes.c_float, ctypes.c_double)
             sig = {
                 "oracle_bf16_rne": (ctypes.c_uint16, [f32]),
+                "oracle_bf16_rne_array": (None, [vp, vp, i64]),
                 "oracle_tree_sum": (f32, [vp, i32]),
                 "oracle_exp": (f32, [f32]),
                 "oracle_log": (f32, [f32]),
@@ -105,6 +106,14 @@ def _check(rc, what):
 
 def bf16_rne(x: float) -> int:
     return int(_load().oracle_bf16_rne(float(x)))
+
+
+def bf16_rne_array(x) -> np.ndarray:
+    """bf16 bits of float32 values, round to nearest even (element-wise)."""
+    a, pa = _c(x, np.float32)
+    out = np.empty(a.shape, dtype=np.uint16)
+    _load().oracle_bf16_rne_array(pa, out.ctypes.data, a.size)
+    return out
 
 
 def exp(x: float) -> float:

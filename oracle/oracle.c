@@ -65,6 +65,10 @@ static uint16_t bf16_rne(float f) {
 
 uint16_t oracle_bf16_rne(float f) { return bf16_rne(f); }
 
+void oracle_bf16_rne_array(const float* x, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = bf16_rne(x[i]);
+}
+
 /* ------------------------------------------------------------------ tree */
 
 /* R1: the halving tree, straight from its definition. */

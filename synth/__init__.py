@@ -162,3 +162,38 @@ def logprob_inputs(M: int, V: int = 151936, H: int = 4096, with_weight: bool = T
     w = normal_bf16(31, (V, H), std=0.02) if with_weight else None
     targets = uniform_int32(32, M, 0, V)
     return hidden, w, targets
+
+
+# ---------------------------------------------------------------------------
+# End-to-end decoder (Llama-style, pre-norm): shapes, seeds and distributions.
+# ---------------------------------------------------------------------------
+
+DECODER_FULL = dict(d=2048, heads=16, head_dim=128, ffn=5632, vocab=32000, layers=4, batch=8, seq=2048,
+                    leaf=256, leaf_ffn=176)
+DECODER_SMALL = dict(d=256, heads=2, head_dim=128, ffn=512, vocab=1024, layers=2, batch=2, seq=80,
+                     leaf=32, leaf_ffn=64)
+
+
+def decoder_weights(cfg):
+    """Random-init weights, every matrix N(0, 0.02^2) bf16, stored [in, out]
+    row-major (the lm_head [vocab, d]); RMSNorm gammas 1.  Seeds 40 (embedding),
+    41 (lm_head), 50 + 10*l + {0..6} (layer l: q, k, v, o, gate, up, down)."""
+    d, f, V = cfg["d"], cfg["ffn"], cfg["vocab"]
+    w = dict(emb=normal_bf16(40, (V, d), std=0.02), lm_head=normal_bf16(41, (V, d), std=0.02), layers=[])
+    for layer in range(cfg["layers"]):
+        s = 50 + 10 * layer
+        w["layers"].append(dict(
+            wq=normal_bf16(s, (d, d), std=0.02), wk=normal_bf16(s + 1, (d, d), std=0.02),
+            wv=normal_bf16(s + 2, (d, d), std=0.02), wo=normal_bf16(s + 3, (d, d), std=0.02),
+            wg=normal_bf16(s + 4, (d, f), std=0.02), wu=normal_bf16(s + 5, (d, f), std=0.02),
+            wd=normal_bf16(s + 6, (f, d), std=0.02)))
+    w["gamma"] = np.full(d, 0x3F80, dtype=np.uint16)  # bf16 1.0
+    return w
+
+
+def decoder_tokens(cfg, seed: int = 90):
+    """Token ids and next-token targets, uniform in [0, vocab), [batch, seq]."""
+    B, S, V = cfg["batch"], cfg["seq"], cfg["vocab"]
+    ids = uniform_int32(seed, B * S, 0, V).reshape(B, S)
+    targets = uniform_int32(seed + 1, B * S, 0, V).reshape(B, S)
+    return ids, targets
