@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decoder", action="store_true", help="skip the end-to-end decoder component")
     ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8"], default=None,
                     help="run only one call of the path, `--steps` times, for ncu captures (no JSON line)")
     ap.add_argument("--tokens", type=int, default=M_TOK, help="tokens per call in --profile-case")
@@ -403,6 +404,7 @@ def run_tbik(args):
                        device=dev)
     g_t8 = avg_ms(lambda: tbik.gemm(A, B, T=8, leaf=LEAF, tc=True, out_bf16=True, out=hid2, workspace=gws8))
     tbik.get_error(stream)
+    dec = None if args.no_decoder else decoder_component(dev, stream)
 
     pk = peaks()
     lp_ms = lp_live_ms
@@ -430,6 +432,7 @@ def run_tbik(args):
             "ms": comp_ms,
             "overhead_vs_noninv": {"gemm": g_inv / g_non - 1.0, "logprob": l_inv / l_non - 1.0,
                                    "gemm_ms": [g_inv, g_non], "logprob_ms": [l_inv, l_non]},
+            "decoder_e2e": dec,
         },
         "roofline": {"kernel": "tbik_logprob (fused tcgen05 GEMM + vocab stats, then row tree)",
                      "bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
@@ -452,6 +455,60 @@ def run_tbik(args):
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     return 0
+
+
+def decoder_component(dev, stream):
+    """The end-to-end decoder (4 layers, d 2048, 16 heads of 128, ffn 5632,
+    vocab 32000, batch 8 x seq 2048): forward + target logprobs in tensor-core
+    mode at T = 1 (tokens/s, CUDA events), the attention kernel alone, the
+    bitwise check against T = 8, and the non-invariant baseline's divergence."""
+    import torch
+
+    import invariant_tree_ordered_b200 as tbik
+    from invariant_tree_ordered_b200.decoder import Decoder, DecoderConfig, positions
+
+    cfg = synth.DECODER_FULL
+    w = synth.decoder_weights(cfg)
+    up = lambda a: synth.as_torch_bf16(a).to(dev)  # noqa: E731
+    layers = [{k: up(v) for k, v in L.items()} for L in w["layers"]]
+    dc = DecoderConfig(d=cfg["d"], heads=cfg["heads"], head_dim=cfg["head_dim"], ffn=cfg["ffn"],
+                       vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"])
+    dec = Decoder(dc, up(w["emb"]), up(w["lm_head"]), up(w["gamma"]), layers)
+    ids_h, tg_h = synth.decoder_tokens(cfg)
+    B, S = ids_h.shape
+    ids = torch.from_numpy(ids_h).to(dev)
+    tg = torch.from_numpy(tg_h).to(dev)
+    pos = torch.from_numpy(positions(B, S)).to(dev)
+    fwd = lambda **kw: dec.forward(ids, tg, pos, stream=stream, **kw)  # noqa: E731
+    base = fwd(T=1, tc=True)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 3
+    a.record(stream)
+    for _ in range(n):
+        fwd(T=1, tc=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    t8 = fwd(T=8, tc=True)
+    non1, non8 = fwd(T=1, tc=True, noninv=True), fwd(T=8, tc=True, noninv=True)
+    q = torch.randn(B, S, cfg["heads"], cfg["head_dim"], device=dev).to(torch.bfloat16)
+    tbik.attention(q, q, q, stream=stream)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        tbik.attention(q, q, q, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    att_ms = a.elapsed_time(b) / n
+    att_flop = 4.0 * B * cfg["heads"] * cfg["head_dim"] * (S * (S + 1) / 2)
+    status = tbik.get_error(stream)
+    return {"workload": "4 layers, d 2048, 16x128 heads, ffn 5632, vocab 32000, batch 8 x seq 2048, TC, T=1",
+            "tokens_per_s": B * S / (ms * 1e-3), "ms_per_forward": ms,
+            "bitwise_T1_vs_T8": bool(torch.equal(base.view(torch.int32), t8.view(torch.int32))),
+            "noninv_max_abs_dlogprob_T8_vs_T1": float((non8 - non1).abs().max()),
+            "attention_ms_per_layer": att_ms, "attention_tflops": att_flop / (att_ms * 1e-3) / 1e12,
+            "status": int(status)}
 
 
 def run_profile_case(args):
