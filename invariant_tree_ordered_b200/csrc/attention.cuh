@@ -7,13 +7,13 @@
 // the batch composition or on how heads are split across devices.
 //
 // One warp per query (batch b, head h, position i).  Lane l owns head
-// dimensions [DPL*l, DPL*l + DPL) of the value sums and the keys 2l, 2l+1 of
+// dimensions [DPL*l, DPL*l + DPL) of the value sums and the keys l, l+32 of
 // each chunk:
 //   score   s_j = fl(dot(q_i, k_j) * scale), the dot accumulated over the head
 //           dimension in ascending order with fma from +0;
 //   chunk   m = max of its scores (keys <= i); p_j = exp(s_j - m), 0 past i;
-//           s = the tree over the chunk's 64 slots of p (slots 2l and 2l+1 in
-//           lane l, then xor butterflies); o[d] = ascending sum over the
+//           s = the tree over the chunk's 64 slots of p (xor butterflies over
+//           each half of 32 slots, then the two halves); o[d] = ascending sum over the
 //           chunk's keys of p_j * v_j[d] by fma from +0;
 //   combine (m,s,o) with (m',s',o'): M = max, e = exp(m - M), e' = exp(m' - M),
 //           s = s*e + s'*e', o = o*e + o'*e' (products rounded on their own);
@@ -45,88 +45,108 @@ __device__ __forceinline__ AttNode<DPL> att_combine(const AttNode<DPL>& a, const
     return r;
 }
 
-// dot(q, k) over HD = 32*DPL dimensions, ascending, fma from +0; q held as
-// HD/2 packed bf16 pairs, k read from global memory in 16-byte vectors.
-template <int DPL>
-__device__ __forceinline__ float att_dot(const uint32_t (&qp)[16 * DPL], const uint16_t* __restrict__ k) {
-    float acc = 0.0f;
-    const uint4* kv = reinterpret_cast<const uint4*>(k);
-#pragma unroll
-    for (int c = 0; c < 4 * DPL; ++c) {
-        const uint4 w = __ldg(kv + c);
-        const uint32_t kw[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const uint32_t qw = qp[4 * c + e];
-            acc = __fmaf_rn(__uint_as_float(qw << 16), __uint_as_float(kw[e] << 16), acc);
-            acc = __fmaf_rn(__uint_as_float(qw & 0xffff0000u), __uint_as_float(kw[e] & 0xffff0000u), acc);
-        }
-    }
-    return acc;
-}
-
+// The 8 warps of a CTA take 8 consecutive query positions of one (b, h) and
+// share each key chunk: its K rows (padded to HD/2 + 1 words, so the 32 rows
+// a warp reads at once fall in 32 different banks) and V rows are staged in
+// shared memory once per CTA.  Lane l scores keys l and l + 32 of a chunk;
+// the tree over the 64 slots is the xor butterfly on each half followed by
+// the top-level add of the two halves.
 template <int DPL>
 __global__ void __launch_bounds__(ATT_WARPS * 32)
     attention_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
                      uint16_t* out, int batch, int seq, int heads, float scale) {
     constexpr int HD = 32 * DPL;
+    constexpr int WPR = HD / 2;    // 32-bit words (bf16 pairs) per row
+    constexpr int KSTR = WPR + 1;  // padded K row stride in words
+    __shared__ uint32_t sK[ATT_CHUNK * KSTR];
+    __shared__ __align__(16) uint32_t sV[ATT_CHUNK * WPR];
+    __shared__ uint32_t sQ[ATT_WARPS][WPR];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int qblocks = (seq + ATT_WARPS - 1) / ATT_WARPS;
     const int bh = blockIdx.x / qblocks;
-    const int i = (blockIdx.x - bh * qblocks) * ATT_WARPS + warp;
-    if (i >= seq) return;
+    const int i0 = (blockIdx.x - bh * qblocks) * ATT_WARPS;
+    const int i = i0 + warp;
+    const bool active = i < seq;
     const int b = bh / heads, h = bh - b * heads;
     const size_t row_stride = (size_t)heads * HD;  // elements between positions
     const size_t base = (size_t)b * seq * row_stride + (size_t)h * HD;
-    uint32_t qp[16 * DPL];
-    {
-        const uint4* qv = reinterpret_cast<const uint4*>(q + base + (size_t)i * row_stride);
-#pragma unroll
-        for (int c = 0; c < 4 * DPL; ++c) {
-            const uint4 w = __ldg(qv + c);
-            qp[4 * c] = w.x, qp[4 * c + 1] = w.y, qp[4 * c + 2] = w.z, qp[4 * c + 3] = w.w;
-        }
-    }
-    const int nc = i / ATT_CHUNK + 1;
+    if (active)
+        for (int w = lane; w < WPR; w += 32)
+            sQ[warp][w] = __ldg(reinterpret_cast<const uint32_t*>(q + base + (size_t)i * row_stride) + w);
+    const int last = min(i0 + ATT_WARPS - 1, seq - 1);
+    const int nc_all = last / ATT_CHUNK + 1;  // chunks any warp of this CTA needs
+    const int nc = active ? i / ATT_CHUNK + 1 : 0;
     AttNode<DPL> stk[8];
     int sp = 0;
     AttNode<DPL> fin;
-    for (int c = 0; c < nc; ++c) {
+    fin.m = 0.0f;
+    fin.s = 1.0f;
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) fin.o[d] = 0.0f;
+    // staging: 4 threads per row, WPR/4 words each
+    const int sr = threadIdx.x >> 2, sq = threadIdx.x & 3;
+    for (int c = 0; c < nc_all; ++c) {
         const int j0 = c * ATT_CHUNK;
-        const int ja = j0 + 2 * lane, jb = ja + 1;
-        const bool va = ja <= i, vb = jb <= i;
+        __syncthreads();  // the previous chunk's rows are no longer read
+        if (j0 + sr < seq) {
+            const uint4* kg = reinterpret_cast<const uint4*>(k + base + (size_t)(j0 + sr) * row_stride) + sq * (WPR / 16);
+            const uint4* vg = reinterpret_cast<const uint4*>(v + base + (size_t)(j0 + sr) * row_stride) + sq * (WPR / 16);
+#pragma unroll
+            for (int e = 0; e < WPR / 16; ++e) {
+                const uint4 kw = __ldg(kg + e);
+                uint32_t* kd = sK + sr * KSTR + sq * (WPR / 4) + 4 * e;
+                kd[0] = kw.x, kd[1] = kw.y, kd[2] = kw.z, kd[3] = kw.w;
+                reinterpret_cast<uint4*>(sV + sr * WPR + sq * (WPR / 4))[e] = __ldg(vg + e);
+            }
+        }
+        __syncthreads();
+        if (c >= nc) continue;  // warp-uniform: this query needs fewer chunks
+        const bool va = j0 + lane <= i, vb = j0 + lane + 32 <= i;
         float sa = -INFINITY, sb = -INFINITY;
-        if (va) sa = __fmul_rn(att_dot<DPL>(qp, k + base + (size_t)ja * row_stride), scale);
-        if (vb) sb = __fmul_rn(att_dot<DPL>(qp, k + base + (size_t)jb * row_stride), scale);
+        {
+            float da = 0.0f, db = 0.0f;
+            const uint32_t* ka = sK + lane * KSTR;
+            const uint32_t* kb = sK + (lane + 32) * KSTR;
+#pragma unroll 16
+            for (int w = 0; w < WPR; ++w) {
+                const uint32_t qw = sQ[warp][w];
+                const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
+                const uint32_t a = ka[w], bb = kb[w];
+                da = __fmaf_rn(q0, __uint_as_float(a << 16), da);
+                da = __fmaf_rn(q1, __uint_as_float(a & 0xffff0000u), da);
+                db = __fmaf_rn(q0, __uint_as_float(bb << 16), db);
+                db = __fmaf_rn(q1, __uint_as_float(bb & 0xffff0000u), db);
+            }
+            if (va) sa = __fmul_rn(da, scale);
+            if (vb) sb = __fmul_rn(db, scale);
+        }
         float m = fmaxf(sa, sb);
 #pragma unroll
         for (int w = 1; w < 32; w <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, w));
         const float pa = va ? exp_spec(__fsub_rn(sa, m)) : 0.0f;
         const float pb = vb ? exp_spec(__fsub_rn(sb, m)) : 0.0f;
-        float s = __fadd_rn(pa, pb);  // slots 2l, 2l+1: the bottom level of the tree over 64 slots
+        // tree over the 64 slots: slots 0..31 in pa (lane = slot), 32..63 in pb
+        float ta = pa, tb = pb;
 #pragma unroll
-        for (int w = 1; w < 32; w <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, w));
+        for (int w = 1; w < 32; w <<= 1) {
+            ta = __fadd_rn(ta, __shfl_xor_sync(0xffffffffu, ta, w));
+            tb = __fadd_rn(tb, __shfl_xor_sync(0xffffffffu, tb, w));
+        }
         AttNode<DPL> cur;
         cur.m = m;
-        cur.s = s;
+        cur.s = __fadd_rn(ta, tb);
 #pragma unroll
         for (int d = 0; d < DPL; ++d) cur.o[d] = 0.0f;
         const int nk = min(ATT_CHUNK, i - j0 + 1);
-        const uint16_t* vrow = v + base + (size_t)j0 * row_stride + DPL * lane;
         for (int t = 0; t < nk; ++t) {
-            const float pt = __shfl_sync(0xffffffffu, (t & 1) ? pb : pa, t >> 1);
+            const float pt = __shfl_sync(0xffffffffu, t < 32 ? pa : pb, t & 31);
             float vf[DPL];
-            if (DPL == 4) {
-                const uint2 w = __ldg(reinterpret_cast<const uint2*>(vrow + (size_t)t * row_stride));
-                vf[0] = __uint_as_float(w.x << 16);
-                vf[1] = __uint_as_float(w.x & 0xffff0000u);
-                vf[2] = __uint_as_float(w.y << 16);
-                vf[3] = __uint_as_float(w.y & 0xffff0000u);
-            } else {
-                const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(vrow + (size_t)t * row_stride));
-                vf[0] = __uint_as_float(w << 16);
-                vf[1] = __uint_as_float(w & 0xffff0000u);
+            const uint32_t* vr = sV + t * WPR + (DPL / 2) * lane;
+#pragma unroll
+            for (int e = 0; e < DPL / 2; ++e) {
+                vf[2 * e] = __uint_as_float(vr[e] << 16);
+                vf[2 * e + 1] = __uint_as_float(vr[e] & 0xffff0000u);
             }
 #pragma unroll
             for (int d = 0; d < DPL; ++d) cur.o[d] = __fmaf_rn(pt, vf[d], cur.o[d]);
@@ -139,6 +159,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32)
         else
             stk[sp++] = cur;
     }
+    if (!active) return;
     uint16_t* o = out + base + (size_t)i * row_stride + DPL * lane;
     float r[DPL];
 #pragma unroll
