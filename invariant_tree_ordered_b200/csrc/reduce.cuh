@@ -121,47 +121,71 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
     }
 }
 
-// Rotate-half RoPE: thread = (tensor, token, head, group of 8 pairs), grid-
-// stride loop; item indices in IDX (32-bit when they fit, for cheap division).
-// Each product is rounded on its own (no fma), then one bf16 rounding.
+// Rotate-half RoPE: thread = (token, head, group of 8 pairs) of both q and k,
+// grid-stride loop; the table row of the token's position is read once for
+// both tensors.  Item indices in IDX (32-bit when they fit, for cheap
+// division).  Each product is rounded on its own (no fma), then one bf16
+// rounding.
+__device__ __forceinline__ void rope8(const uint4& w1, const uint4& w2, const float4 (&cs)[4], uint4& r1, uint4& r2) {
+    float x1[8], x2[8], o1[8], o2[8];
+    unpack8(w1, x1);
+    unpack8(w2, x2);
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+        const float c0 = cs[e2].x, s0 = cs[e2].y, c1 = cs[e2].z, s1 = cs[e2].w;  // (c, s) of two consecutive i
+        const int a = 2 * e2, b = 2 * e2 + 1;
+        o1[a] = __fsub_rn(__fmul_rn(x1[a], c0), __fmul_rn(x2[a], s0));
+        o2[a] = __fadd_rn(__fmul_rn(x2[a], c0), __fmul_rn(x1[a], s0));
+        o1[b] = __fsub_rn(__fmul_rn(x1[b], c1), __fmul_rn(x2[b], s1));
+        o2[b] = __fadd_rn(__fmul_rn(x2[b], c1), __fmul_rn(x1[b], s1));
+    }
+    r1 = pack8(o1);
+    r2 = pack8(o2);
+}
+
 template <typename IDX>
 __global__ void rope_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, uint16_t* q_out,
                             uint16_t* k_out, const int32_t* __restrict__ pos, const float* __restrict__ table,
                             int tokens, int heads, int head_dim, int max_pos) {
-    const uint16_t* x = blockIdx.y == 0 ? q : k;
-    uint16_t* o = blockIdx.y == 0 ? q_out : k_out;
-    if (x == nullptr) return;
     const IDX half = (IDX)(head_dim >> 1);
     const IDX gph = half >> 3;
     const IDX total = (IDX)tokens * (IDX)heads * gph;
+    const bool hq = q != nullptr, hk = k != nullptr;
+    const uint4 nan4 = make_uint4(0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u, 0x7fc07fc0u);
     for (IDX i = blockIdx.x * (IDX)blockDim.x + threadIdx.x; i < total; i += (IDX)gridDim.x * blockDim.x) {
         const IDX th = i / gph;
         const int g = (int)(i - th * gph);
         const int token = (int)(th / (IDX)heads);
-        const size_t hb = (size_t)th * head_dim;
+        const size_t o1 = (size_t)th * head_dim + 8 * g, o2 = o1 + half;
+        uint4 a1, a2, b1, b2;
+        if (hq) {
+            a1 = __ldg(reinterpret_cast<const uint4*>(q + o1));
+            a2 = __ldg(reinterpret_cast<const uint4*>(q + o2));
+        }
+        if (hk) {
+            b1 = __ldg(reinterpret_cast<const uint4*>(k + o1));
+            b2 = __ldg(reinterpret_cast<const uint4*>(k + o2));
+        }
         const int p = __ldg(pos + token);
-        float x1[8], x2[8], o1[8], o2[8];
-        unpack8(__ldg(reinterpret_cast<const uint4*>(x + hb + 8 * g)), x1);
-        unpack8(__ldg(reinterpret_cast<const uint4*>(x + hb + half + 8 * g)), x2);
+        uint4 ra1 = nan4, ra2 = nan4, rb1 = nan4, rb2 = nan4;
         if (p < 0 || p >= max_pos) {
             set_error(TBIK_ERR_POSITION);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o1[e] = o2[e] = __int_as_float(0x7fc00000);
         } else {
-            const float4* cs = reinterpret_cast<const float4*>(table + ((size_t)p * half + 8 * g) * 2);
+            const float4* row = reinterpret_cast<const float4*>(table + ((size_t)p * half + 8 * g) * 2);
+            float4 cs[4];
 #pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-                const float4 t = __ldg(cs + e2);  // (c, s) of two consecutive i
-                const float c0 = t.x, s0 = t.y, c1 = t.z, s1 = t.w;
-                const int a = 2 * e2, b = 2 * e2 + 1;
-                o1[a] = __fsub_rn(__fmul_rn(x1[a], c0), __fmul_rn(x2[a], s0));
-                o2[a] = __fadd_rn(__fmul_rn(x2[a], c0), __fmul_rn(x1[a], s0));
-                o1[b] = __fsub_rn(__fmul_rn(x1[b], c1), __fmul_rn(x2[b], s1));
-                o2[b] = __fadd_rn(__fmul_rn(x2[b], c1), __fmul_rn(x1[b], s1));
-            }
+            for (int e2 = 0; e2 < 4; ++e2) cs[e2] = __ldg(row + e2);
+            if (hq) rope8(a1, a2, cs, ra1, ra2);
+            if (hk) rope8(b1, b2, cs, rb1, rb2);
         }
-        *reinterpret_cast<uint4*>(o + hb + 8 * g) = pack8(o1);
-        *reinterpret_cast<uint4*>(o + hb + half + 8 * g) = pack8(o2);
+        if (hq) {
+            *reinterpret_cast<uint4*>(q_out + o1) = ra1;
+            *reinterpret_cast<uint4*>(q_out + o2) = ra2;
+        }
+        if (hk) {
+            *reinterpret_cast<uint4*>(k_out + o1) = rb1;
+            *reinterpret_cast<uint4*>(k_out + o2) = rb2;
+        }
     }
 }
 

@@ -622,10 +622,10 @@ tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) 
         if (blocks > info->sms * 16) blocks = info->sms * 16;
         const size_t stride = (size_t)blocks * 256;
         if (work + stride < (1ull << 32))  // every index the loop forms fits 32 bits
-            rope_kernel<uint32_t><<<dim3(blocks, 2), 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table,
+            rope_kernel<uint32_t><<<blocks, 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table,
                                                                   a->tokens, a->heads, a->head_dim, a->max_pos);
         else
-            rope_kernel<size_t><<<dim3(blocks, 2), 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table,
+            rope_kernel<size_t><<<blocks, 256, 0, s>>>(a->q, a->k, a->q_out, a->k_out, a->pos, a->table,
                                                                 a->tokens, a->heads, a->head_dim, a->max_pos);
         if ((st = launch_status()) != TBIK_OK) return st;
     }
