@@ -45,12 +45,16 @@ __device__ __forceinline__ AttNode<DPL> att_combine(const AttNode<DPL>& a, const
     return r;
 }
 
-// The 8 warps of a CTA take 8 consecutive query positions of one (b, h) and
-// share each key chunk: its K rows (padded to HD/2 + 1 words, so the 32 rows
-// a warp reads at once fall in 32 different banks) and V rows are staged in
-// shared memory once per CTA.  Lane l scores keys l and l + 32 of a chunk;
-// the tree over the 64 slots is the xor butterfly on each half followed by
-// the top-level add of the two halves.
+// A warp takes QPW consecutive query positions (independent fma chains for
+// the same key rows); the ATT_WARPS warps of a CTA take ATT_WARPS * QPW
+// consecutive positions of one (b, h) and share each key chunk: its K rows
+// (padded to HD/2 + 1 words, so the 32 rows a warp reads at once fall in 32
+// different banks) and V rows are staged in shared memory once per CTA.
+// Lane l scores keys l and l + 32 of a chunk; the tree over the 64 slots is
+// the xor butterfly on each half followed by the top-level add of the halves.
+constexpr int ATT_QPW = 2;
+constexpr int ATT_QPB = ATT_WARPS * ATT_QPW;  // query positions per CTA
+
 template <int DPL>
 __global__ void __launch_bounds__(ATT_WARPS * 32)
     attention_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
@@ -58,89 +62,111 @@ __global__ void __launch_bounds__(ATT_WARPS * 32)
     constexpr int HD = 32 * DPL;
     constexpr int WPR = HD / 2;    // 32-bit words (bf16 pairs) per row
     constexpr int KSTR = WPR + 1;  // padded K row stride in words
+    constexpr int Q = ATT_QPW;
     __shared__ uint32_t sK[ATT_CHUNK * KSTR];
     __shared__ __align__(16) uint32_t sV[ATT_CHUNK * WPR];
-    __shared__ uint32_t sQ[ATT_WARPS][WPR];
+    __shared__ uint32_t sQ[ATT_WARPS][Q][WPR];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int qblocks = (seq + ATT_WARPS - 1) / ATT_WARPS;
+    const int qblocks = (seq + ATT_QPB - 1) / ATT_QPB;
     const int bh = blockIdx.x / qblocks;
-    const int i0 = (blockIdx.x - bh * qblocks) * ATT_WARPS;
-    const int i = i0 + warp;
-    const bool active = i < seq;
+    const int i0 = (blockIdx.x - bh * qblocks) * ATT_QPB;
     const int b = bh / heads, h = bh - b * heads;
     const size_t row_stride = (size_t)heads * HD;  // elements between positions
     const size_t base = (size_t)b * seq * row_stride + (size_t)h * HD;
-    if (active)
-        for (int w = lane; w < WPR; w += 32)
-            sQ[warp][w] = __ldg(reinterpret_cast<const uint32_t*>(q + base + (size_t)i * row_stride) + w);
-    const int last = min(i0 + ATT_WARPS - 1, seq - 1);
-    const int nc_all = last / ATT_CHUNK + 1;  // chunks any warp of this CTA needs
-    const int nc = active ? i / ATT_CHUNK + 1 : 0;
-    AttNode<DPL> stk[8];
-    int sp = 0;
-    AttNode<DPL> fin;
-    fin.m = 0.0f;
-    fin.s = 1.0f;
+    int qi[Q], nc[Q];
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) fin.o[d] = 0.0f;
+    for (int x = 0; x < Q; ++x) {
+        qi[x] = i0 + Q * warp + x;
+        nc[x] = qi[x] < seq ? qi[x] / ATT_CHUNK + 1 : 0;
+        if (qi[x] < seq)
+            for (int w = lane; w < WPR; w += 32)
+                sQ[warp][x][w] = __ldg(reinterpret_cast<const uint32_t*>(q + base + (size_t)qi[x] * row_stride) + w);
+    }
+    const int last = min(i0 + ATT_QPB - 1, seq - 1);
+    const int nc_all = last / ATT_CHUNK + 1;  // chunks any query of this CTA needs
+    const int qlast = min(qi[Q - 1], seq - 1);  // this warp's last position (qi[0] < seq if any is active)
+    const int nc_w = qi[0] < seq ? qlast / ATT_CHUNK + 1 : 0;  // chunks this warp needs
+    AttNode<DPL> stk[Q][8];
+    int sp[Q];
+    AttNode<DPL> fin[Q];
+#pragma unroll
+    for (int x = 0; x < Q; ++x) {
+        sp[x] = 0;
+        fin[x].m = 0.0f;
+        fin[x].s = 1.0f;
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) fin[x].o[d] = 0.0f;
+    }
     // staging: 4 threads per row, WPR/4 words each
-    const int sr = threadIdx.x >> 2, sq = threadIdx.x & 3;
+    const int sr = threadIdx.x >> 2, sq4 = threadIdx.x & 3;
     for (int c = 0; c < nc_all; ++c) {
         const int j0 = c * ATT_CHUNK;
         __syncthreads();  // the previous chunk's rows are no longer read
         if (j0 + sr < seq) {
-            const uint4* kg = reinterpret_cast<const uint4*>(k + base + (size_t)(j0 + sr) * row_stride) + sq * (WPR / 16);
-            const uint4* vg = reinterpret_cast<const uint4*>(v + base + (size_t)(j0 + sr) * row_stride) + sq * (WPR / 16);
+            const uint4* kg = reinterpret_cast<const uint4*>(k + base + (size_t)(j0 + sr) * row_stride) + sq4 * (WPR / 16);
+            const uint4* vg = reinterpret_cast<const uint4*>(v + base + (size_t)(j0 + sr) * row_stride) + sq4 * (WPR / 16);
 #pragma unroll
             for (int e = 0; e < WPR / 16; ++e) {
                 const uint4 kw = __ldg(kg + e);
-                uint32_t* kd = sK + sr * KSTR + sq * (WPR / 4) + 4 * e;
+                uint32_t* kd = sK + sr * KSTR + sq4 * (WPR / 4) + 4 * e;
                 kd[0] = kw.x, kd[1] = kw.y, kd[2] = kw.z, kd[3] = kw.w;
-                reinterpret_cast<uint4*>(sV + sr * WPR + sq * (WPR / 4))[e] = __ldg(vg + e);
+                reinterpret_cast<uint4*>(sV + sr * WPR + sq4 * (WPR / 4))[e] = __ldg(vg + e);
             }
         }
         __syncthreads();
-        if (c >= nc) continue;  // warp-uniform: this query needs fewer chunks
-        const bool va = j0 + lane <= i, vb = j0 + lane + 32 <= i;
-        float sa = -INFINITY, sb = -INFINITY;
+        if (c >= nc_w) continue;  // warp-uniform: no query of this warp needs this chunk
+        float da[Q], db[Q];
+#pragma unroll
+        for (int x = 0; x < Q; ++x) da[x] = db[x] = 0.0f;
         {
-            float da = 0.0f, db = 0.0f;
             const uint32_t* ka = sK + lane * KSTR;
             const uint32_t* kb = sK + (lane + 32) * KSTR;
-#pragma unroll 16
+#pragma unroll 8
             for (int w = 0; w < WPR; ++w) {
-                const uint32_t qw = sQ[warp][w];
-                const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
                 const uint32_t a = ka[w], bb = kb[w];
-                da = __fmaf_rn(q0, __uint_as_float(a << 16), da);
-                da = __fmaf_rn(q1, __uint_as_float(a & 0xffff0000u), da);
-                db = __fmaf_rn(q0, __uint_as_float(bb << 16), db);
-                db = __fmaf_rn(q1, __uint_as_float(bb & 0xffff0000u), db);
+                const float a0 = __uint_as_float(a << 16), a1 = __uint_as_float(a & 0xffff0000u);
+                const float b0 = __uint_as_float(bb << 16), b1 = __uint_as_float(bb & 0xffff0000u);
+#pragma unroll
+                for (int x = 0; x < Q; ++x) {
+                    const uint32_t qw = sQ[warp][x][w];
+                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
+                    da[x] = __fmaf_rn(q0, a0, da[x]);
+                    da[x] = __fmaf_rn(q1, a1, da[x]);
+                    db[x] = __fmaf_rn(q0, b0, db[x]);
+                    db[x] = __fmaf_rn(q1, b1, db[x]);
+                }
             }
-            if (va) sa = __fmul_rn(da, scale);
-            if (vb) sb = __fmul_rn(db, scale);
         }
-        float m = fmaxf(sa, sb);
+        float pa[Q], pb[Q];
+        AttNode<DPL> cur[Q];
 #pragma unroll
-        for (int w = 1; w < 32; w <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, w));
-        const float pa = va ? exp_spec(__fsub_rn(sa, m)) : 0.0f;
-        const float pb = vb ? exp_spec(__fsub_rn(sb, m)) : 0.0f;
-        // tree over the 64 slots: slots 0..31 in pa (lane = slot), 32..63 in pb
-        float ta = pa, tb = pb;
+        for (int x = 0; x < Q; ++x) {
+            const int i = qi[x];
+            const bool va = j0 + lane <= i, vb = j0 + lane + 32 <= i;
+            const float sa = va ? __fmul_rn(da[x], scale) : -INFINITY;
+            const float sb = vb ? __fmul_rn(db[x], scale) : -INFINITY;
+            float m = fmaxf(sa, sb);
 #pragma unroll
-        for (int w = 1; w < 32; w <<= 1) {
-            ta = __fadd_rn(ta, __shfl_xor_sync(0xffffffffu, ta, w));
-            tb = __fadd_rn(tb, __shfl_xor_sync(0xffffffffu, tb, w));
+            for (int w = 1; w < 32; w <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, w));
+            pa[x] = va ? exp_spec(__fsub_rn(sa, m)) : 0.0f;
+            pb[x] = vb ? exp_spec(__fsub_rn(sb, m)) : 0.0f;
+            // tree over the 64 slots: slots 0..31 in pa (lane = slot), 32..63 in pb
+            float ta = pa[x], tb = pb[x];
+#pragma unroll
+            for (int w = 1; w < 32; w <<= 1) {
+                ta = __fadd_rn(ta, __shfl_xor_sync(0xffffffffu, ta, w));
+                tb = __fadd_rn(tb, __shfl_xor_sync(0xffffffffu, tb, w));
+            }
+            cur[x].m = m;
+            cur[x].s = __fadd_rn(ta, tb);
+#pragma unroll
+            for (int d = 0; d < DPL; ++d) cur[x].o[d] = 0.0f;
         }
-        AttNode<DPL> cur;
-        cur.m = m;
-        cur.s = __fadd_rn(ta, tb);
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) cur.o[d] = 0.0f;
-        const int nk = min(ATT_CHUNK, i - j0 + 1);
-        for (int t = 0; t < nk; ++t) {
-            const float pt = __shfl_sync(0xffffffffu, t < 32 ? pa : pb, t & 31);
+        // o: ascending over the chunk's keys; a query whose chunk is partial
+        // (or past its position) stops early: keys past i add nothing
+        const int nk_max = min(ATT_CHUNK, qlast - j0 + 1);
+        for (int t = 0; t < nk_max; ++t) {
             float vf[DPL];
             const uint32_t* vr = sV + t * WPR + (DPL / 2) * lane;
 #pragma unroll
@@ -149,25 +175,38 @@ __global__ void __launch_bounds__(ATT_WARPS * 32)
                 vf[2 * e + 1] = __uint_as_float(vr[e] & 0xffff0000u);
             }
 #pragma unroll
-            for (int d = 0; d < DPL; ++d) cur.o[d] = __fmaf_rn(pt, vf[d], cur.o[d]);
-        }
-        // the chunk tree, streamed: pop the pending left siblings of every node closing here
-        const LeafOps ops = leaf_ops(nc, c);
-        for (int n = leaf_pops(ops); n > 0; --n) cur = att_combine<DPL>(stk[--sp], cur);
-        if (ops.final_)
-            fin = cur;
-        else
-            stk[sp++] = cur;
-    }
-    if (!active) return;
-    uint16_t* o = out + base + (size_t)i * row_stride + DPL * lane;
-    float r[DPL];
+            for (int x = 0; x < Q; ++x) {
+                const float pt = __shfl_sync(0xffffffffu, t < 32 ? pa[x] : pb[x], t & 31);
+                if (j0 + t <= qi[x]) {
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) r[d] = __fdiv_rn(fin.o[d], fin.s);
-    if (DPL == 4) {
-        *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf2(r[0], r[1]), pack_bf2(r[2], r[3]));
-    } else {
-        *reinterpret_cast<uint32_t*>(o) = pack_bf2(r[0], r[1]);
+                    for (int d = 0; d < DPL; ++d) cur[x].o[d] = __fmaf_rn(pt, vf[d], cur[x].o[d]);
+                }
+            }
+        }
+        // the chunk tree of each query, streamed: pop the pending left siblings of every node closing here
+#pragma unroll
+        for (int x = 0; x < Q; ++x) {
+            if (c >= nc[x]) continue;
+            const LeafOps ops = leaf_ops(nc[x], c);
+            for (int n = leaf_pops(ops); n > 0; --n) cur[x] = att_combine<DPL>(stk[x][--sp[x]], cur[x]);
+            if (ops.final_)
+                fin[x] = cur[x];
+            else
+                stk[x][sp[x]++] = cur[x];
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < Q; ++x) {
+        if (qi[x] >= seq) continue;
+        uint16_t* o = out + base + (size_t)qi[x] * row_stride + DPL * lane;
+        float r[DPL];
+#pragma unroll
+        for (int d = 0; d < DPL; ++d) r[d] = __fdiv_rn(fin[x].o[d], fin[x].s);
+        if (DPL == 4) {
+            *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf2(r[0], r[1]), pack_bf2(r[2], r[3]));
+        } else {
+            *reinterpret_cast<uint32_t*>(o) = pack_bf2(r[0], r[1]);
+        }
     }
 }
 

@@ -567,7 +567,7 @@ tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const uint16_t*
     if (batch == 0 || seq == 0) return TBIK_OK;
     if (!q || !k || !v || !out) return TBIK_ERR_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TBIK_ERR_ALIGN;
-    const long long blocks = (long long)batch * heads * ((seq + ATT_WARPS - 1) / ATT_WARPS);
+    const long long blocks = (long long)batch * heads * ((seq + ATT_QPB - 1) / ATT_QPB);
     if (blocks > 0x7fffffffLL) return TBIK_ERR_SHAPE;
     const float scale = (float)(1.0 / std::sqrt((double)head_dim));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
