@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(ATT_WARPS * 32)
     constexpr int Q = ATT_QPW;
     __shared__ uint32_t sK[ATT_CHUNK * KSTR];
     __shared__ __align__(16) uint32_t sV[ATT_CHUNK * WPR];
-    __shared__ uint32_t sQ[ATT_WARPS][Q][WPR];
+    __shared__ __align__(8) float2 sQ[ATT_WARPS][Q][WPR];  // the queries widened to fp32 (exact), pairs
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int qblocks = (seq + ATT_QPB - 1) / ATT_QPB;
@@ -80,8 +80,10 @@ __global__ void __launch_bounds__(ATT_WARPS * 32)
         qi[x] = i0 + Q * warp + x;
         nc[x] = qi[x] < seq ? qi[x] / ATT_CHUNK + 1 : 0;
         if (qi[x] < seq)
-            for (int w = lane; w < WPR; w += 32)
-                sQ[warp][x][w] = __ldg(reinterpret_cast<const uint32_t*>(q + base + (size_t)qi[x] * row_stride) + w);
+            for (int w = lane; w < WPR; w += 32) {
+                const uint32_t qw = __ldg(reinterpret_cast<const uint32_t*>(q + base + (size_t)qi[x] * row_stride) + w);
+                sQ[warp][x][w] = make_float2(__uint_as_float(qw << 16), __uint_as_float(qw & 0xffff0000u));
+            }
     }
     const int last = min(i0 + ATT_QPB - 1, seq - 1);
     const int nc_all = last / ATT_CHUNK + 1;  // chunks any query of this CTA needs
@@ -129,8 +131,8 @@ __global__ void __launch_bounds__(ATT_WARPS * 32)
                 const float b0 = __uint_as_float(bb << 16), b1 = __uint_as_float(bb & 0xffff0000u);
 #pragma unroll
                 for (int x = 0; x < Q; ++x) {
-                    const uint32_t qw = sQ[warp][x][w];
-                    const float q0 = __uint_as_float(qw << 16), q1 = __uint_as_float(qw & 0xffff0000u);
+                    const float2 qf = sQ[warp][x][w];
+                    const float q0 = qf.x, q1 = qf.y;
                     da[x] = __fmaf_rn(q0, a0, da[x]);
                     da[x] = __fmaf_rn(q1, a1, da[x]);
                     db[x] = __fmaf_rn(q0, b0, db[x]);
