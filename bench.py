@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decoder", action="store_true", help="skip the end-to-end decoder component")
-    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8"], default=None,
+    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "attention"], default=None,
                     help="run only one call of the path, `--steps` times, for ncu captures (no JSON line)")
     ap.add_argument("--tokens", type=int, default=M_TOK, help="tokens per call in --profile-case")
     return ap.parse_args()
@@ -519,7 +519,14 @@ def run_profile_case(args):
 
     dev = torch.device("cuda", 0)
     M = args.tokens
-    if args.profile_case == "logprob":
+    if args.profile_case == "attention":
+        # decoder attention: sequences of 2048 positions, 16 heads of 128; --tokens = batch * 2048
+        S, NH, D = 2048, 16, 128
+        Bq = max(1, M // S)
+        qkv = [synth.as_torch_bf16(synth.normal_bf16(450 + i, (Bq, S, NH, D))).to(dev) for i in range(3)]
+        out = torch.empty_like(qkv[0])
+        call = lambda: tbik.attention(*qkv, out=out)  # noqa: E731
+    elif args.profile_case == "logprob":
         h = synth.as_torch_bf16(synth.normal_bf16(30, (M, H))).to(dev)
         w = synth.as_torch_bf16(synth.normal_bf16(31, (V, H), std=0.02)).to(dev)
         t = torch.from_numpy(synth.uniform_int32(32, M, 0, V)).to(dev)
