@@ -14,9 +14,10 @@
 // CTA r holds rows [128r, 128r+128) of A and rows/columns [64r, 64r+64) of B
 // in its shared memory and its own 128 x 128 fp32 accumulators in TMEM.  The
 // leader (rank 0) issues the MMAs; commits arrive on both CTAs' barriers.
-// Each CTA (320 threads, one per SM, persistent over work units):
+// Each CTA (352 threads, one per SM, persistent over work units):
 //   warp 0     TMA producer: its A and B halves, 128 deep (two 64-wide
-//              128-byte-swizzle slices), into a 3-stage ring
+//              128-byte-swizzle slices), into a ring of 3 stages (up to 8
+//              when M is small and only the valid A rows are copied)
 //   warp 1     TMEM allocator (both CTAs) + MMA issuer (leader, lane 0)
 //   warps 2-9  epilogue: drain each leaf from TMEM and apply the tree; warp w
 //              reads TMEM lanes 32*(w%4).. (its row quadrant) and the 64
@@ -27,13 +28,15 @@
 //              tensor pipe a few hundred cycles even when the barrier is
 //              already complete; a named barrier between two warps costs
 //              nothing, so the issuer only issues MMAs and commits.
-// TMEM (512 columns): three leaf accumulators (columns 0, 128, 256), so the
-// epilogue has two leaf-times to drain one, and a slot at column 384.  Pending
-// subtree results wait by size: a single leaf stays in its own accumulator
-// (it is always consumed by the next leaf, which releases both buffers); 2
-// leaves in the TMEM slot; 3-4 leaves in one shared-memory slot; >= 5 leaves in
-// a per-CTA fp32 scratch in global memory that stays in L2.  At most one value
-// of each of the first three classes is pending at a time.
+// TMEM (512 columns): three leaf accumulators (columns 0, 128, 256) and a slot
+// at column 384.  Pending subtree results wait by size: a single leaf stays in
+// its own accumulator (it is always consumed by the next leaf); 2 leaves in
+// the TMEM slot; 3-4 leaves in one shared-memory slot; >= 5 leaves in a
+// per-CTA fp32 scratch in global memory that stays in L2.  At most one value
+// of each of the first three classes is pending at a time.  The epilogue
+// handles a leaf in two phases: it first drains the leaf (and the single leaf
+// it pops) into registers and releases both accumulators, then does the other
+// pops and the push, so the MMA never waits on the rest of the tree work.
 // A work unit is (m tile, n tile, frontier node f): the node's subtree of
 // leaves is reduced by this pair; with more than one frontier node per tile the
 // subtree results go to fp32 partial buffers that a combine kernel reduces
