@@ -465,12 +465,16 @@ def decoder_component(dev, stream):
     import torch
 
     import invariant_tree_ordered_b200 as tbik
-    from invariant_tree_ordered_b200.decoder import Decoder, DecoderConfig, positions
+    from invariant_tree_ordered_b200.decoder import Decoder, DecoderConfig, interleave_gate_up, positions
 
     cfg = synth.DECODER_FULL
     w = synth.decoder_weights(cfg)
     up = lambda a: synth.as_torch_bf16(a).to(dev)  # noqa: E731
-    layers = [{k: up(v) for k, v in L.items()} for L in w["layers"]]
+    layers = []
+    for L in w["layers"]:
+        dl = {k: up(L[k]) for k in ("wq", "wk", "wv", "wo", "wd")}
+        dl["wgu"] = up(interleave_gate_up(L["wg"], L["wu"]))
+        layers.append(dl)
     dc = DecoderConfig(d=cfg["d"], heads=cfg["heads"], head_dim=cfg["head_dim"], ffn=cfg["ffn"],
                        vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"])
     dec = Decoder(dc, up(w["emb"]), up(w["lm_head"]), up(w["gamma"]), layers)

@@ -87,6 +87,13 @@ typedef enum {
 /* Output type of tbik_gemm: */
 #define TBIK_OUT_F32 0x000u  /* C fp32 [M,N] */
 #define TBIK_OUT_BF16 0x100u /* C bf16 [M,N], rounded once (RNE) from the fp32 tree root */
+/* Gate/up projection fused with SwiGLU: B's N = 2F columns hold the gate and
+   up weights interleaved in blocks of 32 (columns [64j, 64j+32) = gate
+   features [32j, 32j+32), columns [64j+32, 64j+64) = up features of the same
+   features); C is bf16 [M, F] = bf16((g / (1 + exp(-g))) * u) from the fp32
+   tree roots g, u (the library's exp specification, no rounding before the
+   output).  F % 32 == 0.  Not combinable with TBIK_NONINV; implies bf16 C. */
+#define TBIK_SWIGLU_OUT 0x200u
 
 /* Vocabulary columns per logprob leaf, and the largest shard count the vocab
    padding is sized for: V is padded to Vpad = ceil(V / (64*8)) * 64*8 with

@@ -35,6 +35,7 @@ B_KN = 0x00
 B_NK = 0x10
 OUT_F32 = 0x000
 OUT_BF16 = 0x100
+SWIGLU_OUT = 0x200
 DEBUG_WITHHOLD_ACC_ARRIVE = 0x1
 DEBUG_SWAP_MN_STRIDES = 0x2
 VOCAB_LEAF = 64
@@ -161,8 +162,10 @@ def gemm_workspace(M, N, K, T, leaf, mode) -> int:
 
 
 def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = False, b_nk: bool = False,
-         out_bf16: bool = False, out=None, workspace=None, stream=None):
-    """C = A @ B with the K reduction in tree order (see tbik_gemm in tbik.h)."""
+         out_bf16: bool = False, swiglu: bool = False, out=None, workspace=None, stream=None):
+    """C = A @ B with the K reduction in tree order (see tbik_gemm in tbik.h).
+    swiglu: B holds gate/up columns interleaved in blocks of 32 and C is the
+    bf16 SwiGLU [M, N/2] of the fp32 roots (TBIK_SWIGLU_OUT)."""
     torch = _torch()
     lib = load_library()
     _need(A, torch.bfloat16, "A")
@@ -173,8 +176,13 @@ def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = F
     if kb != K:
         raise ValueError("inner dimensions differ")
     mode = (TC if tc else EXACT) | (NONINV if noninv else 0) | (B_NK if b_nk else B_KN) | (OUT_BF16 if out_bf16 else OUT_F32)
+    if swiglu:
+        mode |= SWIGLU_OUT
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16 if out_bf16 else torch.float32, device=A.device)
+        if swiglu:
+            out = torch.empty((M, N // 2), dtype=torch.bfloat16, device=A.device)
+        else:
+            out = torch.empty((M, N), dtype=torch.bfloat16 if out_bf16 else torch.float32, device=A.device)
     ws, wsb = _workspace(lib.tbik_gemm_workspace(M, N, K, T, leaf, mode), A.device, workspace)
     _check(lib.tbik_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, T, leaf, mode, _ptr(ws), wsb,
                          _stream_handle(stream)), "tbik_gemm")

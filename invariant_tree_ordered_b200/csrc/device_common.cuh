@@ -36,6 +36,25 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&b);
 }
 
+// eight bf16 values in a 16-byte vector <-> fp32 (exact widening; RNE narrowing)
+__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
+    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(a[i] << 16);
+        f[2 * i + 1] = __uint_as_float(a[i] & 0xffff0000u);
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+    uint4 w;
+    w.x = pack_bf2(f[0], f[1]);
+    w.y = pack_bf2(f[2], f[3]);
+    w.z = pack_bf2(f[4], f[5]);
+    w.w = pack_bf2(f[6], f[7]);
+    return w;
+}
+
 // ----------------------------------------------------- exp / log specs
 // Cody-Waite style specifications (W. J. Cody and W. Waite, "Software Manual
 // for the Elementary Functions", 1980): additive reduction by a split ln 2 and
@@ -73,6 +92,17 @@ __device__ __forceinline__ float exp_spec(float x) {
     const int k1 = k / 2;
     const int k2 = k - k1;
     return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));
+}
+
+// SwiGLU of one element in fp32: (g / (1 + exp(-g))) * u, each step one
+// correctly rounded operation (rounding-location alignment article, winzheng.jp,
+// section "外科手術的な修正：3つのノード": fp32 intermediates, one rounding at the
+// output, which the caller applies).
+__device__ __forceinline__ float swiglu1(float g, float u) {
+    const float e = exp_spec(-g);
+    const float den = __fadd_rn(1.0f, e);
+    const float sg = __fdiv_rn(g, den);
+    return __fmul_rn(sg, u);
 }
 
 // 2^y through the hardware base-2 exponential (ex2.approx, denormal results

@@ -80,6 +80,7 @@ struct TcParams {
     int total_units;
     int direct;       // 1: write final C; 0: write partials[f]
     int out_bf16;
+    int swiglu;       // 1: C = bf16 SwiGLU of the interleaved gate/up roots, [M, N/2] (direct only)
     void* out;        // C [M,N]
     float* partials;  // [F][M][N]
     float* scratch;   // [gridDim.x][gs][128*128], layout per slot [col/4][row][4]
@@ -482,6 +483,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                             scratch_st(scratch_slot(p, g_after), c, rt, v[cc]);
                     }
                     if (cls == 1) tmem_wait_st();
+                } else if (EPI == EPI_TREE && p.swiglu) {
+                    // this warp's 64 columns: gate features f0..f0+31 (chunk 0)
+                    // and the up values of the same features (chunk 1)
+                    if (row < p.M) {
+                        const int f0 = tn * (TC_BN / 2) + half * 32;
+                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                                              (size_t)row * (p.N / 2) + f0);
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            float o[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) o[e] = swiglu1(v[0][8 * q8 + e], v[1][8 * q8 + e]);
+                            if (f0 + 8 * q8 < p.N / 2) dst[q8] = pack8(o);
+                        }
+                    }
                 } else if (EPI == EPI_TREE) {
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {

@@ -9,24 +9,6 @@
 
 namespace tbik {
 
-__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
-    const uint32_t a[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(a[i] << 16);
-        f[2 * i + 1] = __uint_as_float(a[i] & 0xffff0000u);
-    }
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
-    uint4 w;
-    w.x = pack_bf2(f[0], f[1]);
-    w.y = pack_bf2(f[2], f[3]);
-    w.z = pack_bf2(f[4], f[5]);
-    w.w = pack_bf2(f[6], f[7]);
-    return w;
-}
-
 // NT = H/(8*LPT) threads per token; thread t owns the LPT consecutive leaves
 // [LPT*t, LPT*t + LPT) (leaf = 8 elements, one 16-byte vector per tensor).
 // The leaf sums form a power-of-two pairwise tree: the lowest log2(LPT)
@@ -189,12 +171,6 @@ __global__ void rope_kernel(const uint16_t* __restrict__ q, const uint16_t* __re
     }
 }
 
-__device__ __forceinline__ float swiglu1(float g, float u) {
-    const float e = exp_spec(-g);
-    const float den = __fadd_rn(1.0f, e);
-    const float sg = __fdiv_rn(g, den);
-    return __fmul_rn(sg, u);
-}
 
 // out = bf16((g / (1 + exp(-g))) * u), one 8-element vector per thread per
 // iteration of a grid-stride loop; the next iteration's inputs are loaded
@@ -259,6 +235,31 @@ __global__ void swiglu_kernel(const void* __restrict__ g, const void* __restrict
         i = inext;
         cg = ng;
         cu = nu;
+    }
+}
+
+// SwiGLU over an fp32 [M, 2F] matrix whose columns hold gate and up values
+// interleaved in blocks of 32 (the fused gate/up layout); out bf16 [M, F].
+// Thread = 8 consecutive features of one row.
+__global__ void swiglu_interleaved_kernel(const float* __restrict__ gu, uint16_t* out, int M, int F) {
+    const long long per_row = F / 8;
+    const long long total = (long long)M * per_row;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(e / per_row);
+        const int f0 = (int)(e - (long long)m * per_row) * 8;
+        const float* row = gu + (size_t)m * 2 * F;
+        const int gcol = (f0 / 32) * 64 + (f0 % 32);
+        float g[8], u[8], o[8];
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(row + gcol));
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(row + gcol + 4));
+        const float4 u0 = __ldg(reinterpret_cast<const float4*>(row + gcol + 32));
+        const float4 u1 = __ldg(reinterpret_cast<const float4*>(row + gcol + 36));
+        g[0] = g0.x, g[1] = g0.y, g[2] = g0.z, g[3] = g0.w, g[4] = g1.x, g[5] = g1.y, g[6] = g1.z, g[7] = g1.w;
+        u[0] = u0.x, u[1] = u0.y, u[2] = u0.z, u[3] = u0.w, u[4] = u1.x, u[5] = u1.y, u[6] = u1.z, u[7] = u1.w;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = swiglu1(g[k], u[k]);
+        *reinterpret_cast<uint4*>(out + (size_t)m * F + f0) = pack8(o);
     }
 }
 

@@ -23,7 +23,7 @@ namespace {
 
 using namespace tbik;
 
-constexpr unsigned kModeMask = TBIK_EXACT | TBIK_TC | TBIK_NONINV | TBIK_B_NK | TBIK_OUT_BF16;
+constexpr unsigned kModeMask = TBIK_EXACT | TBIK_TC | TBIK_NONINV | TBIK_B_NK | TBIK_OUT_BF16 | TBIK_SWIGLU_OUT;
 constexpr int kMaxDevices = 64;
 
 unsigned g_debug_flags = 0;
@@ -184,13 +184,14 @@ int max_stack_depth(int n) {
 
 struct GemmPlan {
     bool tc = false, noninv = false, b_nk = false, out_bf16 = false;
+    bool swiglu = false, fused = false;  // SwiGLU output; applied in the TC epilogue when fused
     int M = 0, N = 0, K = 0, T = 1, leaf = 1;
     int L = 0, D = 0, F = 1;
     int tiles_m = 0, tiles_n = 0, units = 0, grid = 0, gs = 0;
     bool direct = true;
     std::vector<std::pair<int, int>> nodes;  // (first leaf, leaves) per frontier node
     int leaf_eff = 1;                        // K elements per leaf as launched
-    size_t off_partials = 0, off_shards = 0, off_scratch = 0, total = 0;
+    size_t off_partials = 0, off_shards = 0, off_scratch = 0, off_gu = 0, total = 0;
 };
 
 tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int sms, GemmPlan& p) {
@@ -203,6 +204,10 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
     p.noninv = mode & TBIK_NONINV;
     p.b_nk = mode & TBIK_B_NK;
     p.out_bf16 = mode & TBIK_OUT_BF16;
+    p.swiglu = mode & TBIK_SWIGLU_OUT;
+    if (p.swiglu && p.noninv) return TBIK_ERR_ARG;
+    if (p.swiglu && N % 64) return TBIK_ERR_SHAPE;
+    if (p.swiglu) p.out_bf16 = false;  // the tree roots stay fp32 until the SwiGLU
     p.M = M, p.N = N, p.K = K, p.T = T, p.leaf = leaf;
     p.L = K / leaf;
     if (p.L % T) return TBIK_ERR_SHAPE;
@@ -268,6 +273,11 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
         p.off_scratch = off;
         off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
     }
+    p.fused = p.swiglu && tc && p.direct;
+    if (p.swiglu && !p.fused) {  // fp32 gate/up roots, then the SwiGLU kernel
+        p.off_gu = off;
+        off = align256(off + mn);
+    }
     p.total = off;
     return TBIK_OK;
 }
@@ -328,6 +338,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
                      cudaStream_t s, const DeviceInfo* info) {
     const int sms = info->sms;
     if (p.M == 0) return TBIK_OK;
+    void* Cg = (p.swiglu && !p.fused) ? (void*)(ws + p.off_gu) : C;  // where the GEMM writes
     if (p.tc) {
         CUtensorMap ta, tb;
         const int a_box = a_box_rows(p.M);
@@ -345,7 +356,8 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.total_units = p.units;
         prm.direct = p.direct;
         prm.out_bf16 = p.out_bf16;
-        prm.out = C;
+        prm.swiglu = p.fused ? 1 : 0;
+        prm.out = Cg;
         prm.partials = p.direct ? nullptr : reinterpret_cast<float*>(ws + p.off_partials);
         prm.scratch = p.gs ? reinterpret_cast<float*>(ws + p.off_scratch) : nullptr;
         prm.gs = p.gs;
@@ -373,7 +385,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.total_units = p.units;
         prm.direct = p.direct;
         prm.out_bf16 = p.out_bf16;
-        prm.out = C;
+        prm.out = Cg;
         prm.partials = p.direct ? nullptr : reinterpret_cast<float*>(ws + p.off_partials);
         for (int f = 0; f < p.F; ++f) {
             prm.lo[f] = (short)p.nodes[f].first;
@@ -387,7 +399,15 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
     }
     tbik_status st = launch_status();
     if (st != TBIK_OK) return st;
-    return finish_gemm(p, ws, C, s, sms);
+    st = finish_gemm(p, ws, Cg, s, sms);
+    if (st != TBIK_OK || !p.swiglu || p.fused) return st;
+    const int F = p.N / 2;
+    const long long work = (long long)p.M * (F / 8);
+    long long blocks = (work + 255) / 256;
+    if (blocks > (long long)sms * 8) blocks = (long long)sms * 8;
+    swiglu_interleaved_kernel<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const float*>(Cg),
+                                                         reinterpret_cast<uint16_t*>(C), p.M, F);
+    return launch_status();
 }
 
 // ----------------------------------------------------------- logprob plan

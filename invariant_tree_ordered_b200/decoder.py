@@ -9,10 +9,11 @@ same for every T); RoPE on q, k; causal attention with the keys in chunks of
 64 combined by the tree (heads split across devices: per-head, so the same
 for every T); o Wo (row-parallel: K = d split into T shards, combined by the
 tree, or by the non-invariant chain-and-sum baseline); residual + RMSNorm;
-gate, up (column-parallel); SwiGLU; down (row-parallel); residual.  Then the
-final RMSNorm and the lm_head logprob (T splits the vocabulary).  GEMM outputs
-are rounded to bf16 once; gammas come with the weights; eps 1e-6; RoPE base
-1e6; positions 0..seq-1 in every sequence.
+gate and up as one column-parallel GEMM whose epilogue applies SwiGLU to the
+fp32 roots (one bf16 rounding, after the SwiGLU); down (row-parallel);
+residual.  Then the final RMSNorm and the lm_head logprob (T splits the
+vocabulary).  Other GEMM outputs are rounded to bf16 once; gammas come with
+the weights; eps 1e-6; RoPE base 1e6; positions 0..seq-1 in every sequence.
 """
 from dataclasses import dataclass
 
@@ -35,8 +36,9 @@ class DecoderConfig:
 
 class Decoder:
     """Weights are device bf16 tensors: ``emb`` and ``lm_head`` [vocab, d],
-    ``gamma`` [d], and per layer ``wq wk wv wo`` [d, d], ``wg wu`` [d, ffn],
-    ``wd`` [ffn, d] ([in, out] row-major)."""
+    ``gamma`` [d], and per layer ``wq wk wv wo`` [d, d], ``wgu`` [d, 2 ffn]
+    (gate and up interleaved, see `interleave_gate_up`), ``wd`` [ffn, d]
+    ([in, out] row-major)."""
 
     def __init__(self, cfg: DecoderConfig, emb, lm_head, gamma, layers):
         self.cfg, self.emb, self.lm_head, self.gamma, self.layers = cfg, emb, lm_head, gamma, layers
@@ -77,9 +79,8 @@ class Decoder:
                              v.view(B, S, c.heads, c.head_dim), stream=stream)
             a = dense(o.view(n, c.d), L["wo"], c.leaf, T, noninv)
             y, res = tb.rmsnorm_residual(a, res, self.gamma, eps=1e-6, T=1, stream=stream)
-            g = dense(y, L["wg"], c.leaf)
-            u = dense(y, L["wu"], c.leaf)
-            _, _, act = tb.rope_swiglu(g=g, u=u, stream=stream)
+            act = torch.empty((n, c.ffn), dtype=bf, device=dev)
+            tb.gemm(y, L["wgu"], T=1, leaf=c.leaf, tc=tc, swiglu=True, out=act, stream=stream)
             m = dense(act, L["wd"], c.leaf_ffn, T, noninv)
             y, res = tb.rmsnorm_residual(m, res, self.gamma, eps=1e-6, T=1, stream=stream)
         lp = tb.logprob(y, self.lm_head, targets.reshape(-1), T=T, leaf=c.leaf, tc=tc, noninv=noninv, stream=stream)
@@ -89,3 +90,17 @@ class Decoder:
 def positions(batch: int, seq: int) -> np.ndarray:
     """Position of each token of a [batch, seq] block (0..seq-1 per sequence)."""
     return np.tile(np.arange(seq, dtype=np.int32), batch)
+
+
+def interleave_gate_up(wg: np.ndarray, wu: np.ndarray) -> np.ndarray:
+    """[K, F] gate and up weights -> [K, 2F] with blocks of 32 columns
+    alternating (gate features 32j..32j+31, then the same up features), the
+    layout the SwiGLU-output GEMM expects.  Data layout only."""
+    K, F = wg.shape
+    if wu.shape != wg.shape or F % 32:
+        raise ValueError("gate and up must share the shape [K, F] with F % 32 == 0")
+    out = np.empty((K, F // 32, 2, 32), dtype=wg.dtype)
+    out[:, :, 0] = wg.reshape(K, F // 32, 32)
+    out[:, :, 1] = wu.reshape(K, F // 32, 32)
+    return out.reshape(K, 2 * F)
+

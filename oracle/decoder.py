@@ -7,10 +7,11 @@ Per layer: y = RMSNorm(h) -> q, k, v = y Wq, y Wk, y Wv (column-parallel:
 the whole K tree, the same for every T) -> RoPE(q, k) -> causal attention
 with key chunks of 64 combined by the tree -> o Wo (row-parallel: T shards of
 K, combined by the tree, or the non-invariant chain-and-sum baseline) ->
-residual -> RMSNorm -> gate/up (column-parallel) -> SwiGLU -> down
-(row-parallel) -> residual.  Then the final RMSNorm and the lm_head logprob
-of each target (T splits the vocabulary).  GEMM results are rounded to bf16
-once; RMSNorm gammas are 1, eps 1e-6, RoPE base 1e6, positions 0..seq-1.
+residual -> RMSNorm -> gate/up (column-parallel, kept fp32) -> SwiGLU on the
+fp32 values -> down (row-parallel) -> residual.  Then the final RMSNorm and
+the lm_head logprob of each target (T splits the vocabulary).  Other GEMM
+results are rounded to bf16 once; RMSNorm gammas are 1, eps 1e-6, RoPE base
+1e6, positions 0..seq-1.
 """
 import numpy as np
 
@@ -47,8 +48,9 @@ def forward(cfg, w, ids, targets, *, T: int = 1, noninv: bool = False):
         o = attention(q.reshape(B, S, NH, HD), k.reshape(B, S, NH, HD), v.reshape(B, S, NH, HD), chunk=64)
         a = _dense(o.reshape(n, d), L["wo"], leaf=leaf, T=T, noninv=noninv)
         y, res = rmsnorm_residual(a, res, gamma, eps=1e-6)
-        g = _dense(y, L["wg"], leaf=leaf)
-        u = _dense(y, L["wu"], leaf=leaf)
+        # gate and up stay fp32 until the SwiGLU: one rounding, at its output
+        g = gemm_tree(y, L["wg"], b_nk=False, T=1, leaf=leaf)
+        u = gemm_tree(y, L["wu"], b_nk=False, T=1, leaf=leaf)
         act = swiglu(g, u)
         m = _dense(act, L["wd"], leaf=leaf_ffn, T=T, noninv=noninv)
         y, res = rmsnorm_residual(m, res, gamma, eps=1e-6)

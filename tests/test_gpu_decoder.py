@@ -16,12 +16,16 @@ torch = pytest.importorskip("torch")
 from tests.gpu_util import dev_bf16, dev_i32, host_f32, u32  # noqa: E402
 
 import invariant_tree_ordered_b200 as tbik  # noqa: E402
-from invariant_tree_ordered_b200.decoder import Decoder, DecoderConfig, positions  # noqa: E402
+from invariant_tree_ordered_b200.decoder import Decoder, DecoderConfig, interleave_gate_up, positions  # noqa: E402
 
 
 def build(cfg):
     w = synth.decoder_weights(cfg)
-    layers = [{k: dev_bf16(v) for k, v in L.items()} for L in w["layers"]]
+    layers = []
+    for L in w["layers"]:
+        dl = {k: dev_bf16(L[k]) for k in ("wq", "wk", "wv", "wo", "wd")}
+        dl["wgu"] = dev_bf16(interleave_gate_up(L["wg"], L["wu"]))
+        layers.append(dl)
     dc = DecoderConfig(d=cfg["d"], heads=cfg["heads"], head_dim=cfg["head_dim"], ffn=cfg["ffn"],
                        vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"])
     return w, Decoder(dc, dev_bf16(w["emb"]), dev_bf16(w["lm_head"]), dev_bf16(w["gamma"]), layers)
