@@ -226,6 +226,15 @@ TBIK_API tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const 
 TBIK_API tbik_status tbik_embedding(const int32_t* ids, const uint16_t* table, uint16_t* out, int tokens, int V,
                                     int d, void* stream);
 
+/*
+ * out[c][r] = in[r][c] for bf16 [rows, cols] -> [cols, rows] (device memory,
+ * 2-byte aligned, no overlap).  Data movement only: it gives the weight
+ * gradient dW = X^T dY its A operand, so that dW = tbik_gemm(X^T, dY) reduces
+ * over tokens with the same leaf tree (T = data-parallel shards of the
+ * tokens).  No counterpart on the pages.
+ */
+TBIK_API tbik_status tbik_transpose(const uint16_t* in, uint16_t* out, int rows, int cols, void* stream);
+
 /* ---- fused lm_head -> log-softmax -> target logprob ---------------------- */
 
 TBIK_API size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, unsigned mode);

@@ -84,6 +84,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "tbik_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
             "tbik_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
             "tbik_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp]),
+            "tbik_transpose": (i32, [vp, vp, i32, i32, vp]),
             "tbik_get_error": (i32, [vp]),
             "tbik_debug_set": (i32, [u32, ull]),
         }
@@ -272,6 +273,18 @@ def embedding(ids, table, *, out=None, stream=None):
         out = torch.empty((ids.numel(), d), dtype=torch.bfloat16, device=table.device)
     _check(lib.tbik_embedding(_ptr(ids), _ptr(table), _ptr(out), ids.numel(), V, d, _stream_handle(stream)),
            "tbik_embedding")
+    return out
+
+
+def transpose(x, *, out=None, stream=None):
+    """bf16 [rows, cols] -> [cols, rows] (see tbik_transpose)."""
+    torch = _torch()
+    lib = load_library()
+    _need(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty((cols, rows), dtype=torch.bfloat16, device=x.device)
+    _check(lib.tbik_transpose(_ptr(x), _ptr(out), rows, cols, _stream_handle(stream)), "tbik_transpose")
     return out
 
 

@@ -231,4 +231,19 @@ __global__ void embedding_kernel(const int32_t* __restrict__ ids, const uint16_t
     }
 }
 
+// bf16 transpose through a 32 x 33 shared-memory tile (block 32 x 8).
+__global__ void transpose_kernel(const uint16_t* __restrict__ in, uint16_t* out, int rows, int cols) {
+    __shared__ uint16_t tile[32][33];
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    for (int k = threadIdx.y; k < 32; k += 8) {
+        const int r = r0 + k, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) tile[k][threadIdx.x] = in[(size_t)r * cols + c];
+    }
+    __syncthreads();
+    for (int k = threadIdx.y; k < 32; k += 8) {
+        const int c = c0 + k, r = r0 + threadIdx.x;
+        if (r < rows && c < cols) out[(size_t)c * rows + r] = tile[threadIdx.x][k];
+    }
+}
+
 }  // namespace tbik

@@ -598,6 +598,22 @@ tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const uint16_t*
     return launch_status();
 }
 
+tbik_status tbik_transpose(const uint16_t* in, uint16_t* out, int rows, int cols, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (rows < 0 || cols < 0) return TBIK_ERR_ARG;
+    if (rows == 0 || cols == 0) return TBIK_OK;
+    if (!in || !out) return TBIK_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 1u) return TBIK_ERR_ALIGN;
+    const long long gx = (cols + 31) / 32, gy = (rows + 31) / 32;
+    if (gy > 65535) return TBIK_ERR_SHAPE;
+    transpose_kernel<<<dim3((unsigned)gx, (unsigned)gy), dim3(32, 8), 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        in, out, rows, cols);
+    return launch_status();
+}
+
 tbik_status tbik_embedding(const int32_t* ids, const uint16_t* table, uint16_t* out, int tokens, int V, int d,
                            void* stream) {
     int dev;
