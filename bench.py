@@ -404,7 +404,13 @@ def run_tbik(args):
                        device=dev)
     g_t8 = avg_ms(lambda: tbik.gemm(A, B, T=8, leaf=LEAF, tc=True, out_bf16=True, out=hid2, workspace=gws8))
     tbik.get_error(stream)
-    dec = None if args.no_decoder else decoder_component(dev, stream)
+    dec = None
+    if not args.no_decoder:
+        try:  # an extra measurement: a failure here must not cost the main line
+            dec = decoder_component(dev, stream)
+        except Exception as e:  # noqa: BLE001
+            dec = {"error": f"{type(e).__name__}: {e}"[:300]}
+            torch.cuda.synchronize()
 
     pk = peaks()
     lp_ms = lp_live_ms
