@@ -37,8 +37,10 @@ template <int DPL>
 __device__ __forceinline__ AttNode<DPL> att_combine(const AttNode<DPL>& a, const AttNode<DPL>& b) {
     AttNode<DPL> r;
     r.m = (b.m > a.m) ? b.m : a.m;
-    const float ea = exp_spec(__fsub_rn(a.m, r.m));
-    const float eb = exp_spec(__fsub_rn(b.m, r.m));
+    // the side holding the max has the factor exp(+0) = 1 exactly
+    const bool finite = r.m != INFINITY;
+    const float ea = (finite && a.m == r.m) ? 1.0f : exp_spec(__fsub_rn(a.m, r.m));
+    const float eb = (finite && b.m == r.m) ? 1.0f : exp_spec(__fsub_rn(b.m, r.m));
     r.s = __fadd_rn(__fmul_rn(a.s, ea), __fmul_rn(b.s, eb));
 #pragma unroll
     for (int d = 0; d < DPL; ++d) r.o[d] = __fadd_rn(__fmul_rn(a.o[d], ea), __fmul_rn(b.o[d], eb));

@@ -165,8 +165,11 @@ __device__ __forceinline__ MS ms_combine(MS a, MS b) {
         r.s = 0.0f;
         return r;
     }
-    float ea = exp_spec(__fsub_rn(a.m, r.m));
-    float eb = exp_spec(__fsub_rn(b.m, r.m));
+    // the side that holds the max has the factor exp(+0) = 1 exactly (the
+    // specification returns 1 for +0), so it is not evaluated
+    const bool finite = r.m != INFINITY;
+    const float ea = (finite && a.m == r.m) ? 1.0f : exp_spec(__fsub_rn(a.m, r.m));
+    const float eb = (finite && b.m == r.m) ? 1.0f : exp_spec(__fsub_rn(b.m, r.m));
     r.s = __fadd_rn(__fmul_rn(a.s, ea), __fmul_rn(b.s, eb));
     return r;
 }
