@@ -466,8 +466,9 @@ def run_tbik(args):
 def decoder_component(dev, stream):
     """The end-to-end decoder (4 layers, d 2048, 16 heads of 128, ffn 5632,
     vocab 32000, batch 8 x seq 2048): forward + target logprobs in tensor-core
-    mode at T = 1 (tokens/s, CUDA events), the attention kernel alone, the
-    bitwise check against T = 8, and the non-invariant baseline's divergence."""
+    mode at T = 1 (tokens/s, CUDA events), the same with the residual add fused
+    into the o and down projections, the attention kernel alone, the bitwise
+    checks against T = 8, and the non-invariant baseline's divergence."""
     import torch
 
     import invariant_tree_ordered_b200 as tbik
@@ -500,6 +501,14 @@ def decoder_component(dev, stream):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / n
+    fused = fwd(T=1, tc=True, fuse_residual=True)  # residual add in the o and down projections
+    a.record(stream)
+    for _ in range(n):
+        fwd(T=1, tc=True, fuse_residual=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_fused = a.elapsed_time(b) / n
+    fused8 = fwd(T=8, tc=True, fuse_residual=True)
     t8 = fwd(T=8, tc=True)
     non1, non8 = fwd(T=1, tc=True, noninv=True), fwd(T=8, tc=True, noninv=True)
     q = torch.randn(B, S, cfg["heads"], cfg["head_dim"], device=dev).to(torch.bfloat16)
@@ -516,6 +525,8 @@ def decoder_component(dev, stream):
     return {"workload": "4 layers, d 2048, 16x128 heads, ffn 5632, vocab 32000, batch 8 x seq 2048, TC, T=1",
             "tokens_per_s": B * S / (ms * 1e-3), "ms_per_forward": ms,
             "bitwise_T1_vs_T8": bool(torch.equal(base.view(torch.int32), t8.view(torch.int32))),
+            "ms_per_forward_fused_residual": ms_fused,
+            "fused_residual_bitwise_T1_vs_T8": bool(torch.equal(fused.view(torch.int32), fused8.view(torch.int32))),
             "noninv_max_abs_dlogprob_T8_vs_T1": float((non8 - non1).abs().max()),
             "attention_ms_per_layer": att_ms, "attention_tflops": att_flop / (att_ms * 1e-3) / 1e12,
             "status": int(status)}

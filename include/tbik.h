@@ -134,6 +134,27 @@ TBIK_API size_t tbik_gemm_workspace(int M, int N, int K, int T, int leaf, unsign
 TBIK_API tbik_status tbik_gemm(const uint16_t* A, const uint16_t* B, void* C, int M, int N, int K, int T,
                       int leaf, unsigned mode, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Row-parallel projection with the residual add fused into its last step
+ * (the down or output projection of a pre-norm block: the rounding-location
+ * article, 3つのノード, keeps the residual add in fp32 and rounds once):
+ *   C[i,n] = bf16( root[i,n] + f32(R[i,n]) ),
+ * root = the fp32 tree root tbik_gemm computes for the same arguments, one
+ * correctly rounded fp32 add, then one RNE rounding.  The add happens where
+ * the root is final: the GEMM epilogue when the tiles write C directly, else
+ * the kernel that combines the shard partials (the non-invariant baseline
+ * adds R after its left-to-right shard sum).
+ *   R, C  bf16 [M,N] row-major, 16-byte aligned; C may be R itself (in place)
+ *         but may not overlap it otherwise, nor alias A or B.
+ *   mode  as tbik_gemm without TBIK_OUT_* bits (the output is bf16) and
+ *         without TBIK_SWIGLU_OUT (else TBIK_ERR_ARG).
+ *   ws    tbik_gemm_workspace(M, N, K, T, leaf, mode | TBIK_OUT_BF16) bytes.
+ * Errors and shape rules are those of tbik_gemm; R == NULL is TBIK_ERR_ARG.
+ */
+TBIK_API tbik_status tbik_gemm_residual(const uint16_t* A, const uint16_t* B, const uint16_t* R, uint16_t* C,
+                               int M, int N, int K, int T, int leaf, unsigned mode, void* ws,
+                               size_t ws_bytes, void* stream);
+
 /* ---- residual RMSNorm ---------------------------------------------------- */
 
 /*
@@ -145,7 +166,8 @@ TBIK_API tbik_status tbik_gemm(const uint16_t* A, const uint16_t* B, void* C, in
  *   inv = 1 / sqrt(ms + eps) (correctly rounded ops);
  *   y = bf16((r * inv) * gamma);  res_out = bf16(r).
  * x, res, y, res_out: bf16 [tokens,H]; gamma bf16 [H]; res_out may be NULL;
- * y may alias x.  H % 8 == 0 and H/8 a power of two in [32, 1024]
+ * res may be NULL (r = f32(x): the norm of a residual stream that
+ * tbik_gemm_residual already updated); y may alias x.  H % 8 == 0 and H/8 a power of two in [32, 1024]
  * (H in {256, 512, ..., 8192}); T in {1,2,4,8}.
  */
 TBIK_API tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16_t* gamma,

@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "tbik_status_string": (ctypes.c_char_p, [i32]),
             "tbik_gemm_workspace": (sz, [i32, i32, i32, i32, i32, u32]),
             "tbik_gemm": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
+            "tbik_gemm_residual": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
             "tbik_rmsnorm_residual": (i32, [vp, vp, vp, vp, vp, i32, i32, f32, i32, vp]),
             "tbik_rope_table": (i32, [vp, i32, i32, f64, vp]),
             "tbik_rope_swiglu_fp32": (i32, [ctypes.POINTER(RopeSwigluArgs), vp]),
@@ -163,10 +164,12 @@ def gemm_workspace(M, N, K, T, leaf, mode) -> int:
 
 
 def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = False, b_nk: bool = False,
-         out_bf16: bool = False, swiglu: bool = False, out=None, workspace=None, stream=None):
+         out_bf16: bool = False, swiglu: bool = False, residual=None, out=None, workspace=None, stream=None):
     """C = A @ B with the K reduction in tree order (see tbik_gemm in tbik.h).
     swiglu: B holds gate/up columns interleaved in blocks of 32 and C is the
-    bf16 SwiGLU [M, N/2] of the fp32 roots (TBIK_SWIGLU_OUT)."""
+    bf16 SwiGLU [M, N/2] of the fp32 roots (TBIK_SWIGLU_OUT).
+    residual: bf16 [M, N]; C = bf16(root + residual) (tbik_gemm_residual);
+    ``out`` may be the residual tensor itself (in place)."""
     torch = _torch()
     lib = load_library()
     _need(A, torch.bfloat16, "A")
@@ -176,7 +179,20 @@ def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = F
     kb = B.shape[1] if b_nk else B.shape[0]
     if kb != K:
         raise ValueError("inner dimensions differ")
-    mode = (TC if tc else EXACT) | (NONINV if noninv else 0) | (B_NK if b_nk else B_KN) | (OUT_BF16 if out_bf16 else OUT_F32)
+    mode = (TC if tc else EXACT) | (NONINV if noninv else 0) | (B_NK if b_nk else B_KN)
+    if residual is not None:
+        if swiglu:
+            raise ValueError("residual and swiglu outputs are exclusive")
+        _need(residual, torch.bfloat16, "residual")
+        if tuple(residual.shape) != (M, N):
+            raise ValueError("residual must be [M, N]")
+        if out is None:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+        ws, wsb = _workspace(lib.tbik_gemm_workspace(M, N, K, T, leaf, mode | OUT_BF16), A.device, workspace)
+        _check(lib.tbik_gemm_residual(_ptr(A), _ptr(B), _ptr(residual), _ptr(out), M, N, K, T, leaf, mode,
+                                      _ptr(ws), wsb, _stream_handle(stream)), "tbik_gemm_residual")
+        return out
+    mode |= OUT_BF16 if out_bf16 else OUT_F32
     if swiglu:
         mode |= SWIGLU_OUT
     if out is None:
@@ -195,7 +211,8 @@ def rmsnorm_residual(x, res, gamma, *, eps: float = 1e-6, T: int = 1, y=None, re
     torch = _torch()
     lib = load_library()
     for t, n in ((x, "x"), (res, "res"), (gamma, "gamma")):
-        _need(t, torch.bfloat16, n)
+        if t is not None or n != "res":  # res None: no residual input, r = f32(x)
+            _need(t, torch.bfloat16, n)
     tokens, H = x.shape
     if y is None:
         y = torch.empty_like(x)

@@ -32,14 +32,17 @@ struct ExParams {
     int direct;
     int out_bf16;
     void* out;
+    const uint16_t* residual;  // bf16 [M,N] added to the fp32 root before the bf16 rounding (direct only)
     float* partials;  // [F][M][N]
     short lo[EX_MAX_F];
     short nl[EX_MAX_F];
 };
 
-__device__ __forceinline__ void ex_store(void* out, int bf16, int M, int N, int row, int col, float v) {
+__device__ __forceinline__ void ex_store(void* out, int bf16, int M, int N, int row, int col, float v,
+                                         const uint16_t* residual) {
     if (row >= M || col >= N) return;
     size_t off = (size_t)row * N + col;
+    if (residual) v = __fadd_rn(v, bf2f(residual[off]));
     if (bf16)
         reinterpret_cast<uint16_t*>(out)[off] = f2bf(v);
     else
@@ -123,11 +126,13 @@ __global__ void __launch_bounds__(EX_THREADS) gemm_exact_kernel(const __grid_con
                     if (ops.final_) {
                         void* dst = p.direct ? p.out : (void*)(p.partials + (size_t)f * p.M * p.N);
                         const int bf = p.direct ? p.out_bf16 : 0;
+                        const uint16_t* res = p.direct ? p.residual : nullptr;
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
 #pragma unroll
                             for (int c = 0; c < 4; ++c)
-                                ex_store(dst, bf, p.M, p.N, m0 + ty * 4 + i, n0 + tx * 4 + c, acc[i * 4 + c]);
+                                ex_store(dst, bf, p.M, p.N, m0 + ty * 4 + i, n0 + tx * 4 + c, acc[i * 4 + c],
+                                         res);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) stk[sp][e] = acc[e];
@@ -168,14 +173,24 @@ struct TreeOf<1> {
 };
 
 // out[g] = TREE over P[g*G .. g*G+G) for g < groups; each buffer has MN floats.
-// out is fp32 [groups][MN] or, with out_bf16, bf16 [MN] (groups == 1).
+// out is fp32 [groups][MN] or, with out_bf16, bf16 [MN] (groups == 1); with
+// out_bf16, a non-null R (bf16 [MN], may be `out` itself) is added to the root
+// in fp32 before the rounding.
 template <int G>
-__global__ void tree_combine_kernel(const float* __restrict__ P, size_t MN, int groups, void* out, int out_bf16) {
+__global__ void tree_combine_kernel(const float* __restrict__ P, size_t MN, int groups, void* out, int out_bf16,
+                                    const uint16_t* R) {
     const size_t nvec = MN / 4;
     const size_t total = nvec * groups;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
         const size_t g = i / nvec, e = (i - g * nvec) * 4;
-        const float4 r = TreeOf<G>::vec(P + g * G * MN, MN, e);
+        float4 r = TreeOf<G>::vec(P + g * G * MN, MN, e);
+        if (out_bf16 && R) {
+            const uint2 q = *reinterpret_cast<const uint2*>(R + e);
+            r.x = __fadd_rn(r.x, __uint_as_float(q.x << 16));
+            r.y = __fadd_rn(r.y, __uint_as_float(q.x & 0xffff0000u));
+            r.z = __fadd_rn(r.z, __uint_as_float(q.y << 16));
+            r.w = __fadd_rn(r.w, __uint_as_float(q.y & 0xffff0000u));
+        }
         if (out_bf16) {
             uint2 w;
             w.x = pack_bf2(r.x, r.y);
@@ -189,7 +204,8 @@ __global__ void tree_combine_kernel(const float* __restrict__ P, size_t MN, int 
     const size_t tail = MN - nvec * 4;
     if (blockIdx.x == 0 && threadIdx.x < tail * groups) {
         const size_t g = threadIdx.x / tail, e = nvec * 4 + threadIdx.x % tail;
-        const float r = TreeOf<G>::one(P + g * G * MN, MN, e);
+        float r = TreeOf<G>::one(P + g * G * MN, MN, e);
+        if (out_bf16 && R) r = __fadd_rn(r, bf2f(R[e]));
         if (out_bf16)
             reinterpret_cast<uint16_t*>(out)[e] = f2bf(r);
         else
@@ -197,11 +213,14 @@ __global__ void tree_combine_kernel(const float* __restrict__ P, size_t MN, int 
     }
 }
 
-// Non-invariant combine: ((P0 + P1) + P2) + ... left to right.
-__global__ void seq_combine_kernel(const float* __restrict__ P, size_t MN, int T, void* out, int out_bf16) {
+// Non-invariant combine: ((P0 + P1) + P2) + ... left to right (then + R, as
+// in tree_combine_kernel).
+__global__ void seq_combine_kernel(const float* __restrict__ P, size_t MN, int T, void* out, int out_bf16,
+                                   const uint16_t* R) {
     for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < MN; e += (size_t)gridDim.x * blockDim.x) {
         float acc = P[e];
         for (int t = 1; t < T; ++t) acc = __fadd_rn(acc, P[(size_t)t * MN + e]);
+        if (out_bf16 && R) acc = __fadd_rn(acc, bf2f(R[e]));
         if (out_bf16)
             reinterpret_cast<uint16_t*>(out)[e] = f2bf(acc);
         else

@@ -70,7 +70,10 @@ constexpr int TC_RING_BYTES = TC_STAGES * (TC_A_BYTES + TC_B_BYTES);
 constexpr size_t TC_SMEM_BYTES = (size_t)TC_RING_BYTES + TC_SLOT_FLOATS * 4 +
                                  2 * TC_TAB_MAX * 2 /*op tables*/ + 1024 /*align*/ + 256 /*barriers*/;
 
-enum { EPI_TREE = 0, EPI_LOGPROB = 1 };
+// EPI_TREE_RES: EPI_TREE whose direct tiles add the bf16 residual to the fp32
+// root before the output rounding (a separate instantiation, so the plain
+// tree epilogue carries no residual code).
+enum { EPI_TREE = 0, EPI_LOGPROB = 1, EPI_TREE_RES = 2 };
 
 struct TcParams {
     int M, N, K;
@@ -82,6 +85,7 @@ struct TcParams {
     int out_bf16;
     int swiglu;       // 1: C = bf16 SwiGLU of the interleaved gate/up roots, [M, N/2] (direct only)
     void* out;        // C [M,N]
+    const uint16_t* residual;  // EPI_TREE_RES: bf16 [M,N] added to the root before the rounding (direct only)
     float* partials;  // [F][M][N]
     float* scratch;   // [gridDim.x][gs][128*128], layout per slot [col/4][row][4]
     int gs;           // global stack slots per CTA (pending subtrees of >= 5 leaves)
@@ -162,6 +166,21 @@ __device__ __forceinline__ void store_row32(void* out, int out_bf16, int M, int 
             *reinterpret_cast<float4*>(o) = make_float4(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3]);
             *reinterpret_cast<float4*>(o + 4) = make_float4(v[8 * q + 4], v[8 * q + 5], v[8 * q + 6], v[8 * q + 7]);
         }
+    }
+}
+
+// v[k] += f32(R[row, col0 + k]) for the 32 columns of store_row32 (one fp32
+// add each, before the output's single rounding); N % 8 == 0.
+__device__ __forceinline__ void add_residual32(const uint16_t* R, int M, int N, int row, int col0, float (&v)[32]) {
+    if (row >= M) return;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int col = col0 + 8 * q;
+        if (col >= N) break;
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(R + (size_t)row * N + col), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * q + e] = __fadd_rn(v[8 * q + e], f[e]);
     }
 }
 
@@ -498,13 +517,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                             if (f0 + 8 * q8 < p.N / 2) dst[q8] = pack8(o);
                         }
                     }
-                } else if (EPI == EPI_TREE) {
+                } else if (EPI != EPI_LOGPROB) {
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         const int col = tn * TC_BN + (half * 2 + cc) * 32;
-                        if (p.direct)
+                        if (p.direct) {
+                            if (EPI == EPI_TREE_RES) add_residual32(p.residual, p.M, p.N, row, col, v[cc]);
                             store_row32(p.out, p.out_bf16, p.M, p.N, row, col, v[cc]);
-                        else
+                        } else
                             store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row, col, v[cc]);
                     }
                 } else {

@@ -20,7 +20,8 @@ namespace tbik {
 // group level, so these are the same levels as a per-shard tree followed by
 // the tree over the T shard partials.  A CTA loops over tokens and loads the
 // next token while it reduces and writes the current one; gamma is loaded once.
-template <int NT, int LPT>
+// RES = false: no residual input, r = f32(x) (res is not read).
+template <int NT, int LPT, bool RES>
 __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ res,
                                                               const uint16_t* __restrict__ gamma, uint16_t* y,
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
     for (int l = 0; l < LPT; ++l) {
         gv[l] = __ldg(reinterpret_cast<const uint4*>(gamma) + LPT * tid + l);
         xv[l] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * H) + LPT * tid + l);
-        rv[l] = __ldg(reinterpret_cast<const uint4*>(res + (size_t)t * H) + LPT * tid + l);
+        if (RES) rv[l] = __ldg(reinterpret_cast<const uint4*>(res + (size_t)t * H) + LPT * tid + l);
     }
     for (int it = 0;; ++it) {
         const int tn = t + gridDim.x;
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
 #pragma unroll
             for (int l = 0; l < LPT; ++l) {
                 xn[l] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)tn * H) + LPT * tid + l);
-                rn[l] = __ldg(reinterpret_cast<const uint4*>(res + (size_t)tn * H) + LPT * tid + l);
+                if (RES) rn[l] = __ldg(reinterpret_cast<const uint4*>(res + (size_t)tn * H) + LPT * tid + l);
             }
         }
         float leafsum[LPT];
@@ -56,11 +57,11 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
         for (int l = 0; l < LPT; ++l) {
             float xf[8], rf[8];
             unpack8(xv[l], xf);
-            unpack8(rv[l], rf);
+            if (RES) unpack8(rv[l], rf);
             float acc = 0.0f;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float r = __fadd_rn(xf[e], rf[e]);
+                const float r = RES ? __fadd_rn(xf[e], rf[e]) : xf[e];
                 acc = __fmaf_rn(r, r, acc);
             }
             leafsum[l] = acc;
@@ -83,11 +84,11 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
         for (int l = 0; l < LPT; ++l) {
             float xf[8], rf[8], gf[8], r[8], o[8];
             unpack8(xv[l], xf);
-            unpack8(rv[l], rf);
+            if (RES) unpack8(rv[l], rf);
             unpack8(gv[l], gf);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                r[e] = __fadd_rn(xf[e], rf[e]);
+                r[e] = RES ? __fadd_rn(xf[e], rf[e]) : xf[e];
                 o[e] = __fmul_rn(__fmul_rn(r[e], inv), gf[e]);
             }
             reinterpret_cast<uint4*>(y + (size_t)t * H)[LPT * tid + l] = pack8(o);
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
 #pragma unroll
         for (int l = 0; l < LPT; ++l) {
             xv[l] = xn[l];
-            rv[l] = rn[l];
+            if (RES) rv[l] = rn[l];
         }
     }
 }

@@ -57,6 +57,8 @@ tbik_status device_info(int& dev, DeviceInfo*& info) {
     if (!d.attrs_set) {
         if (cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)TC_SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE_RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TC_SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_tc_kernel<EPI_LOGPROB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)TC_SMEM_BYTES) != cudaSuccess)
             return TBIK_ERR_CUDA;
@@ -285,47 +287,49 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
 tbik_status launch_status() { return cudaGetLastError() == cudaSuccess ? TBIK_OK : TBIK_ERR_CUDA; }
 
 template <int G>
-void launch_tree_combine(const float* P, size_t MN, int groups, void* out, int bf16, cudaStream_t s, int sms) {
+void launch_tree_combine(const float* P, size_t MN, int groups, void* out, int bf16, const uint16_t* R,
+                         cudaStream_t s, int sms) {
     size_t work = (MN / 4) * groups;
     int blocks = (int)((work + 255) / 256);
     if (blocks > sms * 8) blocks = sms * 8;
     if (blocks < 1) blocks = 1;
-    tree_combine_kernel<G><<<blocks, 256, 0, s>>>(P, MN, groups, out, bf16);
+    tree_combine_kernel<G><<<blocks, 256, 0, s>>>(P, MN, groups, out, bf16, R);
 }
 
 tbik_status tree_combine(const float* P, size_t MN, int G, int groups, void* out, int bf16, cudaStream_t s,
-                         int sms) {
+                         int sms, const uint16_t* R = nullptr) {
     switch (G) {
-        case 1: launch_tree_combine<1>(P, MN, groups, out, bf16, s, sms); break;
-        case 2: launch_tree_combine<2>(P, MN, groups, out, bf16, s, sms); break;
-        case 4: launch_tree_combine<4>(P, MN, groups, out, bf16, s, sms); break;
-        case 8: launch_tree_combine<8>(P, MN, groups, out, bf16, s, sms); break;
-        case 16: launch_tree_combine<16>(P, MN, groups, out, bf16, s, sms); break;
-        case 32: launch_tree_combine<32>(P, MN, groups, out, bf16, s, sms); break;
-        case 64: launch_tree_combine<64>(P, MN, groups, out, bf16, s, sms); break;
+        case 1: launch_tree_combine<1>(P, MN, groups, out, bf16, R, s, sms); break;
+        case 2: launch_tree_combine<2>(P, MN, groups, out, bf16, R, s, sms); break;
+        case 4: launch_tree_combine<4>(P, MN, groups, out, bf16, R, s, sms); break;
+        case 8: launch_tree_combine<8>(P, MN, groups, out, bf16, R, s, sms); break;
+        case 16: launch_tree_combine<16>(P, MN, groups, out, bf16, R, s, sms); break;
+        case 32: launch_tree_combine<32>(P, MN, groups, out, bf16, R, s, sms); break;
+        case 64: launch_tree_combine<64>(P, MN, groups, out, bf16, R, s, sms); break;
         default: return TBIK_ERR_SHAPE;
     }
     return launch_status();
 }
 
-// Upper levels of the tree after the GEMM wrote F frontier partials.
-tbik_status finish_gemm(const GemmPlan& p, uint8_t* ws, void* C, cudaStream_t s, int sms) {
+// Upper levels of the tree after the GEMM wrote F frontier partials (and the
+// residual R, when given, added to the root before its bf16 rounding).
+tbik_status finish_gemm(const GemmPlan& p, uint8_t* ws, void* C, cudaStream_t s, int sms, const uint16_t* R) {
     if (p.direct) return TBIK_OK;
     const float* P = reinterpret_cast<const float*>(ws + p.off_partials);
     const size_t MN = (size_t)p.M * p.N;
     if (p.noninv) {
         int blocks = (int)((MN + 255) / 256);
         if (blocks > sms * 8) blocks = sms * 8;
-        seq_combine_kernel<<<blocks, 256, 0, s>>>(P, MN, p.T, C, p.out_bf16);
+        seq_combine_kernel<<<blocks, 256, 0, s>>>(P, MN, p.T, C, p.out_bf16, R);
         return launch_status();
     }
-    if (p.T == 1 || p.F == p.T) return tree_combine(P, MN, p.F, 1, C, p.out_bf16, s, sms);
+    if (p.T == 1 || p.F == p.T) return tree_combine(P, MN, p.F, 1, C, p.out_bf16, s, sms, R);
     // T > 1 and F > T: shard partials first (one fp32 buffer per shard), then
     // the cross-shard levels.
     float* Q = reinterpret_cast<float*>(ws + p.off_shards);
     tbik_status st = tree_combine(P, MN, p.F / p.T, p.T, Q, 0, s, sms);
     if (st != TBIK_OK) return st;
-    return tree_combine(Q, MN, p.T, 1, C, p.out_bf16, s, sms);
+    return tree_combine(Q, MN, p.T, 1, C, p.out_bf16, s, sms, R);
 }
 
 // Wait bound in SM cycles at the device's maximum clock (a slower clock only
@@ -335,7 +339,7 @@ unsigned long long wait_cycles(const DeviceInfo* d) {
 }
 
 tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, void* C, uint8_t* ws,
-                     cudaStream_t s, const DeviceInfo* info) {
+                     cudaStream_t s, const DeviceInfo* info, const uint16_t* R = nullptr) {
     const int sms = info->sms;
     if (p.M == 0) return TBIK_OK;
     void* Cg = (p.swiglu && !p.fused) ? (void*)(ws + p.off_gu) : C;  // where the GEMM writes
@@ -358,6 +362,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.out_bf16 = p.out_bf16;
         prm.swiglu = p.fused ? 1 : 0;
         prm.out = Cg;
+        prm.residual = p.direct ? R : nullptr;
         prm.partials = p.direct ? nullptr : reinterpret_cast<float*>(ws + p.off_partials);
         prm.scratch = p.gs ? reinterpret_cast<float*>(ws + p.off_scratch) : nullptr;
         prm.gs = p.gs;
@@ -373,7 +378,10 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
             prm.nl[f] = (short)p.nodes[f].second;
             if (prm.nl[f] != prm.tab_n[0]) prm.tab_n[1] = prm.nl[f];
         }
-        gemm_tc_kernel<EPI_TREE><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+        if (prm.residual)
+            gemm_tc_kernel<EPI_TREE_RES><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+        else
+            gemm_tc_kernel<EPI_TREE><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
     } else {
         ExParams prm;
         memset(&prm, 0, sizeof(prm));
@@ -386,6 +394,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.direct = p.direct;
         prm.out_bf16 = p.out_bf16;
         prm.out = Cg;
+        prm.residual = p.direct ? R : nullptr;
         prm.partials = p.direct ? nullptr : reinterpret_cast<float*>(ws + p.off_partials);
         for (int f = 0; f < p.F; ++f) {
             prm.lo[f] = (short)p.nodes[f].first;
@@ -399,7 +408,7 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
     }
     tbik_status st = launch_status();
     if (st != TBIK_OK) return st;
-    st = finish_gemm(p, ws, Cg, s, sms);
+    st = finish_gemm(p, ws, Cg, s, sms, R);
     if (st != TBIK_OK || !p.swiglu || p.fused) return st;
     const int F = p.N / 2;
     const long long work = (long long)p.M * (F / 8);
@@ -482,6 +491,21 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
 
 // ====================================================================== ABI
 
+// Four leaves (32 elements) per thread when the width allows it: more bytes
+// in flight per thread; the tree is the same.
+template <bool RES>
+void launch_rmsnorm(int nt, const DeviceInfo* info, cudaStream_t s, const uint16_t* x, const uint16_t* res,
+                    const uint16_t* gamma, uint16_t* y, uint16_t* res_out, int tokens, int H, float eps, int T) {
+    switch (nt) {
+        case 32: launch_token_loop(rmsnorm_residual_kernel<32, 1, RES>, 32, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 64: launch_token_loop(rmsnorm_residual_kernel<64, 1, RES>, 64, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 128: launch_token_loop(rmsnorm_residual_kernel<32, 4, RES>, 32, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 256: launch_token_loop(rmsnorm_residual_kernel<64, 4, RES>, 64, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 512: launch_token_loop(rmsnorm_residual_kernel<128, 4, RES>, 128, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+        case 1024: launch_token_loop(rmsnorm_residual_kernel<256, 4, RES>, 256, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
+    }
+}
+
 extern "C" {
 
 const char* tbik_version(void) { return "tbik-b200 0.1 (sm_100a)"; }
@@ -529,6 +553,24 @@ tbik_status tbik_gemm(const uint16_t* A, const uint16_t* B, void* C, int M, int 
     return run_gemm(p, A, B, C, reinterpret_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream), info);
 }
 
+tbik_status tbik_gemm_residual(const uint16_t* A, const uint16_t* B, const uint16_t* R, uint16_t* C, int M, int N,
+                               int K, int T, int leaf, unsigned mode, void* ws, size_t ws_bytes, void* stream) {
+    if (mode & (TBIK_OUT_BF16 | TBIK_SWIGLU_OUT)) return TBIK_ERR_ARG;
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    GemmPlan p;
+    st = plan_gemm(M, N, K, T, leaf, mode | TBIK_OUT_BF16, info->sms, p);
+    if (st != TBIK_OK) return st;
+    if (M == 0) return TBIK_OK;
+    if (!A || !B || !C || !R) return TBIK_ERR_ARG;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C) || !aligned16(R)) return TBIK_ERR_ALIGN;
+    if (p.total > 0 && (!ws || ws_bytes < p.total)) return TBIK_ERR_WORKSPACE;
+    if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return TBIK_ERR_ALIGN;
+    return run_gemm(p, A, B, C, reinterpret_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream), info, R);
+}
+
 tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16_t* gamma, uint16_t* y,
                                   uint16_t* res_out, int tokens, int H, float eps, int T, void* stream) {
     int dev;
@@ -540,20 +582,15 @@ tbik_status tbik_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const 
     const int nt = H / 8;
     if (nt < 32 || nt > 1024 || (nt & (nt - 1)) || nt % T) return TBIK_ERR_SHAPE;
     if (tokens == 0) return TBIK_OK;
-    if (!x || !res || !gamma || !y) return TBIK_ERR_ARG;
-    if (!aligned16(x) || !aligned16(res) || !aligned16(gamma) || !aligned16(y) || (res_out && !aligned16(res_out)))
+    if (!x || !gamma || !y) return TBIK_ERR_ARG;
+    if (!aligned16(x) || (res && !aligned16(res)) || !aligned16(gamma) || !aligned16(y) ||
+        (res_out && !aligned16(res_out)))
         return TBIK_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // Four leaves (32 elements) per thread when the width allows it: more
-    // bytes in flight per thread; the tree is the same.
-    switch (nt) {
-        case 32: launch_token_loop(rmsnorm_residual_kernel<32, 1>, 32, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
-        case 64: launch_token_loop(rmsnorm_residual_kernel<64, 1>, 64, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
-        case 128: launch_token_loop(rmsnorm_residual_kernel<32, 4>, 32, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
-        case 256: launch_token_loop(rmsnorm_residual_kernel<64, 4>, 64, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
-        case 512: launch_token_loop(rmsnorm_residual_kernel<128, 4>, 128, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
-        case 1024: launch_token_loop(rmsnorm_residual_kernel<256, 4>, 256, tokens, info, s, x, res, gamma, y, res_out, tokens, H, eps, T); break;
-    }
+    if (res)
+        launch_rmsnorm<true>(nt, info, s, x, res, gamma, y, res_out, tokens, H, eps, T);
+    else
+        launch_rmsnorm<false>(nt, info, s, x, res, gamma, y, res_out, tokens, H, eps, T);
     return launch_status();
 }
 

@@ -50,9 +50,16 @@ class Decoder:
             self._tables[key] = tb.rope_table(seq, self.cfg.head_dim, 1e6, device=device)
         return self._tables[key]
 
-    def forward(self, ids, targets, pos, *, T: int = 1, tc: bool = True, noninv: bool = False, stream=None):
+    def forward(self, ids, targets, pos, *, T: int = 1, tc: bool = True, noninv: bool = False,
+                fuse_residual: bool = False, stream=None):
         """ids, targets: device int32 [batch, seq]; pos: device int32 [batch*seq]
-        (the position of each token).  Returns fp32 logprobs [batch, seq]."""
+        (the position of each token).  Returns fp32 logprobs [batch, seq].
+
+        fuse_residual: the o and down projections add their fp32 root to the
+        bf16 residual stream h in their last step (tbik_gemm_residual, one
+        rounding: h = bf16(root + h)) and each RMSNorm normalises h with no
+        residual input; otherwise the projection output is rounded to bf16
+        and the RMSNorm adds it to the residual in fp32."""
         torch = tb._torch()
         c = self.cfg
         B, S = ids.shape
@@ -65,10 +72,22 @@ class Decoder:
             tb.gemm(a, w, T=shards, leaf=leaf, tc=tc, noninv=baseline, out_bf16=True, out=out, stream=stream)
             return out
 
+        def add_norm(w, a, leaf, res):
+            """(y, res) after the row-parallel projection a @ w and its residual add."""
+            if fuse_residual:  # res is the stream h, updated in place
+                tb.gemm(a, w, T=T, leaf=leaf, tc=tc, noninv=noninv, residual=res, out=res, stream=stream)
+                y, _ = tb.rmsnorm_residual(res, None, self.gamma, eps=1e-6, T=1, want_res_out=False, stream=stream)
+                return y, res
+            return tb.rmsnorm_residual(dense(a, w, leaf, T, noninv), res, self.gamma, eps=1e-6, T=1, stream=stream)
+
         x = tb.embedding(ids.reshape(-1), self.emb, stream=stream)
-        res = torch.zeros((n, c.d), dtype=bf, device=dev)
         table = self._table(S, dev)
-        y, res = tb.rmsnorm_residual(x, res, self.gamma, eps=1e-6, T=1, stream=stream)
+        if fuse_residual:
+            res = x
+            y, _ = tb.rmsnorm_residual(x, None, self.gamma, eps=1e-6, T=1, want_res_out=False, stream=stream)
+        else:
+            res = torch.zeros((n, c.d), dtype=bf, device=dev)
+            y, res = tb.rmsnorm_residual(x, res, self.gamma, eps=1e-6, T=1, stream=stream)
         for L in self.layers:
             q = dense(y, L["wq"], c.leaf)
             k = dense(y, L["wk"], c.leaf)
@@ -77,12 +96,10 @@ class Decoder:
             tb.rope_swiglu(q=q3, k=k3, pos=pos, table=table, q_out=q3, k_out=k3, stream=stream)
             o = tb.attention(q.view(B, S, c.heads, c.head_dim), k.view(B, S, c.heads, c.head_dim),
                              v.view(B, S, c.heads, c.head_dim), stream=stream)
-            a = dense(o.view(n, c.d), L["wo"], c.leaf, T, noninv)
-            y, res = tb.rmsnorm_residual(a, res, self.gamma, eps=1e-6, T=1, stream=stream)
+            y, res = add_norm(L["wo"], o.view(n, c.d), c.leaf, res)
             act = torch.empty((n, c.ffn), dtype=bf, device=dev)
             tb.gemm(y, L["wgu"], T=1, leaf=c.leaf, tc=tc, swiglu=True, out=act, stream=stream)
-            m = dense(act, L["wd"], c.leaf_ffn, T, noninv)
-            y, res = tb.rmsnorm_residual(m, res, self.gamma, eps=1e-6, T=1, stream=stream)
+            y, res = add_norm(L["wd"], act, c.leaf_ffn, res)
         lp = tb.logprob(y, self.lm_head, targets.reshape(-1), T=T, leaf=c.leaf, tc=tc, noninv=noninv, stream=stream)
         return lp.view(B, S)
 

@@ -75,6 +75,7 @@ def _load():
                 "oracle_gemm_noninv": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp]),
                 "oracle_gemm_f64": (None, [vp, vp, i32, i32, i32, i32, vp]),
                 "oracle_rmsnorm_residual": (i32, [vp, vp, vp, vp, vp, i32, i32, f32, i32]),
+                "oracle_add_residual_bf16": (None, [vp, vp, vp, i64]),
                 "oracle_rope_table": (None, [vp, i32, i32, f64]),
                 "oracle_rope": (None, [vp, vp, vp, vp, i32, i32, i32]),
                 "oracle_swiglu_bf16": (None, [vp, vp, vp, i64]),
@@ -176,6 +177,26 @@ def gemm_noninv(a_bits, b_bits, *, b_nk: bool, T: int, shards: bool = False):
     return (c, q) if shards else c
 
 
+def add_residual_bf16(root, r_bits) -> np.ndarray:
+    """bf16 bits of root + f32(R): one fp32 add, one RNE rounding."""
+    c, pc = _c(root, np.float32)
+    r, pr = _c(r_bits, np.uint16)
+    if c.shape != r.shape:
+        raise ValueError("root and residual shapes differ")
+    out = np.empty(c.shape, dtype=np.uint16)
+    _load().oracle_add_residual_bf16(pc, pr, out.ctypes.data, c.size)
+    return out
+
+
+def gemm_residual(a_bits, b_bits, r_bits, *, b_nk: bool, T: int, leaf: int, noninv: bool = False):
+    """bf16 bits of the tree GEMM's fp32 root (or the baseline's) plus the residual R."""
+    if noninv:
+        root = gemm_noninv(a_bits, b_bits, b_nk=b_nk, T=T)
+    else:
+        root = gemm_tree(a_bits, b_bits, b_nk=b_nk, T=T, leaf=leaf)
+    return add_residual_bf16(root, r_bits)
+
+
 def gemm_f64(a_bits, b_bits, *, b_nk: bool):
     a, pa = _c(a_bits, np.uint16)
     b, pb = _c(b_bits, np.uint16)
@@ -189,8 +210,11 @@ def gemm_f64(a_bits, b_bits, *, b_nk: bool):
 # ------------------------------------------------------------ reductions
 
 def rmsnorm_residual(x_bits, res_bits, gamma_bits, *, eps: float = 1e-6, T: int = 1):
+    """y and res_out bf16 bits; res_bits None: no residual input (r = f32(x))."""
     x, px = _c(x_bits, np.uint16)
-    r, pr = _c(res_bits, np.uint16)
+    pr = None
+    if res_bits is not None:
+        r, pr = _c(res_bits, np.uint16)
     g, pg = _c(gamma_bits, np.uint16)
     tokens, H = x.shape
     y = np.empty_like(x)

@@ -283,6 +283,7 @@ void oracle_gemm_f64(const uint16_t* A, const uint16_t* B, int b_nk, int M, int 
  *   ss      = TREE(Q, 0, T),  Q_t = TREE(P, t*nl/T, nl/T),  nl = H/8     (R1, R3)
  *   ms      = ss / H;  inv = 1 / sqrt(ms + eps)   (each op correctly rounded)
  *   y       = bf16((r * inv) * gamma);  res_out = bf16(r)
+ * res == NULL means no residual input: r = f32(x) (no addition).
  * Returns 0, or -1 when H is not a multiple of 8 or T does not divide H/8.
  */
 int oracle_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16_t* gamma,
@@ -294,8 +295,12 @@ int oracle_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16
     float* Q = (float*)malloc(sizeof(float) * (size_t)T);
     for (int t = 0; t < tokens; ++t) {
         const uint16_t* xr = x + (size_t)t * H;
-        const uint16_t* rr = res + (size_t)t * H;
-        for (int h = 0; h < H; ++h) r[h] = bf(xr[h]) + bf(rr[h]);
+        if (res) {
+            const uint16_t* rr = res + (size_t)t * H;
+            for (int h = 0; h < H; ++h) r[h] = bf(xr[h]) + bf(rr[h]);
+        } else {
+            for (int h = 0; h < H; ++h) r[h] = bf(xr[h]);
+        }
         for (int j = 0; j < nl; ++j) {
             float acc = 0.0f;
             for (int e = 0; e < 8; ++e) acc = fmaf(r[8 * j + e], r[8 * j + e], acc);
@@ -315,6 +320,15 @@ int oracle_rmsnorm_residual(const uint16_t* x, const uint16_t* res, const uint16
     free(P);
     free(Q);
     return 0;
+}
+
+/*
+ * Residual add at the end of a row-parallel projection ([RLA]: the residual
+ * add in fp32, one rounding): C[i] = bf16(root[i] + f32(R[i])), root the fp32
+ * result of oracle_gemm_tree (or of oracle_gemm_noninv for the baseline).
+ */
+void oracle_add_residual_bf16(const float* root, const uint16_t* R, uint16_t* C, size_t n) {
+    for (size_t i = 0; i < n; ++i) C[i] = bf16_rne(root[i] + bf(R[i]));
 }
 
 /* -------------------------------------------------------------- RoPE */

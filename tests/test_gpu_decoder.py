@@ -1,6 +1,7 @@
 """End-to-end decoder (Llama-style, pre-norm) built from the library's calls:
 per-token logprobs bit-exact to the oracle decoder in exact-order mode (small
-configuration), and in tensor-core mode bitwise identical across T in
+configuration, with the residual add in the RMSNorm or fused into the o and
+down projections), and in tensor-core mode bitwise identical across T in
 {1,2,4,8} and across batch compositions at the full configuration (4 layers,
 d 2048, 16 heads of 128, ffn 5632, vocab 32000, batch 8 x seq 2048), while the
 non-invariant baseline diverges with T."""
@@ -53,6 +54,18 @@ def test_small_exact_matches_oracle_decoder(small):
     assert tbik.get_error() == tbik.TBIK_OK
 
 
+def test_small_fused_residual_exact_matches_oracle_decoder(small):
+    cfg, w, dec, ids, tg = small
+    for T, noninv in ((1, False), (8, False), (4, True)):
+        got = run(dec, ids, tg, T=T, tc=False, noninv=noninv, fuse_residual=True)
+        ref = odec.forward(cfg, w, ids, tg, T=T, noninv=noninv, fuse_residual=True)
+        assert np.array_equal(u32(got), u32(ref)), (T, noninv)
+    outs = [run(dec, ids, tg, T=T, tc=True, fuse_residual=True) for T in (1, 2, 8)]
+    for o in outs[1:]:
+        assert np.array_equal(u32(o), u32(outs[0]))
+    assert tbik.get_error() == tbik.TBIK_OK
+
+
 def test_small_tc_invariant_and_close_to_oracle(small):
     cfg, w, dec, ids, tg = small
     outs = [run(dec, ids, tg, T=T, tc=True) for T in (1, 2, 4, 8)]
@@ -87,6 +100,11 @@ def test_full_config_tc_invariant_over_T_and_batch(full):
     assert np.array_equal(u32(sub), u32(base[[6, 1]]))
     # a plausible scale for random init: close to -ln(vocab)
     assert abs(float(base.mean()) + np.log(cfg["vocab"])) < 0.5
+    # the residual add fused into the o and down projections: invariant too,
+    # and within bf16 rounding of the unfused composition
+    fused = run(dec, ids, tg, T=1, tc=True, fuse_residual=True)
+    assert np.array_equal(u32(run(dec, ids, tg, T=8, tc=True, fuse_residual=True)), u32(fused))
+    assert float(np.mean(np.abs(fused - base))) < 2e-2
     assert tbik.get_error() == tbik.TBIK_OK
 
 

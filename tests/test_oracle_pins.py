@@ -230,6 +230,61 @@ def test_noninv_baseline_structure_and_divergence():
     assert any(not np.array_equal(bits(outs[0]), bits(o)) for o in outs[1:])
 
 
+def test_residual_add_integer_exact_and_single_rounding():
+    """bf16(root + R): with integer inputs the sum is an integer below 256, exactly
+    representable, so it must equal the int64 result (a dropped R or a wrong sign
+    fails); a root just below a bf16 rounding midpoint plus a small R rounds up,
+    while rounding the root first would round down (one rounding, not two)."""
+    M, N, K = 6, 10, 16
+    a = synth.int_bf16(95, (M, K), 3)
+    b = synth.int_bf16(96, (K, N), 3)
+    r = synth.int_bf16(97, (M, N), 100)
+    exact = F(a).astype(np.int64) @ F(b).astype(np.int64) + F(r).astype(np.int64)
+    for T, leaf in ((1, 16), (2, 4), (4, 2)):
+        c = oracle.gemm_residual(a, b, r, b_nk=False, T=T, leaf=leaf)
+        assert np.array_equal(F(c).astype(np.int64), exact)
+    one = oracle.bf16_rne
+    a1 = np.array([[one(1.0), one(2.0 ** -8), one(-(2.0 ** -12)), 0]], dtype=np.uint16)
+    b1 = np.full((4, 1), one(1.0), dtype=np.uint16)
+    r1 = np.array([[one(2.0 ** -11)]], dtype=np.uint16)
+    c1 = oracle.gemm_residual(a1, b1, r1, b_nk=False, T=1, leaf=4)
+    assert F(c1)[0, 0] == 1.0 + 2.0 ** -7
+    twice = one(float(np.float32(F(np.array([one(1.0 + 2.0 ** -8 - 2.0 ** -12)]))[0]) + np.float32(2.0 ** -11)))
+    assert F(np.array([twice]))[0] == 1.0
+
+
+def test_residual_add_zero_operands():
+    """B = 0: root = +0 and C = R (a -0 residual becomes +0, as +0 + -0 = +0);
+    R = +0: C is the single rounding of the root."""
+    M, N, K = 3, 8, 64
+    a = synth.normal_bf16(98, (M, K))
+    r = synth.normal_bf16(99, (M, N))
+    r[0, 0] = 0x8000  # -0
+    c = oracle.gemm_residual(a, np.zeros((K, N), dtype=np.uint16), r, b_nk=False, T=2, leaf=16)
+    expect = r.copy()
+    expect[0, 0] = 0
+    assert np.array_equal(c, expect)
+    b = synth.normal_bf16(100, (K, N), std=0.1)
+    for noninv in (False, True):
+        root = (oracle.gemm_noninv(a, b, b_nk=False, T=4) if noninv
+                else oracle.gemm_tree(a, b, b_nk=False, T=4, leaf=16))
+        c0 = oracle.gemm_residual(a, b, np.zeros((M, N), dtype=np.uint16), b_nk=False, T=4, leaf=16, noninv=noninv)
+        assert np.array_equal(c0, oracle.bf16_rne_array(root))
+
+
+def test_rmsnorm_without_residual_input():
+    """res = None means r = f32(x): the same as a +0 residual for rows without -0,
+    and y = gamma for a row of ones (r = 1, ms = 1, inv = 1 with eps = 0)."""
+    d = synth.reduction_inputs(7, H=1024, F=16)
+    zero = np.zeros_like(d["x"])
+    y0, r0 = oracle.rmsnorm_residual(d["x"], zero, d["gamma"], eps=1e-6)
+    y1, r1 = oracle.rmsnorm_residual(d["x"], None, d["gamma"], eps=1e-6)
+    assert np.array_equal(y0, y1) and np.array_equal(r1, d["x"]) and np.array_equal(r0, r1)
+    x = np.full((1, 1024), oracle.bf16_rne(1.0), dtype=np.uint16)
+    y, _ = oracle.rmsnorm_residual(x, None, d["gamma"], eps=0.0)
+    assert np.array_equal(y[0], d["gamma"])
+
+
 # ---------------------------------------------------------------- exp / log
 
 def test_exp_log_specs_against_libm():
