@@ -56,7 +56,8 @@ def parse():
     ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decoder", action="store_true", help="skip the end-to-end decoder component")
-    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "attention"], default=None,
+    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "attention", "swiglu", "rmsnorm"],
+                    default=None,
                     help="run only one call of the path, `--steps` times, for ncu captures (no JSON line)")
     ap.add_argument("--tokens", type=int, default=M_TOK, help="tokens per call in --profile-case")
     return ap.parse_args()
@@ -405,6 +406,8 @@ def run_tbik(args):
                        device=dev)
     g_t8 = avg_ms(lambda: tbik.gemm(A, B, T=8, leaf=LEAF, tc=True, out_bf16=True, out=hid2, workspace=gws8))
     tbik.get_error(stream)
+    pk = peaks()
+    red8k = reductions_component(8192, dev, stream, gamma, table, pk["hbm"])
     dec = None
     if not args.no_decoder:
         try:  # an extra measurement: a failure here must not cost the main line
@@ -413,7 +416,6 @@ def run_tbik(args):
             dec = {"error": f"{type(e).__name__}: {e}"[:300]}
             torch.cuda.synchronize()
 
-    pk = peaks()
     lp_ms = lp_live_ms
     achieved = LOGPROB_FLOP / (lp_ms * 1e-3) / 1e12
     ms_step = ms_total / args.steps
@@ -439,6 +441,7 @@ def run_tbik(args):
             "rope_gbs": gb(2 * 2 * M_TOK * HEADS * HEAD_DIM * 2 + M_TOK * (4 + HEAD_DIM * 4), comp_ms["rope"]),
             "swiglu_gbs": gb(3 * M_TOK * F * 2, comp_ms["swiglu"]),
             "ms": comp_ms,
+            "reductions_8192_tokens": red8k,
             "overhead_vs_noninv": {"gemm": g_inv / g_non - 1.0, "logprob": l_inv / l_non - 1.0,
                                    "gemm_ms": [g_inv, g_non], "logprob_ms": [l_inv, l_non]},
             "decoder_e2e": dec,
@@ -464,6 +467,47 @@ def run_tbik(args):
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     return 0
+
+
+def reductions_component(tokens, dev, stream, gamma, table, copy_gbs):
+    """RMSNorm, RoPE and SwiGLU at `tokens` tokens (8192: the size their HBM
+    bar is set at): each averaged over 20 back-to-back calls after 3 warm-up
+    calls; every call moves more than the 126 MB L2 (268, 273 and 705 MB)."""
+    import torch
+
+    import invariant_tree_ordered_b200 as tbik
+
+    d = synth.reduction_inputs(tokens, F=F)
+    t = {k: (synth.as_torch_bf16(v) if v.dtype == np.uint16 else torch.from_numpy(v)).to(dev)
+         for k, v in d.items() if k != "gamma"}
+    y, ro = torch.empty_like(t["x"]), torch.empty_like(t["x"])
+    qo, ko = torch.empty_like(t["q"]), torch.empty_like(t["k"])
+    act = torch.empty_like(t["g"])
+    calls = {
+        "rmsnorm": lambda: tbik.rmsnorm_residual(t["x"], t["res"], gamma, eps=1e-6, T=1, y=y, res_out=ro,
+                                                 stream=stream),
+        "rope": lambda: tbik.rope_swiglu(q=t["q"], k=t["k"], pos=t["pos"], table=table, q_out=qo, k_out=ko,
+                                         stream=stream),
+        "swiglu": lambda: tbik.rope_swiglu(g=t["g"], u=t["u"], out=act, stream=stream),
+    }
+    nbytes = {"rmsnorm": 4 * tokens * H * 2,
+              "rope": 2 * 2 * tokens * HEADS * HEAD_DIM * 2 + tokens * (4 + HEAD_DIM * 4),
+              "swiglu": 3 * tokens * F * 2}
+    out = {"tokens": tokens}
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for k, fn in calls.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(20):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / 20
+        gbs = nbytes[k] / (ms * 1e-3) / 1e9
+        out[k] = {"us": ms * 1e3, "gbs": gbs, "frac_of_measured_copy": gbs / copy_gbs}
+    return out
 
 
 def decoder_component(dev, stream):
@@ -550,6 +594,15 @@ def run_profile_case(args):
         qkv = [synth.as_torch_bf16(synth.normal_bf16(450 + i, (Bq, S, NH, D))).to(dev) for i in range(3)]
         out = torch.empty_like(qkv[0])
         call = lambda: tbik.attention(*qkv, out=out)  # noqa: E731
+    elif args.profile_case in ("swiglu", "rmsnorm"):
+        d = synth.reduction_inputs(M, F=F)
+        t = {k: synth.as_torch_bf16(d[k]).to(dev) for k in ("x", "res", "gamma", "g", "u")}
+        if args.profile_case == "swiglu":
+            out = torch.empty_like(t["g"])
+            call = lambda: tbik.rope_swiglu(g=t["g"], u=t["u"], out=out)  # noqa: E731
+        else:
+            y, ro = torch.empty_like(t["x"]), torch.empty_like(t["x"])
+            call = lambda: tbik.rmsnorm_residual(t["x"], t["res"], t["gamma"], eps=1e-6, y=y, res_out=ro)  # noqa: E731
     elif args.profile_case == "logprob":
         h = synth.as_torch_bf16(synth.normal_bf16(30, (M, H))).to(dev)
         w = synth.as_torch_bf16(synth.normal_bf16(31, (V, H), std=0.02)).to(dev)

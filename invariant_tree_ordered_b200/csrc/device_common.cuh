@@ -68,9 +68,10 @@ __device__ __forceinline__ float pow2i(int n) { return __uint_as_float((uint32_t
 // scale by 2^(k/2) exactly, then by 2^(k-k/2) (one rounding).
 // Instruction choices that keep those bits: rint of y = x*log2e (|y| < 151)
 // is (y + 1.5*2^23) - 1.5*2^23 in round-to-nearest-even, and the integer k
-// sits in the low bits of that sum; when 2^k is a normal float (k in
-// [-126, 127]) the product p*2^k is rounded once, exactly as the two-step
-// scaling rounds it (its first step, by 2^(k/2), is exact).
+// sits in the low bits of that sum.  |r| <= ln2/2 (plus rounding), so p lies
+// in [0.70, 1.42] and has exponent -1 or 0; for k in [-125, 127] the product
+// p*2^k is then a normal float, exact, and its bits are p's with k added to
+// the exponent field (one integer add).  Other k take the two-step scaling.
 __device__ __forceinline__ float exp_spec(float x) {
     if (x != x) return __fadd_rn(x, x);
     x = fminf(fmaxf(x, -104.0f), 89.0f);
@@ -88,7 +89,7 @@ __device__ __forceinline__ float exp_spec(float x) {
     p = __fmaf_rn(p, r, 0.5f);
     p = __fmaf_rn(p, r, 1.0f);
     p = __fmaf_rn(p, r, 1.0f);
-    if (k >= -126 && k <= 127) return __fmul_rn(p, pow2i(k));
+    if (k >= -125 && k <= 127) return __int_as_float(__float_as_int(p) + (int)((uint32_t)k << 23));
     const int k1 = k / 2;
     const int k2 = k - k1;
     return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));

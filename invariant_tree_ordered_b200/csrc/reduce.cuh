@@ -188,8 +188,8 @@ struct Vec8<1> {
     float4 a, b;
 };
 
-template <int IN_F32>
-__device__ __forceinline__ Vec8<IN_F32> load_vec8(const void* p, long long i) {
+template <int IN_F32, typename IDX>
+__device__ __forceinline__ Vec8<IN_F32> load_vec8(const void* p, IDX i) {
     Vec8<IN_F32> r;
     if constexpr (IN_F32) {
         const float4* q = reinterpret_cast<const float4*>(p) + 2 * i;
@@ -211,15 +211,18 @@ __device__ __forceinline__ void unpack_vec8(const Vec8<IN_F32>& r, float (&f)[8]
     }
 }
 
-template <int IN_F32>
+// Grid-stride loop over 8-element vectors, the next vector's loads issued
+// before the current one is computed.  Vector indices in IDX (32-bit when
+// every index the loop forms fits, for cheaper address arithmetic).
+template <int IN_F32, typename IDX>
 __global__ void swiglu_kernel(const void* __restrict__ g, const void* __restrict__ u, uint16_t* out, long long n) {
-    const long long nv = n >> 3;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    const IDX nv = (IDX)(n >> 3);
+    const IDX stride = (IDX)gridDim.x * blockDim.x;
+    IDX i = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= nv) return;
     Vec8<IN_F32> cg = load_vec8<IN_F32>(g, i), cu = load_vec8<IN_F32>(u, i);
     while (true) {
-        const long long inext = i + stride;
+        const IDX inext = i + stride;
         const bool more = inext < nv;
         Vec8<IN_F32> ng, nu;
         if (more) {

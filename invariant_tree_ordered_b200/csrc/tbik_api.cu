@@ -706,10 +706,20 @@ tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) 
         const long long nv = a->n / 8;
         long long blocks = (nv + 255) / 256;
         if (blocks > (long long)info->sms * 16) blocks = (long long)info->sms * 16;
-        if (a->in_f32)
-            swiglu_kernel<1><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
-        else
-            swiglu_kernel<0><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+        // 32-bit indices when every index the loop forms, doubled for the fp32
+        // inputs' float4 pairs, stays below 2^32
+        const bool narrow = (unsigned long long)nv + (unsigned long long)blocks * 256 < (1ull << 31);
+        if (a->in_f32) {
+            if (narrow)
+                swiglu_kernel<1, uint32_t><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+            else
+                swiglu_kernel<1, long long><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+        } else {
+            if (narrow)
+                swiglu_kernel<0, uint32_t><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+            else
+                swiglu_kernel<0, long long><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+        }
         if ((st = launch_status()) != TBIK_OK) return st;
     }
     return TBIK_OK;
