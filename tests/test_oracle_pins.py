@@ -527,3 +527,31 @@ def test_attention_within_binary64_softmax(chunk):
     # one bf16 rounding (half an ulp of 2^-7 relative) plus fp32 reduction error
     tol = np.abs(ref) * (2.0**-8 + 2e-5) + 1e-6
     assert np.all(np.abs(got - ref) <= tol)
+
+
+# ----------------------------------------------------------------- decoder
+
+def test_decoder_zero_layers_leave_the_residual_stream_unchanged():
+    """With every layer weight zero, attention gives exactly 0 (v = 0) and so does
+    the FFN (silu(0) * 0 = 0), so the oracle decoder must reduce to
+    RMSNorm(embedding[ids]) followed by the logprob of the targets, with the
+    residual add in the RMSNorm or fused into the projections alike (a residual
+    added twice, a misaligned target or a skipped norm fails); a zero lm_head on
+    top gives -ln V for every token."""
+    import oracle.decoder as odec
+    cfg = synth.DECODER_SMALL
+    w = synth.decoder_weights(cfg)
+    for layer in w["layers"]:
+        for k in layer:
+            layer[k] = np.zeros_like(layer[k])
+    ids, tg = synth.decoder_tokens(cfg)
+    x = w["emb"][ids.reshape(-1)]
+    y, _ = oracle.rmsnorm_residual(x, None, w["gamma"], eps=1e-6)
+    expect = oracle.logprob(y, w["lm_head"], tg.reshape(-1).astype(np.int32), T=1,
+                            leaf=cfg["leaf"]).reshape(ids.shape)
+    for fuse in (False, True):
+        got = odec.forward(cfg, w, ids, tg, T=2, fuse_residual=fuse)
+        assert np.array_equal(bits(got), bits(expect)), fuse
+    w["lm_head"] = np.zeros_like(w["lm_head"])
+    got = odec.forward(cfg, w, ids, tg, T=1)
+    assert np.allclose(got, -math.log(cfg["vocab"]), rtol=0, atol=1e-6)
