@@ -135,6 +135,13 @@ def _stream_handle(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _need_out(t, dtype, shape, name="out"):
+    """A caller-provided output: a contiguous CUDA tensor of this dtype and shape."""
+    _need(t, dtype, name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
 def _need(t, dtype, name):
     torch = _torch()
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
@@ -188,6 +195,7 @@ def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = F
             raise ValueError("residual must be [M, N]")
         if out is None:
             out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+        _need_out(out, torch.bfloat16, (M, N))
         ws, wsb = _workspace(lib.tbik_gemm_workspace(M, N, K, T, leaf, mode | OUT_BF16), A.device, workspace)
         _check(lib.tbik_gemm_residual(_ptr(A), _ptr(B), _ptr(residual), _ptr(out), M, N, K, T, leaf, mode,
                                       _ptr(ws), wsb, _stream_handle(stream)), "tbik_gemm_residual")
@@ -195,11 +203,11 @@ def gemm(A, B, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = F
     mode |= OUT_BF16 if out_bf16 else OUT_F32
     if swiglu:
         mode |= SWIGLU_OUT
+    out_dtype = torch.bfloat16 if (swiglu or out_bf16) else torch.float32
+    out_shape = (M, N // 2) if swiglu else (M, N)
     if out is None:
-        if swiglu:
-            out = torch.empty((M, N // 2), dtype=torch.bfloat16, device=A.device)
-        else:
-            out = torch.empty((M, N), dtype=torch.bfloat16 if out_bf16 else torch.float32, device=A.device)
+        out = torch.empty(out_shape, dtype=out_dtype, device=A.device)
+    _need_out(out, out_dtype, out_shape)
     ws, wsb = _workspace(lib.tbik_gemm_workspace(M, N, K, T, leaf, mode), A.device, workspace)
     _check(lib.tbik_gemm(_ptr(A), _ptr(B), _ptr(out), M, N, K, T, leaf, mode, _ptr(ws), wsb,
                          _stream_handle(stream)), "tbik_gemm")
@@ -213,11 +221,20 @@ def rmsnorm_residual(x, res, gamma, *, eps: float = 1e-6, T: int = 1, y=None, re
     for t, n in ((x, "x"), (res, "res"), (gamma, "gamma")):
         if t is not None or n != "res":  # res None: no residual input, r = f32(x)
             _need(t, torch.bfloat16, n)
+    if x.dim() != 2:
+        raise ValueError("x must be [tokens, H]")
     tokens, H = x.shape
+    if res is not None and res.shape != x.shape:
+        raise ValueError("res must have the shape of x")
+    if tuple(gamma.shape) != (H,):
+        raise ValueError("gamma must be [H]")
     if y is None:
         y = torch.empty_like(x)
+    _need_out(y, torch.bfloat16, x.shape, "y")
     if res_out is None and want_res_out:
         res_out = torch.empty_like(x)
+    if res_out is not None:
+        _need_out(res_out, torch.bfloat16, x.shape, "res_out")
     _check(lib.tbik_rmsnorm_residual(_ptr(x), _ptr(res), _ptr(gamma), _ptr(y), _ptr(res_out), tokens, H,
                                      float(eps), T, _stream_handle(stream)), "tbik_rmsnorm_residual")
     return y, res_out
@@ -242,11 +259,26 @@ def rope_swiglu(*, q=None, k=None, pos=None, table=None, q_out=None, k_out=None,
         _need(ref, torch.bfloat16, "q/k")
         _need(pos, torch.int32, "pos")
         _need(table, torch.float32, "table")
+        if ref.dim() != 3:
+            raise ValueError("q and k must be [tokens, heads, head_dim]")
         tokens, heads, hd = ref.shape
+        for t, n in ((q, "q"), (k, "k")):
+            if t is not None:
+                _need(t, torch.bfloat16, n)
+                if t.shape != ref.shape:
+                    raise ValueError("q and k must share one shape")
+        if pos.numel() != tokens:
+            raise ValueError("pos must hold one position per token")
+        if table.dim() != 3 or tuple(table.shape[1:]) != (hd // 2, 2):
+            raise ValueError("table must be [max_pos, head_dim/2, 2]")
         if q is not None and q_out is None:
             q_out = torch.empty_like(q)
         if k is not None and k_out is None:
             k_out = torch.empty_like(k)
+        if q is not None:
+            _need_out(q_out, torch.bfloat16, ref.shape, "q_out")
+        if k is not None:
+            _need_out(k_out, torch.bfloat16, ref.shape, "k_out")
         a.q, a.k, a.q_out, a.k_out = _ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out)
         a.pos, a.table = _ptr(pos), _ptr(table)
         a.tokens, a.heads, a.head_dim, a.max_pos = tokens, heads, hd, table.shape[0]
@@ -255,8 +287,11 @@ def rope_swiglu(*, q=None, k=None, pos=None, table=None, q_out=None, k_out=None,
             raise TypeError("g and u must both be bf16 or both fp32")
         _need(g, g.dtype, "g")
         _need(u, g.dtype, "u")
+        if u.shape != g.shape:
+            raise ValueError("g and u must share one shape")
         if out is None:
             out = torch.empty(g.shape, dtype=torch.bfloat16, device=g.device)
+        _need_out(out, torch.bfloat16, g.shape)
         a.g, a.u, a.out, a.n, a.in_f32 = _ptr(g), _ptr(u), _ptr(out), g.numel(), int(g.dtype == torch.float32)
     _check(lib.tbik_rope_swiglu_fp32(ctypes.byref(a), _stream_handle(stream)), "tbik_rope_swiglu_fp32")
     return q_out, k_out, out
@@ -274,6 +309,7 @@ def attention(q, k, v, *, out=None, chunk: int = 64, stream=None):
     B, S, NH, D = q.shape
     if out is None:
         out = torch.empty_like(q)
+    _need_out(out, torch.bfloat16, q.shape)
     _check(lib.tbik_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, NH, D, chunk, _stream_handle(stream)),
            "tbik_attention")
     return out
@@ -288,6 +324,7 @@ def embedding(ids, table, *, out=None, stream=None):
     V, d = table.shape
     if out is None:
         out = torch.empty((ids.numel(), d), dtype=torch.bfloat16, device=table.device)
+    _need_out(out, torch.bfloat16, (ids.numel(), d))
     _check(lib.tbik_embedding(_ptr(ids), _ptr(table), _ptr(out), ids.numel(), V, d, _stream_handle(stream)),
            "tbik_embedding")
     return out
@@ -301,12 +338,20 @@ def transpose(x, *, out=None, stream=None):
     rows, cols = x.shape
     if out is None:
         out = torch.empty((cols, rows), dtype=torch.bfloat16, device=x.device)
+    _need_out(out, torch.bfloat16, (cols, rows))
     _check(lib.tbik_transpose(_ptr(x), _ptr(out), rows, cols, _stream_handle(stream)), "tbik_transpose")
     return out
 
 
 def logprob_workspace(M, V, H, T, leaf, mode) -> int:
     return int(load_library().tbik_logprob_workspace(M, V, H, T, leaf, mode))
+
+
+def _logprob_shapes(hidden, W, targets):
+    if hidden.dim() != 2 or W.dim() != 2 or W.shape[1] != hidden.shape[1]:
+        raise ValueError("hidden must be [M, H] and W_lm [V, H]")
+    if targets.numel() != hidden.shape[0]:
+        raise ValueError("targets must hold one index per row of hidden")
 
 
 def logprob(hidden, W, targets, *, T: int = 1, leaf: int = 256, tc: bool = True, noninv: bool = False, out=None,
@@ -318,9 +363,11 @@ def logprob(hidden, W, targets, *, T: int = 1, leaf: int = 256, tc: bool = True,
     _need(targets, torch.int32, "targets")
     M, H = hidden.shape
     V = W.shape[0]
+    _logprob_shapes(hidden, W, targets)
     mode = (TC if tc else EXACT) | (NONINV if noninv else 0)
     if out is None:
         out = torch.empty(M, dtype=torch.float32, device=hidden.device)
+    _need_out(out, torch.float32, (M,))
     ws, wsb = _workspace(lib.tbik_logprob_workspace(M, V, H, T, leaf, mode), hidden.device, workspace)
     _check(lib.tbik_logprob(_ptr(hidden), _ptr(W), _ptr(targets), _ptr(out), M, V, H, T, leaf, mode, _ptr(ws), wsb,
                             _stream_handle(stream)), "tbik_logprob")
@@ -356,9 +403,11 @@ def logprob_noalloc(hidden, W, targets, *, T: int = 1, leaf: int = 256, noninv: 
     _need(targets, torch.int32, "targets")
     M, H = hidden.shape
     V = W.shape[0]
+    _logprob_shapes(hidden, W, targets)
     mode = TC | (NONINV if noninv else 0)
     if out is None:
         out = torch.empty(M, dtype=torch.float32, device=hidden.device)
+    _need_out(out, torch.float32, (M,))
     _check(lib.tbik_logprob_noalloc(_ptr(hidden), _ptr(W), _ptr(targets), _ptr(out), M, V, H, T, leaf, mode,
                                     _stream_handle(stream)), "tbik_logprob_noalloc")
     return out
