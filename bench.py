@@ -46,6 +46,9 @@ WORKLOAD = ("tbik hot path, M=4096 tokens/step: residual RMSNorm H=4096 -> RoPE 
 GEMM_FLOP = 2.0 * M_TOK * F * H
 LOGPROB_FLOP = 2.0 * M_TOK * V * H
 KERNELS_PER_STEP = 6  # rmsnorm, rope, swiglu, gemm, logprob gemm+stats, logprob row tree
+# fp32 FMA peak of the exact-order (CUDA-core) mode: 148 SMs x 128 fp32 lanes x
+# 2 flop x 1.965 GHz (the maximum SM clock)
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def parse():
@@ -56,7 +59,8 @@ def parse():
     ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decoder", action="store_true", help="skip the end-to-end decoder component")
-    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "attention", "swiglu", "rmsnorm"],
+    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "gemm-exact", "attention", "swiglu",
+                                               "rmsnorm"],
                     default=None,
                     help="run only one call of the path, `--steps` times, for ncu captures (no JSON line)")
     ap.add_argument("--tokens", type=int, default=M_TOK, help="tokens per call in --profile-case")
@@ -406,6 +410,15 @@ def run_tbik(args):
                        device=dev)
     g_t8 = avg_ms(lambda: tbik.gemm(A, B, T=8, leaf=LEAF, tc=True, out_bf16=True, out=hid2, workspace=gws8))
     tbik.get_error(stream)
+    try:  # the exact-order (CUDA-core) mode of the same down_proj call: an extra measurement
+        ex_ms = avg_ms(lambda: tbik.gemm(A, B, T=1, leaf=LEAF, tc=False, out_bf16=True, out=hid2), 3)
+        ex_tf = GEMM_FLOP / (ex_ms * 1e-3) / 1e12
+        exact = {"down_proj_exact_ms": ex_ms, "down_proj_exact_tflops": ex_tf, "bound": "alu",
+                 "peak_tflops": FP32_FMA_PEAK_TFLOPS, "frac": ex_tf / FP32_FMA_PEAK_TFLOPS,
+                 "status": int(tbik.get_error(stream))}
+    except Exception as e:  # noqa: BLE001
+        exact = {"error": f"{type(e).__name__}: {e}"[:300]}
+        torch.cuda.synchronize()
     pk = peaks()
     red8k = reductions_component(8192, dev, stream, gamma, table, pk["hbm"])
     dec = None
@@ -442,6 +455,7 @@ def run_tbik(args):
             "swiglu_gbs": gb(3 * M_TOK * F * 2, comp_ms["swiglu"]),
             "ms": comp_ms,
             "reductions_8192_tokens": red8k,
+            "exact_mode": exact,
             "overhead_vs_noninv": {"gemm": g_inv / g_non - 1.0, "logprob": l_inv / l_non - 1.0,
                                    "gemm_ms": [g_inv, g_non], "logprob_ms": [l_inv, l_non]},
             "decoder_e2e": dec,
@@ -612,20 +626,28 @@ def run_profile_case(args):
         call = lambda: tbik.logprob(h, w, t, T=1, leaf=LEAF, tc=True, out=out, workspace=ws)  # noqa: E731
     else:
         T = 8 if args.profile_case == "gemm-t8" else 1
+        tc = args.profile_case != "gemm-exact"
         std = 0.02 * np.sqrt(H)
         g = synth.as_torch_bf16(synth.normal_bf16(11, (M, F), std=std)).to(dev)
         u = synth.as_torch_bf16(synth.normal_bf16(12, (M, F), std=std)).to(dev)
         a = tbik.rope_swiglu(g=g, u=u)[2]
         b = synth.as_torch_bf16(synth.down_proj_weight(F, H, "kn")).to(dev)
-        mode = tbik.TC | tbik.OUT_BF16
+        mode = (tbik.TC if tc else tbik.EXACT) | tbik.OUT_BF16
         ws = torch.empty(max(tbik.gemm_workspace(M, H, F, T, LEAF, mode), 256), dtype=torch.uint8, device=dev)
         out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
-        call = lambda: tbik.gemm(a, b, T=T, leaf=LEAF, tc=True, out_bf16=True, out=out, workspace=ws)  # noqa: E731
-    for _ in range(args.steps):
+        call = lambda: tbik.gemm(a, b, T=T, leaf=LEAF, tc=tc, out_bf16=True, out=out, workspace=ws)  # noqa: E731
+    call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps - 1):
         call()
+    e1.record()
     torch.cuda.synchronize()
     status = tbik.get_error()
-    print(f"profile case {args.profile_case}: {args.steps} calls, status {status}", flush=True)
+    ms = e0.elapsed_time(e1) / max(args.steps - 1, 1)
+    print(f"profile case {args.profile_case}: {args.steps} calls, {ms:.3f} ms per call after the first, "
+          f"status {status}", flush=True)
     return 0 if status == tbik.TBIK_OK else 1
 
 
