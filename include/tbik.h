@@ -302,10 +302,13 @@ TBIK_API tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W_lm, 
  *    tbik_logprob_workspace() for the same arguments is larger).  For the
  *    151936 x 4096 lm_head with leaf 256 on a 148-SM B200 this allows up to
  *    1251 rows per call.
- *  - Returns TBIK_ERR_ARG for any mode without TBIK_TC or with TBIK_EXACT.
+ *  - Returns TBIK_ERR_ARG for any mode without TBIK_TC or with TBIK_EXACT;
+ *    otherwise the status tbik_logprob would return for the same arguments
+ *    (TBIK_ERR_ARG, _SHAPE, _CUDA, _UNSUPPORTED) before the size check.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept for the life of the
+ *    process: do not use this entry point across a cudaDeviceReset.
  *  - All calls share the one array, which keeps the last call's contents.
  *    Nothing in it needs clearing (every value read is written earlier in the
  *    same call), but calls that overlap on the GPU (two streams, or two host
@@ -330,11 +333,9 @@ TBIK_API tbik_status tbik_get_error(void* stream);
  * epilogue withhold its "accumulator drained" arrive, so the MMA issuer's
  * bounded wait expires: the kernel must record TBIK_ERR_TIMEOUT, drain its own
  * copies in flight, free its TMEM and return.  wait_limit_ns bounds every
- * device-side wait (0 keeps the default of 2 s).  TBIK_DEBUG_SWAP_MN_STRIDES
- * swaps the two stride fields of the [K,N] B operand descriptor (layout check).
+ * device-side wait (0 keeps the default of 2 s).
  */
 #define TBIK_DEBUG_WITHHOLD_ACC_ARRIVE 0x1u
-#define TBIK_DEBUG_SWAP_MN_STRIDES 0x2u
 TBIK_API tbik_status tbik_debug_set(unsigned flags, unsigned long long wait_limit_ns);
 
 #ifdef __cplusplus

@@ -37,7 +37,6 @@ OUT_F32 = 0x000
 OUT_BF16 = 0x100
 SWIGLU_OUT = 0x200
 DEBUG_WITHHOLD_ACC_ARRIVE = 0x1
-DEBUG_SWAP_MN_STRIDES = 0x2
 VOCAB_LEAF = 64
 T_MAX = 8
 

@@ -175,41 +175,48 @@ struct TreeOf<1> {
 // out[g] = TREE over P[g*G .. g*G+G) for g < groups; each buffer has MN floats.
 // out is fp32 [groups][MN] or, with out_bf16, bf16 [MN] (groups == 1); with
 // out_bf16, a non-null R (bf16 [MN], may be `out` itself) is added to the root
-// in fp32 before the rounding.
-template <int G>
+// in fp32 before the rounding.  VEC = 1 reads and writes 16-byte vectors and
+// needs MN % 4 == 0 (every buffer start P + j*MN and out + g*MN is then
+// 16-byte aligned, given 16-byte aligned P and out); VEC = 0 is the element
+// loop for any MN.  Same additions in the same order either way.
+template <int G, int VEC>
 __global__ void tree_combine_kernel(const float* __restrict__ P, size_t MN, int groups, void* out, int out_bf16,
                                     const uint16_t* R) {
-    const size_t nvec = MN / 4;
-    const size_t total = nvec * groups;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const size_t g = i / nvec, e = (i - g * nvec) * 4;
-        float4 r = TreeOf<G>::vec(P + g * G * MN, MN, e);
-        if (out_bf16 && R) {
-            const uint2 q = *reinterpret_cast<const uint2*>(R + e);
-            r.x = __fadd_rn(r.x, __uint_as_float(q.x << 16));
-            r.y = __fadd_rn(r.y, __uint_as_float(q.x & 0xffff0000u));
-            r.z = __fadd_rn(r.z, __uint_as_float(q.y << 16));
-            r.w = __fadd_rn(r.w, __uint_as_float(q.y & 0xffff0000u));
+    if (VEC) {
+        const size_t nvec = MN / 4;
+        const size_t total = nvec * groups;
+        for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+             i += (size_t)gridDim.x * blockDim.x) {
+            const size_t g = i / nvec, e = (i - g * nvec) * 4;
+            float4 r = TreeOf<G>::vec(P + g * G * MN, MN, e);
+            if (out_bf16 && R) {
+                const uint2 q = *reinterpret_cast<const uint2*>(R + e);
+                r.x = __fadd_rn(r.x, __uint_as_float(q.x << 16));
+                r.y = __fadd_rn(r.y, __uint_as_float(q.x & 0xffff0000u));
+                r.z = __fadd_rn(r.z, __uint_as_float(q.y << 16));
+                r.w = __fadd_rn(r.w, __uint_as_float(q.y & 0xffff0000u));
+            }
+            if (out_bf16) {
+                uint2 w;
+                w.x = pack_bf2(r.x, r.y);
+                w.y = pack_bf2(r.z, r.w);
+                *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + e) = w;
+            } else {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + g * MN + e) = r;
+            }
         }
-        if (out_bf16) {
-            uint2 w;
-            w.x = pack_bf2(r.x, r.y);
-            w.y = pack_bf2(r.z, r.w);
-            *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + e) = w;
-        } else {
-            *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + g * MN + e) = r;
+    } else {
+        const size_t total = MN * groups;
+        for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+             i += (size_t)gridDim.x * blockDim.x) {
+            const size_t g = i / MN, e = i - g * MN;
+            float r = TreeOf<G>::one(P + g * G * MN, MN, e);
+            if (out_bf16 && R) r = __fadd_rn(r, bf2f(R[e]));
+            if (out_bf16)
+                reinterpret_cast<uint16_t*>(out)[e] = f2bf(r);
+            else
+                reinterpret_cast<float*>(out)[g * MN + e] = r;
         }
-    }
-    // ragged tail (MN % 4)
-    const size_t tail = MN - nvec * 4;
-    if (blockIdx.x == 0 && threadIdx.x < tail * groups) {
-        const size_t g = threadIdx.x / tail, e = nvec * 4 + threadIdx.x % tail;
-        float r = TreeOf<G>::one(P + g * G * MN, MN, e);
-        if (out_bf16 && R) r = __fadd_rn(r, bf2f(R[e]));
-        if (out_bf16)
-            reinterpret_cast<uint16_t*>(out)[e] = f2bf(r);
-        else
-            reinterpret_cast<float*>(out)[g * MN + e] = r;
     }
 }
 

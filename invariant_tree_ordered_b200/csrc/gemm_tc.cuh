@@ -90,7 +90,6 @@ struct TcParams {
     float* scratch;   // [gridDim.x][gs][128*128], layout per slot [col/4][row][4]
     int gs;           // global stack slots per CTA (pending subtrees of >= 5 leaves)
     int b_mn;         // 1: B is [K,N] (MN-major operand)
-    uint32_t b_lbo, b_sbo;
     // logprob epilogue
     const int32_t* targets;
     float* stats;  // [vocab leaves][M][2]  (max, sum-exp) per row and 64-column vocab leaf
@@ -308,7 +307,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         if (rank == 0) {
             const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, TC_BN, 0, p.b_mn);
             const bool b_mn = p.b_mn != 0;
-            const uint32_t b_lbo = p.b_lbo, b_sbo = p.b_sbo;
+            // MN-major B (a [K,N] operand): each CTA's 64 columns are one
+            // 128-byte swizzle atom wide, so the leading (MN) offset spans the
+            // whole half tile and the stride between 8-deep K groups is 1024 B.
+            constexpr uint32_t b_lbo = (uint32_t)TC_B_BYTES, b_sbo = 1024u;
             const uint32_t ring_u = smem_u32(ring);
             const uint32_t stage_bytes = p.stage_bytes, a_slice = p.a_slice;
             const int stages = p.stages;

@@ -17,6 +17,10 @@
 
 #include "tbik.h"
 
+// Defined in tbik_api.cu (library-internal): tbik_logprob's planning status for
+// these arguments and, when TBIK_OK, its workspace bytes.
+tbik_status tbik_logprob_plan_status(int M, int V, int H, int T, int leaf, unsigned mode, size_t* bytes);
+
 namespace {
 
 // The shared scratch area.  In host code this name is only a host-side stand-in
@@ -28,7 +32,10 @@ void* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
 // Set-up, once per device, with that device current: look up the device
-// address of the scratch array.
+// address of the scratch array.  The address is kept for the life of the
+// process; a cudaDeviceReset (which unloads the module and may place the array
+// elsewhere when it is loaded again) makes it stale, so this entry point is not
+// for use across a device reset.
 tbik_status scratch_address(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TBIK_ERR_CUDA;
@@ -48,11 +55,12 @@ extern "C" TBIK_API tbik_status tbik_logprob_noalloc(const uint16_t* hidden, con
                                                      const int32_t* targets, float* out, int M, int V, int H, int T,
                                                      int leaf, unsigned mode, void* stream) {
     if (!(mode & TBIK_TC) || (mode & TBIK_EXACT)) return TBIK_ERR_ARG;
-    const size_t need = tbik_logprob_workspace(M, V, H, T, leaf, mode);
-    if (need == (size_t)-1) return TBIK_ERR_SHAPE;
+    size_t need = 0;
+    tbik_status st = tbik_logprob_plan_status(M, V, H, T, leaf, mode, &need);
+    if (st != TBIK_OK) return st;  // the code tbik_logprob would return
     if (need > (size_t)TBIK_NOALLOC_SCRATCH_BYTES) return TBIK_ERR_WORKSPACE;
     void* ws = nullptr;
-    const tbik_status st = scratch_address(&ws);
+    st = scratch_address(&ws);
     if (st != TBIK_OK) return st;
     // Every region of the scratch that the kernels read is written earlier in
     // the same call, so nothing has to be cleared between calls.

@@ -286,14 +286,20 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
 
 tbik_status launch_status() { return cudaGetLastError() == cudaSuccess ? TBIK_OK : TBIK_ERR_CUDA; }
 
+// 16-byte vectors when M*N % 4 == 0 (every partial buffer then starts on a
+// 16-byte boundary), else the element loop.
 template <int G>
 void launch_tree_combine(const float* P, size_t MN, int groups, void* out, int bf16, const uint16_t* R,
                          cudaStream_t s, int sms) {
-    size_t work = (MN / 4) * groups;
-    int blocks = (int)((work + 255) / 256);
-    if (blocks > sms * 8) blocks = sms * 8;
+    const bool vec = (MN % 4) == 0;
+    const size_t work = (vec ? MN / 4 : MN) * groups;
+    size_t blocks = (work + 255) / 256;
+    if (blocks > (size_t)sms * 8) blocks = (size_t)sms * 8;
     if (blocks < 1) blocks = 1;
-    tree_combine_kernel<G><<<blocks, 256, 0, s>>>(P, MN, groups, out, bf16, R);
+    if (vec)
+        tree_combine_kernel<G, 1><<<(int)blocks, 256, 0, s>>>(P, MN, groups, out, bf16, R);
+    else
+        tree_combine_kernel<G, 0><<<(int)blocks, 256, 0, s>>>(P, MN, groups, out, bf16, R);
 }
 
 tbik_status tree_combine(const float* P, size_t MN, int G, int groups, void* out, int bf16, cudaStream_t s,
@@ -367,9 +373,6 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         prm.scratch = p.gs ? reinterpret_cast<float*>(ws + p.off_scratch) : nullptr;
         prm.gs = p.gs;
         prm.b_mn = p.b_nk ? 0 : 1;
-        const bool swap = g_debug_flags & TBIK_DEBUG_SWAP_MN_STRIDES;
-        prm.b_lbo = swap ? 1024u : (uint32_t)TC_B_BYTES;
-        prm.b_sbo = swap ? (uint32_t)TC_B_BYTES : 1024u;
         prm.debug = g_debug_flags;
         prm.wait_cycles = wait_cycles(info);
         prm.tab_n[0] = prm.tab_n[1] = p.nodes[0].second;
@@ -733,6 +736,27 @@ size_t tbik_logprob_workspace(int M, int V, int H, int T, int leaf, unsigned mod
     if (plan_logprob(M, V, H, T, leaf, mode, info->sms, p) != TBIK_OK) return (size_t)-1;
     return p.total;
 }
+
+}  // extern "C"
+
+// Library-internal (hidden visibility, not part of the ABI): the status that
+// tbik_logprob's planning gives these arguments on the current device and, when
+// it is TBIK_OK, the workspace bytes.  Lets another entry point report the same
+// status codes as tbik_logprob (ARG, SHAPE, CUDA, UNSUPPORTED) instead of the
+// bare (size_t)-1 of tbik_logprob_workspace.
+tbik_status tbik_logprob_plan_status(int M, int V, int H, int T, int leaf, unsigned mode, size_t* bytes) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    LogprobPlan p;
+    st = plan_logprob(M, V, H, T, leaf, mode, info->sms, p);
+    if (st != TBIK_OK) return st;
+    *bytes = p.total;
+    return TBIK_OK;
+}
+
+extern "C" {
 
 tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* targets, float* out, int M, int V,
                          int H, int T, int leaf, unsigned mode, void* ws, size_t ws_bytes, void* stream) {

@@ -82,6 +82,27 @@ def test_ragged_exact_bitwise_and_tc_tolerance(M, N, K, leaf, b_nk):
     assert rel_frob(tc_outs[0], c64) <= 2e-5
 
 
+@pytest.mark.parametrize("M,N", [(3, 5), (1, 7), (5, 9)])
+def test_exact_frontier_split_with_odd_output_count(M, N):
+    """M*N % 4 != 0 with the tree cut into frontier partials (few output tiles)
+    and, for T > 1, per-shard buffers: the shard combine takes its element
+    path (the buffers do not start on 16-byte boundaries).  Bit-exact for every
+    T, fp32 and bf16 outputs, with and without the fused residual."""
+    K, leaf = 256, 32
+    a = synth.normal_bf16(125 + M, (M, K))
+    b = synth.normal_bf16(126 + N, (K, N), std=0.1)
+    r = synth.normal_bf16(127 + N, (M, N))
+    ref = oracle.gemm_tree(a, b, b_nk=False, T=1, leaf=leaf)
+    ref_bf = np.array([oracle.bf16_rne(float(v)) for v in ref.ravel()], dtype=np.uint16).reshape(ref.shape)
+    ref_res = oracle.add_residual_bf16(ref, r)
+    for T in TS:
+        assert np.array_equal(u32(run(a, b, T=T, leaf=leaf, tc=False)), u32(ref)), T
+        assert np.array_equal(run(a, b, T=T, leaf=leaf, tc=False, out_bf16=True), ref_bf), T
+        got = tbik.gemm(dev_bf16(a), dev_bf16(b), T=T, leaf=leaf, tc=False, residual=dev_bf16(r))
+        assert tbik.get_error() == tbik.TBIK_OK
+        assert np.array_equal(host_bits16(got), ref_res), T
+
+
 def test_exact_leaf_one_and_odd_leaf_counts():
     """Exact mode follows the tree for leaf = 1 and non-power-of-two leaf counts."""
     a = synth.normal_bf16(120, (5, 96))

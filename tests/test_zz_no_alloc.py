@@ -54,6 +54,27 @@ def test_noalloc_logprob_matches_allocating_entry_point_on_two_calls():
         assert np.array_equal(u32(got), u32(ref))
 
 
+def test_noalloc_noninv_baseline_matches_allocating_entry_point():
+    """The non-invariant baseline (TBIK_TC | TBIK_NONINV: a different chain
+    plan and scratch size) through the fixed array, bitwise equal to
+    tbik_logprob(noninv=True), on two calls in a row."""
+    lib, noalloc = _entry()
+    stream = torch.cuda.current_stream().cuda_stream
+    V, H, leaf = 12000, 2048, 256
+    w = dev_bf16(synth.normal_bf16(510, (V, H), std=0.05))
+    for M, T, seed in ((260, 4, 511), (77, 8, 513)):
+        h = dev_bf16(synth.normal_bf16(seed, (M, H)))
+        t = dev_i32(synth.uniform_int32(seed + 1, M, 0, V))
+        ref = host_f32(tbik.logprob(h, w, t, T=T, leaf=leaf, tc=True, noninv=True))
+        assert tbik.get_error() == tbik.TBIK_OK
+        out = torch.full((M,), float("nan"), dtype=torch.float32, device="cuda")
+        status = noalloc(h.data_ptr(), w.data_ptr(), t.data_ptr(), out.data_ptr(), M, V, H, T, leaf,
+                         tbik.TC | tbik.NONINV, stream)
+        assert status == tbik.TBIK_OK
+        assert tbik.get_error() == tbik.TBIK_OK
+        assert np.array_equal(u32(host_f32(out)), u32(ref))
+
+
 def _largest_fitting_rows(lib, V, H, T, leaf):
     lo, hi = 1, 1 << 20
     while lo < hi:  # largest M whose scratch fits the fixed array
@@ -82,6 +103,11 @@ def test_noalloc_refuses_arguments_beyond_its_scratch():
     assert status == tbik.TBIK_ERR_WORKSPACE
     assert noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 4, V, H, T, leaf, tbik.EXACT,
                    stream) == tbik.TBIK_ERR_ARG
+    # the statuses tbik_logprob gives: an unknown mode bit, a bad shard count
+    assert noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 4, V, H, T, leaf,
+                   tbik.TC | 0x80, stream) == tbik.TBIK_ERR_ARG
+    assert noalloc(dummy.data_ptr(), dummy.data_ptr(), tg.data_ptr(), out.data_ptr(), 4, V, H, 3, leaf, tbik.TC,
+                   stream) == tbik.TBIK_ERR_SHAPE
     torch.cuda.synchronize()
     assert torch.isnan(out).all()
     assert tbik.get_error() == tbik.TBIK_OK
