@@ -8,6 +8,7 @@ library.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -57,40 +58,80 @@ def build(force: bool = False) -> str:
     return so
 
 
+def _open(path: str) -> ctypes.CDLL:
+    """Load an oracle build at ``path`` and declare its function signatures."""
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, f32, f64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_double)
+    sig = {
+        "oracle_bf16_rne": (ctypes.c_uint16, [f32]),
+        "oracle_bf16_rne_array": (None, [vp, vp, i64]),
+        "oracle_tree_sum": (f32, [vp, i32]),
+        "oracle_exp": (f32, [f32]),
+        "oracle_log": (f32, [f32]),
+        "oracle_tree_ms": (None, [vp, vp, i32, vp, vp]),
+        "oracle_gemm_tree": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
+        "oracle_gemm_noninv": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp]),
+        "oracle_gemm_f64": (None, [vp, vp, i32, i32, i32, i32, vp]),
+        "oracle_rmsnorm_residual": (i32, [vp, vp, vp, vp, vp, i32, i32, f32, i32]),
+        "oracle_add_residual_bf16": (None, [vp, vp, vp, i64]),
+        "oracle_rope_table": (None, [vp, i32, i32, f64]),
+        "oracle_rope": (None, [vp, vp, vp, vp, i32, i32, i32]),
+        "oracle_swiglu_bf16": (None, [vp, vp, vp, i64]),
+        "oracle_swiglu_f32": (None, [vp, vp, vp, i64]),
+        "oracle_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]),
+        "oracle_logprob_f64": (None, [vp, vp, vp, vp, i32, i32, i32]),
+        "oracle_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32]),
+        "oracle_attention_f64": (None, [vp, vp, vp, vp, i32, i32, i32, i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
-            vp, i32, i64, f32, f64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
-                                      ctypes.c_float, ctypes.c_double)
-            sig = {
-                "oracle_bf16_rne": (ctypes.c_uint16, [f32]),
-                "oracle_bf16_rne_array": (None, [vp, vp, i64]),
-                "oracle_tree_sum": (f32, [vp, i32]),
-                "oracle_exp": (f32, [f32]),
-                "oracle_log": (f32, [f32]),
-                "oracle_tree_ms": (None, [vp, vp, i32, vp, vp]),
-                "oracle_gemm_tree": (i32, [vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]),
-                "oracle_gemm_noninv": (i32, [vp, vp, i32, i32, i32, i32, i32, vp, vp]),
-                "oracle_gemm_f64": (None, [vp, vp, i32, i32, i32, i32, vp]),
-                "oracle_rmsnorm_residual": (i32, [vp, vp, vp, vp, vp, i32, i32, f32, i32]),
-                "oracle_add_residual_bf16": (None, [vp, vp, vp, i64]),
-                "oracle_rope_table": (None, [vp, i32, i32, f64]),
-                "oracle_rope": (None, [vp, vp, vp, vp, i32, i32, i32]),
-                "oracle_swiglu_bf16": (None, [vp, vp, vp, i64]),
-                "oracle_swiglu_f32": (None, [vp, vp, vp, i64]),
-                "oracle_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp]),
-                "oracle_logprob_f64": (None, [vp, vp, vp, vp, i32, i32, i32]),
-                "oracle_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32]),
-                "oracle_attention_f64": (None, [vp, vp, vp, vp, i32, i32, i32, i32]),
-            }
-            for name, (res, args) in sig.items():
-                fn = getattr(lib, name)
-                fn.restype = res
-                fn.argtypes = args
-            _lib = lib
+            _lib = _open(build())
     return _lib
+
+
+@contextlib.contextmanager
+def library(path: str):
+    """Run the wrappers against another build of oracle.c (a shared object at
+    ``path``) for the duration of the block.  Test use only: the oracle's
+    mutation tests compile copies of oracle.c with one mistake planted and
+    check that the pins catch it."""
+    global _lib
+    other = _open(path)
+    with _lock:
+        saved = _lib
+        _lib = other
+    try:
+        yield other
+    finally:
+        with _lock:
+            _lib = saved
+
+
+def compile_variant(src_text: str, out_path: str) -> str:
+    """Compile C source text (a variant of oracle.c) with the oracle's flags."""
+    src = out_path + ".c"
+    with open(src, "w") as f:
+        f.write(src_text)
+    flags = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+    if _cpu_has_fma():
+        flags.append("-mfma")
+    subprocess.check_call(["gcc", *flags, "-o", out_path, src, "-lm"])
+    return out_path
+
+
+def source() -> str:
+    """The text of oracle.c."""
+    with open(_SRC) as f:
+        return f.read()
 
 
 def _c(a, dtype):

@@ -555,3 +555,45 @@ def test_decoder_zero_layers_leave_the_residual_stream_unchanged():
     w["lm_head"] = np.zeros_like(w["lm_head"])
     got = odec.forward(cfg, w, ids, tg, T=1)
     assert np.allclose(got, -math.log(cfg["vocab"]), rtol=0, atol=1e-6)
+
+
+# ------------------------------------------------------ ordering probes
+# Hand-derived outputs (tests/golden/ordering_probes.json) on inputs where the
+# reduction order, the leaf size or the place of eps changes the result far
+# beyond rounding; tests/test_oracle_mutants.py shows each planted mistake fails.
+
+def test_baseline_combine_is_left_to_right():
+    from tests import ordering_probes
+    ordering_probes.check_baseline_shard_sum()
+
+
+def test_logprob_baseline_logits_are_summed_left_to_right():
+    from tests import ordering_probes
+    ordering_probes.check_logprob_baseline_logit_sum()
+
+
+def test_rmsnorm_leaf_size_mean_and_eps_placement():
+    from tests import ordering_probes
+    ordering_probes.check_rmsnorm_cancellation()
+
+
+def test_vocab_leaf_sum_is_ascending():
+    from tests import ordering_probes
+    ordering_probes.check_vocab_leaf_ascending_sum()
+
+
+def test_rmsnorm_eps_inside_square_root_closed_form():
+    """A row of magnitude ~1e-3 with eps = 1e-6: 1/sqrt(ms + eps) and
+    1/(sqrt(ms) + eps) differ by ~30 %; the oracle follows the first within
+    one bf16 ulp of the binary64 closed form."""
+    H = 4096
+    c = 2.0 ** -10
+    x = np.full((1, H), c, dtype=np.float32)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    gamma = np.full(H, 0x3F80, dtype=np.uint16)
+    y, _ = oracle.rmsnorm_residual(xb, None, gamma, eps=1e-6)
+    want = c / math.sqrt(c * c + float(np.float32(1e-6)))
+    wrong = c / (c + float(np.float32(1e-6)))
+    got = float(F(y[0, :1])[0])
+    assert abs(got - want) <= want * 2 ** -8
+    assert abs(got - wrong) > 0.25 * wrong
