@@ -49,6 +49,8 @@ KERNELS_PER_STEP = 6  # rmsnorm, rope, swiglu, gemm, logprob gemm+stats, logprob
 # fp32 FMA peak of the exact-order (CUDA-core) mode: 148 SMs x 128 fp32 lanes x
 # 2 flop x 1.965 GHz (the maximum SM clock)
 FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# Timed regions at least this long are compared with the sustained bf16 peak.
+SUSTAINED_REGION_S = 3.0
 
 
 def parse():
@@ -180,6 +182,24 @@ def whole_job_tokens_per_s(ms_total_max: float, steps: int, world: int, tokens_p
 
 # ------------------------------------------------------------- CPU oracle
 
+def host_cpu() -> dict:
+    """The host the oracle ran on: logical CPUs available and the CPU model."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = os.cpu_count()
+    return {"host_cores": os.cpu_count(), "host_cores_available": avail, "cpu_model": model}
+
+
 _ORACLE_INPUTS = {}
 
 
@@ -225,7 +245,8 @@ def run_reference(args):
                    "T": 1, "leaf": LEAF},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                          "sample": f"{tokens} token(s) of the step per step: RMSNorm, RoPE q/k, SwiGLU, one "
-                                   f"down_proj row, one lm_head logprob row (single-threaded C oracle)"},
+                                   f"down_proj row, one lm_head logprob row (single-threaded C oracle)",
+                         **host_cpu()},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -431,6 +452,12 @@ def run_tbik(args):
 
     lp_ms = lp_live_ms
     achieved = LOGPROB_FLOP / (lp_ms * 1e-3) / 1e12
+    # The peak that matches the timing conditions: a short timed region runs at
+    # the burst clock (the burst cuBLAS figure), a region of several seconds
+    # settles under the power cap (the sustained figure).
+    region_s = ms_total * 1e-3
+    peak_kind = "burst" if region_s < SUSTAINED_REGION_S else "sustained"
+    peak = pk["bf16"] if peak_kind == "burst" else pk["bf16_sus"]
     ms_step = ms_total / args.steps
     value = whole_job_tokens_per_s(ms_total, args.steps, world)
     gb = lambda nbytes, ms: nbytes / (ms * 1e-3) / 1e9  # noqa: E731
@@ -461,9 +488,12 @@ def run_tbik(args):
             "decoder_e2e": dec,
         },
         "roofline": {"kernel": "tbik_logprob (fused tcgen05 GEMM + vocab stats, then row tree)",
-                     "bound": "tensor", "achieved": achieved, "peak": pk["bf16_sus"], "unit": "TFLOP/s",
-                     "frac": achieved / pk["bf16_sus"], "traffic": profiled_traffic(),
-                     "peak_source": f"{pk['src']} bf16 sustained"},
+                     "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "peak_source": f"{pk['src']} bf16 {peak_kind} (timed region {region_s:.2f} s; burst "
+                                    f"below {SUSTAINED_REGION_S:.0f} s)",
+                     "frac_of_burst": achieved / pk["bf16"], "frac_of_sustained": achieved / pk["bf16_sus"],
+                     "achieved_formula": "2*M*V*H / mean in-step CUDA-event time of the logprob call"},
         "e2e": {"value": whole_job_tokens_per_s(e2e_ms, args.steps, world), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
@@ -474,7 +504,8 @@ def run_tbik(args):
         dt = oracle_step_sample(tok)
         line["cpu_baseline"] = {"value": tok / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{tok} tokens of the step (RMSNorm, RoPE, SwiGLU, down_proj rows, "
-                                          f"lm_head logprob rows), single-threaded C oracle, {dt:.1f} s"}
+                                          f"lm_head logprob rows), single-threaded C oracle, {dt:.1f} s",
+                                **host_cpu()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
