@@ -285,6 +285,60 @@ TBIK_API tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W_lm, 
                          float* out, int M, int V, int H, int T, int leaf, unsigned mode, void* ws,
                          size_t ws_bytes, void* stream);
 
+/* ---- tensor parallelism across GPUs: the shard level of the tree ---------- */
+/*
+ * The TBIK summary page (技术框架) orders the reduction ACROSS GPUs by the same
+ * binary tree as the local one.  With T ranks, rank t computes the root of its
+ * own subtree (its shard), the T shard results are exchanged into every rank's
+ * own memory (for example an NCCL all-gather; never a sum all-reduce, whose
+ * order depends on the rank count), and every rank applies the top log2(T)
+ * levels of the tree with the calls below.  The result is bitwise the same as
+ * tbik_gemm / tbik_logprob on one GPU, for every T.
+ *
+ * Row-parallel GEMM (K split into T contiguous shards of whole leaves): rank t
+ * calls tbik_gemm on its [M, K/T] and [K/T, N] (or [N, K/T]) slices with T = 1
+ * and an fp32 output (the root of its subtree: TREE over its L/T leaves; with
+ * TBIK_NONINV, its one chain), gathers the T results as fp32 [T][M*N] in rank
+ * order, and calls:
+ *
+ *   out = TREE over t of partials[t] (T in {1,2,4,8}; with TBIK_NONINV the
+ *         left-to-right sum ((P0 + P1) + P2) + ... of the baseline instead);
+ *   mode  TBIK_OUT_BF16 for a bf16 output rounded once (else fp32), optionally
+ *         | TBIK_NONINV; R (bf16 [MN], nullable, needs TBIK_OUT_BF16) is added
+ *         to the fp32 root before the rounding, as in tbik_gemm_residual.
+ *   partials fp32 [T][MN] and out, R: device memory, 16-byte aligned; out may
+ *   be R (in place) but may not overlap partials.
+ */
+TBIK_API tbik_status tbik_tree_combine(const float* partials, void* out, long long MN, int T, unsigned mode,
+                                       const uint16_t* R, void* stream);
+
+/*
+ * Vocabulary-parallel logprob.  The padded vocabulary of tbik_logprob
+ * (Vpad = ceil(V / 512) * 512 columns, Lv = Vpad / 64 leaves) is split into T
+ * contiguous shards of Lv/T leaves: shard t covers vocabulary indices
+ * [v0, v0 + Vpad/T) with v0 = t * Vpad / T, of which Vs = clamp(V - v0, 0,
+ * Vpad/T) are real columns.  Rank t holds W_shard = rows [v0, v0 + Vs) of W_lm
+ * (bf16 [Vs, H]) and calls tbik_logprob_partial with Lvs = Lv / T:
+ *   part[i] = (m, s, z, own) as 4 floats: (m, s) = TREE over the shard's Lvs
+ *   vocabulary leaves (leaves past its Vs columns are identities); own = 1
+ *   and z = the target's logit when targets[i] is in [v0, v0 + Vs), else
+ *   own = 0 and z = 0.  Everything else as tbik_logprob in TBIK_TC or
+ *   TBIK_EXACT mode (TBIK_NONINV is refused with TBIK_ERR_ARG).  Vs may be 0
+ *   (a shard of padding only; W_shard is then not read).
+ * Then gather the T part arrays as fp32 [T][M][4] in rank order and call
+ * tbik_logprob_combine: per row TREE over the T (m, s), z from the owning
+ * shard, out = (z - m) - log(s); a target outside [0, V) (or owned by no
+ * shard) gives NaN and records TBIK_ERR_TARGET.
+ * part, parts: 16-byte aligned device memory; ws as for tbik_logprob, sized by
+ * tbik_logprob_partial_workspace.
+ */
+TBIK_API size_t tbik_logprob_partial_workspace(int M, int Vs, int Lvs, int H, int leaf, unsigned mode);
+TBIK_API tbik_status tbik_logprob_partial(const uint16_t* hidden, const uint16_t* W_shard, const int32_t* targets,
+                                          float* part, int M, int Vs, int v0, int Lvs, int H, int leaf,
+                                          unsigned mode, void* ws, size_t ws_bytes, void* stream);
+TBIK_API tbik_status tbik_logprob_combine(const float* parts, const int32_t* targets, float* out, int M, int V,
+                                          int T, void* stream);
+
 /*
  * tbik_logprob_noalloc -- the pages have no counterpart for this entry point.
  *

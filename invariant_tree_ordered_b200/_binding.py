@@ -85,6 +85,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "tbik_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
             "tbik_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp]),
             "tbik_transpose": (i32, [vp, vp, i32, i32, vp]),
+            "tbik_tree_combine": (i32, [vp, vp, ctypes.c_longlong, i32, u32, vp, vp]),
+            "tbik_logprob_partial_workspace": (sz, [i32, i32, i32, i32, i32, u32]),
+            "tbik_logprob_partial": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
+            "tbik_logprob_combine": (i32, [vp, vp, vp, i32, i32, i32, vp]),
             "tbik_get_error": (i32, [vp]),
             "tbik_debug_set": (i32, [u32, ull]),
         }
@@ -370,6 +374,91 @@ def logprob(hidden, W, targets, *, T: int = 1, leaf: int = 256, tc: bool = True,
     ws, wsb = _workspace(lib.tbik_logprob_workspace(M, V, H, T, leaf, mode), hidden.device, workspace)
     _check(lib.tbik_logprob(_ptr(hidden), _ptr(W), _ptr(targets), _ptr(out), M, V, H, T, leaf, mode, _ptr(ws), wsb,
                             _stream_handle(stream)), "tbik_logprob")
+    return out
+
+
+# ------------------------------------------- shard level across GPUs (TP)
+
+def vocab_shard(V: int, T: int, t: int):
+    """Shard t of T of the padded vocabulary (tbik.h, vocabulary-parallel
+    logprob): (v0, Vs, Lvs) = first vocabulary index, real columns, leaves."""
+    step = VOCAB_LEAF * T_MAX
+    vpad = ((V + step - 1) // step) * step
+    if T not in (1, 2, 4, 8) or not 0 <= t < T:
+        raise ValueError("T must be 1, 2, 4 or 8 and 0 <= t < T")
+    width = vpad // T
+    v0 = t * width
+    vs = max(0, min(V - v0, width))
+    return v0, vs, width // VOCAB_LEAF
+
+
+def tree_combine(partials, *, noninv: bool = False, out_bf16: bool = False, residual=None, out=None, stream=None):
+    """tbik_tree_combine: the shard level of the tree over fp32 partials [T, ...]
+    gathered in rank order (left to right with noninv).  Returns fp32 or bf16
+    of shape partials.shape[1:]; residual (bf16, that shape) is added to the
+    fp32 root before the bf16 rounding."""
+    torch = _torch()
+    lib = load_library()
+    _need(partials, torch.float32, "partials")
+    T = partials.shape[0]
+    shape = tuple(partials.shape[1:])
+    mn = partials[0].numel()
+    if residual is not None:
+        out_bf16 = True
+        _need_out(residual, torch.bfloat16, shape, "residual")
+    dtype = torch.bfloat16 if out_bf16 else torch.float32
+    if out is None:
+        out = torch.empty(shape, dtype=dtype, device=partials.device)
+    _need_out(out, dtype, shape)
+    mode = (NONINV if noninv else 0) | (OUT_BF16 if out_bf16 else 0)
+    _check(lib.tbik_tree_combine(_ptr(partials), _ptr(out), mn, T, mode, _ptr(residual), _stream_handle(stream)),
+           "tbik_tree_combine")
+    return out
+
+
+def logprob_partial(hidden, W_shard, targets, *, v0: int, Lvs: int, leaf: int = 256, tc: bool = True, out=None,
+                    workspace=None, stream=None):
+    """tbik_logprob_partial: one vocabulary shard's per-row (m, s, z, own),
+    fp32 [M, 4].  W_shard holds vocabulary rows [v0, v0 + Vs) (Vs may be 0)."""
+    torch = _torch()
+    lib = load_library()
+    _need(hidden, torch.bfloat16, "hidden")
+    _need(W_shard, torch.bfloat16, "W_shard")
+    _need(targets, torch.int32, "targets")
+    M, H = hidden.shape
+    Vs = W_shard.shape[0]
+    if W_shard.dim() != 2 or (Vs > 0 and W_shard.shape[1] != H):
+        raise ValueError("W_shard must be [Vs, H]")
+    if targets.numel() != M:
+        raise ValueError("targets must hold one index per row of hidden")
+    mode = TC if tc else EXACT
+    if out is None:
+        out = torch.empty((M, 4), dtype=torch.float32, device=hidden.device)
+    _need_out(out, torch.float32, (M, 4))
+    ws, wsb = _workspace(lib.tbik_logprob_partial_workspace(M, Vs, Lvs, H, leaf, mode), hidden.device, workspace)
+    wptr = _ptr(W_shard) if Vs > 0 else None
+    _check(lib.tbik_logprob_partial(_ptr(hidden), wptr, _ptr(targets), _ptr(out), M, Vs, v0, Lvs, H, leaf, mode,
+                                    _ptr(ws), wsb, _stream_handle(stream)), "tbik_logprob_partial")
+    return out
+
+
+def logprob_combine(parts, targets, V: int, *, out=None, stream=None):
+    """tbik_logprob_combine: parts fp32 [T, M, 4] (shard summaries in rank
+    order) -> logprob fp32 [M]."""
+    torch = _torch()
+    lib = load_library()
+    _need(parts, torch.float32, "parts")
+    _need(targets, torch.int32, "targets")
+    if parts.dim() != 3 or parts.shape[2] != 4:
+        raise ValueError("parts must be [T, M, 4]")
+    T, M = parts.shape[0], parts.shape[1]
+    if targets.numel() != M:
+        raise ValueError("targets must hold one index per row")
+    if out is None:
+        out = torch.empty(M, dtype=torch.float32, device=parts.device)
+    _need_out(out, torch.float32, (M,))
+    _check(lib.tbik_logprob_combine(_ptr(parts), _ptr(targets), _ptr(out), M, V, T, _stream_handle(stream)),
+           "tbik_logprob_combine")
     return out
 
 

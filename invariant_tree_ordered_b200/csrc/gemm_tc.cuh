@@ -94,6 +94,8 @@ struct TcParams {
     const int32_t* targets;
     float* stats;  // [vocab leaves][M][2]  (max, sum-exp) per row and 64-column vocab leaf
     float* zt;     // [M]  logit of the target
+    int* zflag;    // [M] or null: set to 1 where zt is written (vocabulary shard summaries)
+    int v0;        // vocabulary index of column 0 of B (a shard's first column; 0 otherwise)
     int V;
     unsigned debug;
     unsigned long long wait_cycles;  // bound of every device-side wait, in SM cycles
@@ -539,16 +541,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                     const int c0 = tn * TC_BN + half * 64;
                     const int vleaf = 2 * tn + half;
                     if (c0 < p.V) {
-                        const int tgt = (row < p.M) ? p.targets[row] : -1;
+                        // target column relative to this call's first vocabulary column
+                        const long long tgt = (row < p.M) ? (long long)p.targets[row] - p.v0 : -1;
                         const int ncol = min(64, p.V - c0);
-                        const int kt = tgt - c0;  // target column within this leaf
-                        const bool have_t = (unsigned)kt < (unsigned)ncol;
+                        const long long kt = tgt - c0;  // target column within this leaf
+                        const bool have_t = kt >= 0 && kt < ncol;
+                        const int kti = have_t ? (int)kt : -1;
                         float zval = 0.0f;
                         if (have_t) {
 #pragma unroll
                             for (int k = 0; k < 32; ++k) {
-                                if (k == kt) zval = v[0][k];
-                                if (k + 32 == kt) zval = v[1][k];
+                                if (k == kti) zval = v[0][k];
+                                if (k + 32 == kti) zval = v[1][k];
                             }
                         }
                         if (ncol < 64) {  // the last vocab leaf: columns past V add nothing
@@ -576,7 +580,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                         const float s = __fadd_rn(s0, s1);
                         if (row < p.M) {
                             *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
-                            if (have_t) p.zt[row] = zval;
+                            if (have_t) {
+                                p.zt[row] = zval;
+                                if (p.zflag) p.zflag[row] = 1;
+                            }
                         }
                     }
                 }

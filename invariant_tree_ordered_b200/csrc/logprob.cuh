@@ -17,8 +17,12 @@ namespace tbik {
 
 constexpr int VLEAF = 64;  // vocabulary columns per leaf
 
+// v0: vocabulary index of z's column 0 (a shard's first column), so the
+// target's column here is targets[row] - v0; zflag (nullable) is set to 1 for
+// the rows whose target falls in this call's columns.
 __global__ void vocab_stats_kernel(const float* __restrict__ z, const int32_t* __restrict__ targets,
-                                   float* __restrict__ stats, float* __restrict__ zt, int M, int V, int nvt) {
+                                   float* __restrict__ stats, float* __restrict__ zt, int* __restrict__ zflag,
+                                   int M, int V, int nvt, int v0) {
     const size_t total = (size_t)M * nvt;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
         const int row = (int)(i / nvt);
@@ -32,8 +36,11 @@ __global__ void vocab_stats_kernel(const float* __restrict__ z, const int32_t* _
         float s = 0.0f;
         for (int c = c0; c < c1; ++c) s = __fadd_rn(s, exp_spec(__fsub_rn(zr[c], m)));
         *reinterpret_cast<float2*>(stats + ((size_t)j * M + row) * 2) = make_float2(m, s);
-        const int t = targets[row];
-        if (t >= c0 && t < c1) zt[row] = zr[t];
+        const long long t = (long long)targets[row] - v0;
+        if (t >= c0 && t < c1) {
+            zt[row] = zr[t];
+            if (zflag) zflag[row] = 1;
+        }
     }
 }
 
@@ -76,7 +83,7 @@ constexpr int ROW_BLOCK = 32;  // rows per CTA of the row kernel (one per lane),
 __global__ void __launch_bounds__(ROW_BLOCK * 32)
     logprob_row_kernel(const float* __restrict__ stats, const float* __restrict__ zt,
                        const int32_t* __restrict__ targets, float* __restrict__ out, float* shard_ms, int M, int V,
-                       int nvt, int Lv, int T) {
+                       int nvt, int Lv, int T, const int* __restrict__ zflag, float4* __restrict__ shard_sum) {
     constexpr int TAB = 512;
     __shared__ uint16_t tab[2][TAB];        // leaf operation codes for the two frontier subtree sizes
     __shared__ float2 part[32][ROW_BLOCK];  // [frontier node][row in block]
@@ -155,6 +162,13 @@ __global__ void __launch_bounds__(ROW_BLOCK * 32)
     }
     for (int w = 1; w < T; w <<= 1) sv = butterfly_ms(sv, lane, w);
     const MS fin = sv;
+    if (shard_sum != nullptr) {  // a vocabulary shard's summary (T == 1): (m, s, z_t, owns the target)
+        if (lane == 0) {
+            const bool own = zflag[row] != 0;
+            shard_sum[row] = make_float4(fin.m, fin.s, own ? zt[row] : 0.0f, own ? 1.0f : 0.0f);
+        }
+        return;
+    }
     if (lane == 0) {
         const int t = targets[row];
         if (t < 0 || t >= V) {
@@ -162,6 +176,40 @@ __global__ void __launch_bounds__(ROW_BLOCK * 32)
             out[row] = __int_as_float(0x7fc00000);
         } else {
             out[row] = __fsub_rn(__fsub_rn(zt[row], fin.m), log_spec(fin.s));
+        }
+    }
+}
+
+// The shard level of a vocabulary-parallel logprob: parts [T][M] hold each
+// shard's (m, s, z_t, owner) for every row (a shard's summary is the TREE over
+// its own contiguous vocabulary leaves).  Per row: TREE over the T summaries
+// (T a power of two: adjacent pairs level by level, the lower shard the left
+// operand, as in logprob_row_kernel's shard level), z_t from the shard that
+// owns the target, out = (z_t - m) - log(s).  A target outside [0, V), or one
+// that no shard owns, gives NaN and TBIK_ERR_TARGET.
+__global__ void logprob_combine_kernel(const float4* __restrict__ parts, const int32_t* __restrict__ targets,
+                                       float* __restrict__ out, int M, int V, int T) {
+    for (int row = blockIdx.x * blockDim.x + threadIdx.x; row < M; row += gridDim.x * blockDim.x) {
+        MS v[8];
+        float z = 0.0f;
+        int owners = 0;
+        for (int t = 0; t < T; ++t) {
+            const float4 q = parts[(size_t)t * M + row];
+            v[t].m = q.x;
+            v[t].s = q.y;
+            if (q.w != 0.0f) {
+                z = q.z;
+                ++owners;
+            }
+        }
+        for (int w = 1; w < T; w <<= 1)
+            for (int i = 0; i + w < T; i += 2 * w) v[i] = ms_combine(v[i], v[i + w]);
+        const int tg = targets[row];
+        if (tg < 0 || tg >= V || owners != 1) {
+            set_error(TBIK_ERR_TARGET);
+            out[row] = __int_as_float(0x7fc00000);
+        } else {
+            out[row] = __fsub_rn(__fsub_rn(z, v[0].m), log_spec(v[0].s));
         }
     }
 }

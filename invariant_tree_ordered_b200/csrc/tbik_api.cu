@@ -427,8 +427,10 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
 struct LogprobPlan {
     int M = 0, V = 0, H = 0, T = 1, leaf = 256;
     bool tc = false, noninv = false;
+    bool part = false;  // a vocabulary shard's summary (tbik_logprob_partial): T = 1, Lv given
     int Vpad = 0, Lv = 0, nvl = 0, nvt = 0, Lk = 0, tiles_m = 0, units = 0, grid = 0, gs = 0;
-    size_t off_stats = 0, off_zt = 0, off_shard = 0, off_scratch = 0, off_z = 0, off_zgemm = 0, total = 0;
+    size_t off_stats = 0, off_zt = 0, off_shard = 0, off_scratch = 0, off_z = 0, off_zgemm = 0, off_zflag = 0,
+           total = 0;
     GemmPlan zplan;  // exact mode: the logits GEMM
 };
 
@@ -438,18 +440,29 @@ tbik_status zgemm_plan(const LogprobPlan& p, int sms, GemmPlan& z) {
     return plan_gemm(M, p.V, p.H, 1, p.leaf, TBIK_EXACT | TBIK_B_NK, sms, z);
 }
 
-tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, int sms, LogprobPlan& p) {
+// part_lv > 0: the summary of one vocabulary shard of V columns reduced over
+// part_lv leaves (T = 1; leaves past the shard's columns are identities).
+tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, int sms, LogprobPlan& p,
+                         int part_lv = 0) {
     if (mode & ~(TBIK_EXACT | TBIK_TC | TBIK_NONINV)) return TBIK_ERR_ARG;
     const bool exact = mode & TBIK_EXACT, tc = mode & TBIK_TC;
     if (exact == tc) return TBIK_ERR_ARG;
-    if (M < 0 || V <= 0 || H <= 0 || leaf <= 0) return TBIK_ERR_ARG;
+    if (M < 0 || H <= 0 || leaf <= 0 || (part_lv > 0 ? V < 0 : V <= 0)) return TBIK_ERR_ARG;
     if (!valid_T(T) || H % leaf || H % 8 || leaf % 16) return TBIK_ERR_SHAPE;
     p.M = M, p.V = V, p.H = H, p.T = T, p.leaf = leaf;
     p.tc = tc;
     p.noninv = mode & TBIK_NONINV;
-    const int step = VLEAF * TBIK_T_MAX;
-    p.Vpad = (int)(((long long)V + step - 1) / step * step);
-    p.Lv = p.Vpad / VLEAF;
+    p.part = part_lv > 0;
+    if (p.part) {
+        if (T != 1) return TBIK_ERR_SHAPE;
+        if ((long long)part_lv * VLEAF < (long long)V || part_lv > (1 << 24)) return TBIK_ERR_SHAPE;
+        p.Lv = part_lv;
+        p.Vpad = part_lv * VLEAF;
+    } else {
+        const int step = VLEAF * TBIK_T_MAX;
+        p.Vpad = (int)(((long long)V + step - 1) / step * step);
+        p.Lv = p.Vpad / VLEAF;
+    }
     p.nvl = (V + VLEAF - 1) / VLEAF;        // vocab leaves holding columns
     p.nvt = (V + TC_BN - 1) / TC_BN;        // 128-column GEMM tiles (two vocab leaves each)
     // The baseline's logits: T chains over H/T each, summed left to right.
@@ -477,7 +490,11 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
         p.off_scratch = off;
         off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
     }
-    if (exact) {
+    if (p.part) {  // which rows' targets fall in this shard
+        p.off_zflag = off;
+        off = align256(off + (size_t)M * sizeof(int));
+    }
+    if (exact && V > 0) {
         // logits z fp32 [M][V] from the exact GEMM (the K tree, or the baseline's T chains summed in order)
         tbik_status st = zgemm_plan(p, sms, p.zplan);
         if (st != TBIK_OK) return st;
@@ -488,6 +505,70 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
     }
     p.total = off;
     return TBIK_OK;
+}
+
+// The logprob kernels for a plan: the fused GEMM + vocab statistics (or the
+// exact logits GEMM + statistics kernel), then the row tree.  With `part`
+// (a vocabulary shard, p.part) the row kernel writes the shard's per-row
+// summary instead of the logprob; v0 is the shard's first vocabulary index.
+tbik_status run_logprob(const LogprobPlan& p, const uint16_t* hidden, const uint16_t* W, const int32_t* targets,
+                        float* out, float4* part, int v0, uint8_t* w8, cudaStream_t s, const DeviceInfo* info) {
+    const int M = p.M, V = p.V, H = p.H, T = p.T, leaf = p.leaf;
+    tbik_status st;
+    float* stats = reinterpret_cast<float*>(w8 + p.off_stats);
+    float* zt = reinterpret_cast<float*>(w8 + p.off_zt);
+    float* shard = reinterpret_cast<float*>(w8 + p.off_shard);
+    int* zflag = p.part ? reinterpret_cast<int*>(w8 + p.off_zflag) : nullptr;
+    if (zflag && cudaMemsetAsync(zflag, 0, (size_t)M * sizeof(int), s) != cudaSuccess) return TBIK_ERR_CUDA;
+    if (V > 0 && p.tc) {
+        CUtensorMap ta, tb;
+        const int a_box = a_box_rows(M);
+        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
+        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, 64, TC_BN / 2)) return TBIK_ERR_CUDA;
+        TcParams prm;
+        memset(&prm, 0, sizeof(prm));
+        set_ring(prm, a_box);
+        prm.M = M, prm.N = V, prm.K = H;
+        prm.leaf = p.noninv ? H / T : leaf;
+        prm.seq = p.noninv ? 1 : 0;
+        prm.F = 1;
+        prm.tiles_m = p.tiles_m, prm.tiles_n = p.nvt;
+        prm.group_m = p.tiles_m;  // all row tiles of a vocab tile run together: W_lm is read once
+        prm.total_units = p.units;
+        prm.direct = 1;
+        prm.scratch = p.gs ? reinterpret_cast<float*>(w8 + p.off_scratch) : nullptr;
+        prm.gs = p.gs;
+        prm.b_mn = 0;
+        prm.targets = targets;
+        prm.stats = stats;
+        prm.zt = zt;
+        prm.zflag = zflag;
+        prm.v0 = v0;
+        prm.V = V;
+        prm.debug = g_debug_flags & ~TBIK_DEBUG_WITHHOLD_ACC_ARRIVE;
+        prm.wait_cycles = wait_cycles(info);
+        prm.lo[0] = 0;
+        prm.nl[0] = (short)p.Lk;
+        prm.tab_n[0] = prm.tab_n[1] = prm.nl[0];
+        gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+        if ((st = launch_status()) != TBIK_OK) return st;
+    } else if (V > 0) {
+        float* z = reinterpret_cast<float*>(w8 + p.off_z);
+        GemmPlan zp;
+        st = zgemm_plan(p, info->sms, zp);
+        if (st != TBIK_OK) return st;
+        if (zp.total > p.zplan.total) return TBIK_ERR_WORKSPACE;
+        st = run_gemm(zp, hidden, W, z, w8 + p.off_zgemm, s, info);
+        if (st != TBIK_OK) return st;
+        const size_t work = (size_t)M * p.nvl;
+        int blocks = (int)((work + 255) / 256);
+        if (blocks > info->sms * 16) blocks = info->sms * 16;
+        vocab_stats_kernel<<<blocks, 256, 0, s>>>(z, targets, stats, zt, zflag, M, V, p.nvl, v0);
+        if ((st = launch_status()) != TBIK_OK) return st;
+    }
+    logprob_row_kernel<<<(M + ROW_BLOCK - 1) / ROW_BLOCK, ROW_BLOCK * 32, 0, s>>>(stats, zt, targets, out, shard, M,
+                                                                                V, p.nvl, p.Lv, T, zflag, part);
+    return launch_status();
 }
 
 }  // namespace
@@ -772,58 +853,82 @@ tbik_status tbik_logprob(const uint16_t* hidden, const uint16_t* W, const int32_
     if (!aligned16(hidden) || !aligned16(W) || !aligned16(targets) || !aligned16(out)) return TBIK_ERR_ALIGN;
     if (!ws || ws_bytes < p.total) return TBIK_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return TBIK_ERR_ALIGN;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
-    float* stats = reinterpret_cast<float*>(w8 + p.off_stats);
-    float* zt = reinterpret_cast<float*>(w8 + p.off_zt);
-    float* shard = reinterpret_cast<float*>(w8 + p.off_shard);
-    if (p.tc) {
-        CUtensorMap ta, tb;
-        const int a_box = a_box_rows(M);
-        if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
-        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, 64, TC_BN / 2)) return TBIK_ERR_CUDA;
-        TcParams prm;
-        memset(&prm, 0, sizeof(prm));
-        set_ring(prm, a_box);
-        prm.M = M, prm.N = V, prm.K = H;
-        prm.leaf = p.noninv ? H / T : leaf;
-        prm.seq = p.noninv ? 1 : 0;
-        prm.F = 1;
-        prm.tiles_m = p.tiles_m, prm.tiles_n = p.nvt;
-        prm.group_m = p.tiles_m;  // all row tiles of a vocab tile run together: W_lm is read once
-        prm.total_units = p.units;
-        prm.direct = 1;
-        prm.scratch = p.gs ? reinterpret_cast<float*>(w8 + p.off_scratch) : nullptr;
-        prm.gs = p.gs;
-        prm.b_mn = 0;
-        prm.targets = targets;
-        prm.stats = stats;
-        prm.zt = zt;
-        prm.V = V;
-        prm.debug = g_debug_flags & ~TBIK_DEBUG_WITHHOLD_ACC_ARRIVE;
-        prm.wait_cycles = wait_cycles(info);
-        prm.lo[0] = 0;
-        prm.nl[0] = (short)p.Lk;
-        prm.tab_n[0] = prm.tab_n[1] = prm.nl[0];
-        gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
-        if ((st = launch_status()) != TBIK_OK) return st;
-    } else {
-        float* z = reinterpret_cast<float*>(w8 + p.off_z);
-        GemmPlan zp;
-        st = zgemm_plan(p, info->sms, zp);
-        if (st != TBIK_OK) return st;
-        if (zp.total > p.zplan.total) return TBIK_ERR_WORKSPACE;
-        st = run_gemm(zp, hidden, W, z, w8 + p.off_zgemm, s, info);
-        if (st != TBIK_OK) return st;
-        const size_t work = (size_t)M * p.nvl;
-        int blocks = (int)((work + 255) / 256);
-        if (blocks > info->sms * 16) blocks = info->sms * 16;
-        vocab_stats_kernel<<<blocks, 256, 0, s>>>(z, targets, stats, zt, M, V, p.nvl);
-        if ((st = launch_status()) != TBIK_OK) return st;
-    }
-    logprob_row_kernel<<<(M + ROW_BLOCK - 1) / ROW_BLOCK, ROW_BLOCK * 32, 0, s>>>(stats, zt, targets, out, shard, M,
-                                                                                V, p.nvl, p.Lv, T);
+    return run_logprob(p, hidden, W, targets, out, nullptr, 0, reinterpret_cast<uint8_t*>(ws),
+                       reinterpret_cast<cudaStream_t>(stream), info);
+}
+
+size_t tbik_logprob_partial_workspace(int M, int Vs, int Lvs, int H, int leaf, unsigned mode) {
+    int dev;
+    DeviceInfo* info;
+    if (device_info(dev, info) != TBIK_OK) return (size_t)-1;
+    LogprobPlan p;
+    if (Lvs <= 0 || (mode & TBIK_NONINV) || plan_logprob(M, Vs, H, 1, leaf, mode, info->sms, p, Lvs) != TBIK_OK)
+        return (size_t)-1;
+    return p.total;
+}
+
+tbik_status tbik_logprob_partial(const uint16_t* hidden, const uint16_t* W_shard, const int32_t* targets, float* part,
+                                 int M, int Vs, int v0, int Lvs, int H, int leaf, unsigned mode, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (mode & TBIK_NONINV) return TBIK_ERR_ARG;
+    if (Lvs <= 0 || v0 < 0) return TBIK_ERR_ARG;
+    LogprobPlan p;
+    st = plan_logprob(M, Vs, H, 1, leaf, mode, info->sms, p, Lvs);
+    if (st != TBIK_OK) return st;
+    if (M == 0) return TBIK_OK;
+    if (!hidden || (Vs > 0 && !W_shard) || !targets || !part) return TBIK_ERR_ARG;
+    if (!aligned16(hidden) || (Vs > 0 && !aligned16(W_shard)) || !aligned16(targets) || !aligned16(part))
+        return TBIK_ERR_ALIGN;
+    if (!ws || ws_bytes < p.total) return TBIK_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return TBIK_ERR_ALIGN;
+    return run_logprob(p, hidden, W_shard, targets, nullptr, reinterpret_cast<float4*>(part), v0,
+                       reinterpret_cast<uint8_t*>(ws), reinterpret_cast<cudaStream_t>(stream), info);
+}
+
+tbik_status tbik_logprob_combine(const float* parts, const int32_t* targets, float* out, int M, int V, int T,
+                                 void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (M < 0 || V <= 0) return TBIK_ERR_ARG;
+    if (!valid_T(T)) return TBIK_ERR_SHAPE;
+    if (M == 0) return TBIK_OK;
+    if (!parts || !targets || !out) return TBIK_ERR_ARG;
+    if (!aligned16(parts) || !aligned16(targets) || !aligned16(out)) return TBIK_ERR_ALIGN;
+    int blocks = (M + 255) / 256;
+    if (blocks > info->sms * 8) blocks = info->sms * 8;
+    logprob_combine_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const float4*>(parts), targets, out, M, V, T);
     return launch_status();
+}
+
+tbik_status tbik_tree_combine(const float* partials, void* out, long long MN, int T, unsigned mode, const uint16_t* R,
+                              void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    if (mode & ~(TBIK_NONINV | TBIK_OUT_BF16)) return TBIK_ERR_ARG;
+    if (MN < 0) return TBIK_ERR_ARG;
+    if (!valid_T(T)) return TBIK_ERR_SHAPE;
+    const bool bf16 = mode & TBIK_OUT_BF16;
+    if (R && !bf16) return TBIK_ERR_ARG;
+    if (MN == 0) return TBIK_OK;
+    if (!partials || !out) return TBIK_ERR_ARG;
+    if (!aligned16(partials) || !aligned16(out) || (R && !aligned16(R))) return TBIK_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (mode & TBIK_NONINV) {
+        size_t blocks = ((size_t)MN + 255) / 256;
+        if (blocks > (size_t)info->sms * 8) blocks = (size_t)info->sms * 8;
+        seq_combine_kernel<<<(int)blocks, 256, 0, s>>>(partials, (size_t)MN, T, out, bf16 ? 1 : 0, R);
+        return launch_status();
+    }
+    return tree_combine(partials, (size_t)MN, T, 1, out, bf16 ? 1 : 0, s, info->sms, R);
 }
 
 tbik_status tbik_get_error(void* stream) {

@@ -13,7 +13,7 @@ import synth
 pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
-from tests.gpu_util import dev_bf16, host_bits16, host_f32, rel_frob, u32  # noqa: E402
+from tests.gpu_util import dev_bf16, host_bits16, host_f32, oracle_rows, rel_frob, sample_rows, u32  # noqa: E402
 
 import invariant_tree_ordered_b200 as tbik  # noqa: E402
 
@@ -181,16 +181,18 @@ def test_down_proj_tc_invariance_over_T_and_M(down_proj):
     # row i sits in a different tile position when the batch is shifted
     sub = run(a[5:133], b, T=4, leaf=256, tc=True)
     assert np.array_equal(u32(sub), u32(full[1][5:133]))
-    rows = [0, 1, 777, 4095]
-    c64 = oracle.gemm_f64(a[rows], b, b_nk=False)
+    rows = sample_rows(35, 4096, 64, must=(0, 1, 255, 256, 4095))
+    c64 = oracle_rows(lambda rs: oracle.gemm_f64(a[rs], b, b_nk=False), rows)
     assert rel_frob(full[1][rows], c64) <= 2e-5
 
 
 def test_down_proj_exact_sampled_rows_full_M(down_proj):
+    """64 seeded rows (tile edges included) of the exact-mode 4096-row launch at
+    T = 8, bit-exact to the oracle."""
     a, b = down_proj
     got = run(a, b, T=8, leaf=256, tc=False)
-    rows = [0, 2049, 4095]
-    ref = oracle.gemm_tree(a[rows], b, b_nk=False, T=1, leaf=256)
+    rows = sample_rows(36, 4096, 64, must=(0, 63, 64, 2049, 4095))
+    ref = oracle_rows(lambda rs: oracle.gemm_tree(a[rs], b, b_nk=False, T=1, leaf=256), rows)
     assert np.array_equal(u32(got[rows]), u32(ref))
 
 

@@ -13,7 +13,7 @@ import synth
 pytestmark = pytest.mark.gpu
 
 torch = pytest.importorskip("torch")
-from tests.gpu_util import dev_bf16, dev_i32, host_f32, u32  # noqa: E402
+from tests.gpu_util import dev_bf16, dev_i32, host_f32, oracle_rows, sample_rows, u32  # noqa: E402
 
 import invariant_tree_ordered_b200 as tbik  # noqa: E402
 
@@ -91,13 +91,27 @@ def test_lm_head_full_size_invariance_over_T_M_and_order(lm_head):
 
 
 def test_lm_head_full_size_vs_oracle_sampled_rows(lm_head):
+    """64 seeded rows of the 4096-token launch, compared with the oracle row by
+    row.  Their targets are set to the cases where an order or index mistake
+    would show: the first and last vocabulary columns, both sides of vocab-leaf
+    boundaries (64 columns), of the T = 8 shard boundaries (19008 columns) and
+    of 128-column GEMM tiles, and every column of the last vocabulary leaf's
+    edges [151872, 151936)."""
     hidden, w, targets, hd, wd, td = lm_head
-    tc = lp(hd, wd, td, T=8, tc=True)
-    rows = [0, 4095]
-    ref = oracle.logprob(hidden[rows], w, targets[rows], T=1, leaf=256)
+    V = 151936
+    rows = sample_rows(34, 4096, 64, must=(0, 1, 4095))
+    edge = [0, V - 1, 63, 64, 127, 128, 19007, 19008, 38015, 38016, 133055, 133056, 151871, 151872, 151873,
+            151935, 76031, 76032, 114047, 114048]
+    tg = targets.copy()
+    for i, r in enumerate(rows):
+        if i < len(edge):
+            tg[r] = edge[i]
+    tdd = dev_i32(tg)
+    tc = lp(hd, wd, tdd, T=8, tc=True)  # the full launch, T = 8
+    ref = oracle_rows(lambda rs: oracle.logprob(hidden[rs], w, tg[rs], T=1, leaf=256), rows)
     assert np.max(np.abs(tc[rows] - ref)) <= 1e-4
-    ex = lp(hd[:2].contiguous(), wd, td[:2].contiguous(), T=2, tc=False)
-    assert np.array_equal(u32(ex), u32(oracle.logprob(hidden[:2], w, targets[:2], T=1, leaf=256)))
+    ex = lp(hd[rows].contiguous(), wd, tdd[rows].contiguous(), T=2, tc=False)
+    assert np.array_equal(u32(ex), u32(ref))
 
 
 def test_lm_head_argument_errors(lm_head):
