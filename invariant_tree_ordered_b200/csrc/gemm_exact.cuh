@@ -5,20 +5,26 @@
 // reference mode of the library; it also yields the non-invariant baseline
 // (one leaf per shard) and the logits of the exact logprob mode.
 //
-// 64x64 output tile per CTA, 256 threads, 4x4 outputs per thread, K staged
-// through shared memory 16 deep as fp32 (bf16 widening is exact).  The tree
-// stack lives in per-thread local memory (touched once per leaf).
+// 128x128 output tile per CTA, 256 threads, 8x8 outputs per thread (rows
+// 4*ty + {0..3} and 64 + 4*ty + {0..3}, columns 4*tx + {0..3} and
+// 64 + 4*tx + {0..3}), so each k step reads four 16-byte shared-memory
+// vectors (two of A broadcast to the 16 threads of a row group, two of B) for
+// 64 fmas: the fp32 pipe, not shared memory, sets the pace.  K is staged 16
+// deep through shared memory as fp32 (bf16 widening is exact), double
+// buffered: the next chunk's global loads are in flight while the current one
+// is computed, one barrier per chunk.  The tree stack lives in per-thread local
+// memory (touched once per leaf).
 #pragma once
 
 #include "device_common.cuh"
 
 namespace tbik {
 
-constexpr int EX_BM = 64;
-constexpr int EX_BN = 64;
+constexpr int EX_BM = 128;
+constexpr int EX_BN = 128;
 constexpr int EX_KC = 16;
 constexpr int EX_THREADS = 256;
-constexpr int EX_MAXD = 20;
+constexpr int EX_MAXD = 16;
 constexpr int EX_MAX_F = 64;
 
 struct ExParams {
@@ -49,13 +55,68 @@ __device__ __forceinline__ void ex_store(void* out, int bf16, int M, int N, int 
         reinterpret_cast<float*>(out)[off] = v;
 }
 
+// Eight consecutive bf16 of one row, widened; elements at or past `lim` (or a
+// row past the matrix) read as 0.  VEC: one 16-byte load (the caller
+// guarantees 16-byte alignment and that the row holds all eight when p < lim).
+template <int VEC>
+__device__ __forceinline__ void ld8(const uint16_t* row_base, bool row_ok, int k, int lim, float (&f)[8]) {
+    if (VEC && row_ok && k + 8 <= lim) {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(row_base + k)), f);
+        return;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = (row_ok && k + e < lim) ? bf2f(row_base[k + e]) : 0.0f;
+}
+
+// One 16-deep K chunk [k0, k0+16) of the unit, cut at kend, into registers:
+// thread t holds 8 values of A (row t/2, k offsets 8*(t%2)..) and 8 of B.
+template <int B_NK, int VEC>
+__device__ __forceinline__ void ex_load_chunk(const ExParams& p, int m0, int n0, int k0, int kend, float (&fa)[8],
+                                              float (&fb)[8]) {
+    const int t = threadIdx.x;
+    {
+        const int r = t >> 1, kk = (t & 1) * 8, gm = m0 + r;
+        ld8<VEC>(p.A + (size_t)gm * p.K, gm < p.M, k0 + kk, kend, fa);
+    }
+    if (B_NK) {
+        const int c = t >> 1, kk = (t & 1) * 8, gn = n0 + c;
+        ld8<VEC>(p.B + (size_t)gn * p.K, gn < p.N, k0 + kk, kend, fb);
+    } else {
+        const int kk = t >> 4, c = (t & 15) * 8, gk = k0 + kk;
+        ld8<VEC>(p.B + (size_t)gk * p.N + n0, gk < kend, c, p.N - n0, fb);
+    }
+}
+
 template <int B_NK>
-__global__ void __launch_bounds__(EX_THREADS) gemm_exact_kernel(const __grid_constant__ ExParams p) {
-    __shared__ float As[EX_KC][EX_BM];
-    __shared__ __align__(16) float Bs[EX_KC][EX_BN];
+__device__ __forceinline__ void ex_store_chunk(float (*As)[EX_BM], float (*Bs)[EX_BN], const float (&fa)[8],
+                                               const float (&fb)[8]) {
+    const int t = threadIdx.x;
+    {
+        const int r = t >> 1, kk = (t & 1) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) As[kk + e][r] = fa[e];
+    }
+    if (B_NK) {
+        const int c = t >> 1, kk = (t & 1) * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) Bs[kk + e][c] = fb[e];
+    } else {
+        const int kk = t >> 4, c = (t & 15) * 8;
+        *reinterpret_cast<float4*>(&Bs[kk][c]) = make_float4(fb[0], fb[1], fb[2], fb[3]);
+        *reinterpret_cast<float4*>(&Bs[kk][c + 4]) = make_float4(fb[4], fb[5], fb[6], fb[7]);
+    }
+}
+
+// VEC = 1 needs K % 8 == 0, the leaf length % 8 == 0 (chunk starts are then
+// multiples of 8 elements) and, for [K,N] B, N % 8 == 0: every 16-byte load is
+// then aligned.  VEC = 0 loads element by element.  Same arithmetic either way.
+template <int B_NK, int VEC>
+__global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_constant__ ExParams p) {
+    __shared__ __align__(16) float As[2][EX_KC][EX_BM];
+    __shared__ __align__(16) float Bs[2][EX_KC][EX_BN];
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    float stk[EX_MAXD][16];
+    float stk[EX_MAXD][64];
 
     for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
         const int tiles = p.tiles_m * p.tiles_n;
@@ -66,84 +127,69 @@ __global__ void __launch_bounds__(EX_THREADS) gemm_exact_kernel(const __grid_con
         const int n = p.nl[f];
         const int kbeg = p.lo[f] * p.leaf;
         const int kend = kbeg + n * p.leaf;
-        float acc[16];
+        float acc[64];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
         int sp = 0, j = 0;
         int next_b = kbeg + p.leaf;
-
+        float fa[8], fb[8];
+        ex_load_chunk<B_NK, VEC>(p, m0, n0, kbeg, kend, fa, fb);
+        ex_store_chunk<B_NK>(As[0], Bs[0], fa, fb);
+        __syncthreads();
+        int buf = 0;
         for (int k0 = kbeg; k0 < kend; k0 += EX_KC) {
-            __syncthreads();
-            {
-                const int r = tid >> 2, kk = (tid & 3) * 4;
-                const int gm = m0 + r;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int gk = k0 + kk + e;
-                    As[kk + e][r] = (gm < p.M && gk < kend) ? bf2f(p.A[(size_t)gm * p.K + gk]) : 0.0f;
-                }
-            }
-            if (B_NK) {
-                const int c = tid >> 2, kk = (tid & 3) * 4;
-                const int gn = n0 + c;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int gk = k0 + kk + e;
-                    Bs[kk + e][c] = (gn < p.N && gk < kend) ? bf2f(p.B[(size_t)gn * p.K + gk]) : 0.0f;
-                }
-            } else {
-                const int kk = tid >> 4, c = (tid & 15) * 4;
-                const int gk = k0 + kk;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int gn = n0 + c + e;
-                    Bs[kk][c + e] = (gn < p.N && gk < kend) ? bf2f(p.B[(size_t)gk * p.N + gn]) : 0.0f;
-                }
-            }
-            __syncthreads();
+            const bool more = k0 + EX_KC < kend;
+            if (more) ex_load_chunk<B_NK, VEC>(p, m0, n0, k0 + EX_KC, kend, fa, fb);
             const int kc = min(EX_KC, kend - k0);
-            for (int kk = 0; kk < kc; ++kk) {
-                float a[4], b[4];
+            int kk = 0;
+            while (kk < kc) {
+                // k steps up to the next leaf boundary inside this chunk
+                const int seg = min(kc, next_b - k0);
+#pragma unroll 4
+                for (; kk < seg; ++kk) {
+                    const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+                    const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+                    const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+                    const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+                    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
-                const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-                b[0] = bv.x;
-                b[1] = bv.y;
-                b[2] = bv.z;
-                b[3] = bv.w;
+                    for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) acc[i * 4 + c] = __fmaf_rn(a[i], b[c], acc[i * 4 + c]);
-                if (k0 + kk + 1 == next_b) {
+                        for (int c = 0; c < 8; ++c) acc[i * 8 + c] = __fmaf_rn(a[i], b[c], acc[i * 8 + c]);
+                }
+                if (k0 + kk == next_b) {
                     // leaf j complete: apply the tree
                     const LeafOps ops = leaf_ops(n, j);
                     for (int i = 0; i < leaf_pops(ops); ++i) {
                         --sp;
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) acc[e] = __fadd_rn(stk[sp][e], acc[e]);
+                        for (int e = 0; e < 64; ++e) acc[e] = __fadd_rn(stk[sp][e], acc[e]);
                     }
                     if (ops.final_) {
                         void* dst = p.direct ? p.out : (void*)(p.partials + (size_t)f * p.M * p.N);
                         const int bf = p.direct ? p.out_bf16 : 0;
                         const uint16_t* res = p.direct ? p.residual : nullptr;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
+                        for (int i = 0; i < 8; ++i)
 #pragma unroll
-                            for (int c = 0; c < 4; ++c)
-                                ex_store(dst, bf, p.M, p.N, m0 + ty * 4 + i, n0 + tx * 4 + c, acc[i * 4 + c],
-                                         res);
+                            for (int c = 0; c < 8; ++c)
+                                ex_store(dst, bf, p.M, p.N, m0 + (i >> 2) * 64 + ty * 4 + (i & 3),
+                                         n0 + (c >> 2) * 64 + tx * 4 + (c & 3), acc[i * 8 + c], res);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) stk[sp][e] = acc[e];
+                        for (int e = 0; e < 64; ++e) stk[sp][e] = acc[e];
                         ++sp;
                     }
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+                    for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
                     ++j;
                     next_b += p.leaf;
                 }
             }
+            if (more) ex_store_chunk<B_NK>(As[buf ^ 1], Bs[buf ^ 1], fa, fb);
+            __syncthreads();
+            buf ^= 1;
         }
     }
 }

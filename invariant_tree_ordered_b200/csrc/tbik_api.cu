@@ -403,11 +403,20 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
             prm.lo[f] = (short)p.nodes[f].first;
             prm.nl[f] = (short)p.nodes[f].second;
         }
-        int grid = p.units < sms * 4 ? p.units : sms * 4;
-        if (p.b_nk)
-            gemm_exact_kernel<1><<<grid, EX_THREADS, 0, s>>>(prm);
-        else
-            gemm_exact_kernel<0><<<grid, EX_THREADS, 0, s>>>(prm);
+        int grid = p.units < sms ? p.units : sms;  // one resident CTA per SM
+        // 16-byte loads when every chunk start and row stride is 8 elements aligned
+        const bool vec = (p.K % 8 == 0) && (p.leaf_eff % 8 == 0) && (p.b_nk || p.N % 8 == 0);
+        if (p.b_nk) {
+            if (vec)
+                gemm_exact_kernel<1, 1><<<grid, EX_THREADS, 0, s>>>(prm);
+            else
+                gemm_exact_kernel<1, 0><<<grid, EX_THREADS, 0, s>>>(prm);
+        } else {
+            if (vec)
+                gemm_exact_kernel<0, 1><<<grid, EX_THREADS, 0, s>>>(prm);
+            else
+                gemm_exact_kernel<0, 0><<<grid, EX_THREADS, 0, s>>>(prm);
+        }
     }
     tbik_status st = launch_status();
     if (st != TBIK_OK) return st;
