@@ -106,6 +106,82 @@ __device__ __forceinline__ float swiglu1(float g, float u) {
     return __fmul_rn(sg, u);
 }
 
+// ---- two lanes per instruction (packed f32x2 add / mul / fma, sm_100) ------
+// Each lane of a packed operation is the IEEE round-to-nearest-even result of
+// the scalar operation on that lane, so the paired forms below return exactly
+// the bits of their scalar counterparts while issuing half the instructions.
+typedef unsigned long long f2x;
+
+__device__ __forceinline__ f2x pk2(float lo, float hi) {
+    f2x d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+__device__ __forceinline__ void upk2(f2x v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2x add2(f2x a, f2x b) {
+    f2x d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2x mul2(f2x a, f2x b) {
+    f2x d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2x fma2(f2x a, f2x b, f2x c) {
+    f2x d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// The scaling step of exp_spec for one lane: p * 2^k from the rint sum t.
+__device__ __forceinline__ float exp_scale(float p, float t) {
+    const int k = __float_as_int(t) - 0x4b400000;
+    if (k >= -125 && k <= 127) return __int_as_float(__float_as_int(p) + (int)((uint32_t)k << 23));
+    const int k1 = k / 2;
+    const int k2 = k - k1;
+    return __fmul_rn(__fmul_rn(p, pow2i(k1)), pow2i(k2));
+}
+
+// exp_spec of two values with the same operations in the same order: the
+// clamp, the rint by 1.5*2^23, the two-fma reduction (fma(-k, c, x) written as
+// fma(k, -c, x), the same exact product), the Horner polynomial and the scaling.
+__device__ __forceinline__ void exp_spec2(float x0, float x1, float& e0, float& e1) {
+    const float c0 = fminf(fmaxf(x0, -104.0f), 89.0f), c1 = fminf(fmaxf(x1, -104.0f), 89.0f);
+    const f2x x = pk2(c0, c1);
+    const f2x big = pk2(0x1.8p23f, 0x1.8p23f);
+    const f2x t = add2(mul2(x, pk2(0x1.715476p+0f, 0x1.715476p+0f)), big);
+    const f2x kf = add2(t, pk2(-0x1.8p23f, -0x1.8p23f));
+    f2x r = fma2(kf, pk2(-0x1.62e4p-1f, -0x1.62e4p-1f), x);
+    r = fma2(kf, pk2(-0x1.7f7d1cp-20f, -0x1.7f7d1cp-20f), r);
+    f2x p = pk2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
+    p = fma2(p, r, pk2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
+    p = fma2(p, r, pk2(0x1.111112p-7f, 0x1.111112p-7f));
+    p = fma2(p, r, pk2(0x1.555556p-5f, 0x1.555556p-5f));
+    p = fma2(p, r, pk2(0x1.555556p-3f, 0x1.555556p-3f));
+    p = fma2(p, r, pk2(0.5f, 0.5f));
+    p = fma2(p, r, pk2(1.0f, 1.0f));
+    p = fma2(p, r, pk2(1.0f, 1.0f));
+    float p0, p1, t0, t1;
+    upk2(p, p0, p1);
+    upk2(t, t0, t1);
+    e0 = (x0 != x0) ? __fadd_rn(x0, x0) : exp_scale(p0, t0);
+    e1 = (x1 != x1) ? __fadd_rn(x1, x1) : exp_scale(p1, t1);
+}
+
+// swiglu1 of two elements: the exponential, the "1 +" and the product by u
+// packed; the correctly rounded division stays one per lane.
+__device__ __forceinline__ void swiglu2(float g0, float g1, float u0, float u1, float& o0, float& o1) {
+    float e0, e1;
+    exp_spec2(-g0, -g1, e0, e1);
+    float d0, d1;
+    upk2(add2(pk2(1.0f, 1.0f), pk2(e0, e1)), d0, d1);
+    const f2x sg = pk2(__fdiv_rn(g0, d0), __fdiv_rn(g1, d1));
+    upk2(mul2(sg, pk2(u0, u1)), o0, o1);
+}
+
 // 2^y through the hardware base-2 exponential (ex2.approx, denormal results
 // flushed to zero).  Used where results are compared by tolerance (the
 // tensor-core logprob's per-leaf sums of exp(z - max), whose terms are at

@@ -141,23 +141,31 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
             const bool more = k0 + EX_KC < kend;
             if (more) ex_load_chunk<B_NK, VEC>(p, m0, n0, k0 + EX_KC, kend, fa, fb);
             const int kc = min(EX_KC, kend - k0);
+            // one k step: acc[i][c] = fma(A[row i][k], B[k][col c], acc[i][c])
+            auto kstep = [&](int kk) {
+                const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+                const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+                const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+                const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc[i * 8 + c] = __fmaf_rn(a[i], b[c], acc[i * 8 + c]);
+            };
             int kk = 0;
-            while (kk < kc) {
+            if (kc == EX_KC && next_b - k0 >= EX_KC) {
+                // the whole chunk lies inside one leaf (the common case): straight-line steps
+#pragma unroll
+                for (int q = 0; q < EX_KC; ++q) kstep(q);
+                kk = EX_KC;
+            }
+            while (kk < kc || k0 + kk == next_b) {
                 // k steps up to the next leaf boundary inside this chunk
                 const int seg = min(kc, next_b - k0);
 #pragma unroll 4
-                for (; kk < seg; ++kk) {
-                    const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
-                    const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
-                    const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-                    const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
-                    const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) acc[i * 8 + c] = __fmaf_rn(a[i], b[c], acc[i * 8 + c]);
-                }
+                for (; kk < seg; ++kk) kstep(kk);
                 if (k0 + kk == next_b) {
                     // leaf j complete: apply the tree
                     const LeafOps ops = leaf_ops(n, j);

@@ -176,7 +176,8 @@ __global__ void rope_kernel(const uint16_t* __restrict__ q, const uint16_t* __re
 // out = bf16((g / (1 + exp(-g))) * u), one 8-element vector per thread per
 // iteration of a grid-stride loop; the next iteration's inputs are loaded
 // before this one's arithmetic, so loads stay in flight during the (ALU-heavy)
-// exp and division.
+// exp and division.  Elements go through swiglu2 in pairs (packed f32x2
+// arithmetic, the same bits as swiglu1).
 template <int IN_F32>
 struct Vec8;
 template <>
@@ -233,7 +234,7 @@ __global__ void swiglu_kernel(const void* __restrict__ g, const void* __restrict
         unpack_vec8<IN_F32>(cg, gf);
         unpack_vec8<IN_F32>(cu, uf);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = swiglu1(gf[e], uf[e]);
+        for (int e = 0; e < 8; e += 2) swiglu2(gf[e], gf[e + 1], uf[e], uf[e + 1], o[e], o[e + 1]);
         reinterpret_cast<uint4*>(out)[i] = pack8(o);
         if (!more) break;
         i = inext;
@@ -262,7 +263,7 @@ __global__ void swiglu_interleaved_kernel(const float* __restrict__ gu, uint16_t
         g[0] = g0.x, g[1] = g0.y, g[2] = g0.z, g[3] = g0.w, g[4] = g1.x, g[5] = g1.y, g[6] = g1.z, g[7] = g1.w;
         u[0] = u0.x, u[1] = u0.y, u[2] = u0.z, u[3] = u0.w, u[4] = u1.x, u[5] = u1.y, u[6] = u1.z, u[7] = u1.w;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = swiglu1(g[k], u[k]);
+        for (int k = 0; k < 8; k += 2) swiglu2(g[k], g[k + 1], u[k], u[k + 1], o[k], o[k + 1]);
         *reinterpret_cast<uint4*>(out + (size_t)m * F + f0) = pack8(o);
     }
 }

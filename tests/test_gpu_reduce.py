@@ -108,6 +108,23 @@ def test_swiglu_bitwise_fp32_inputs_and_special_values():
     assert np.all(same)
 
 
+def test_swiglu_every_bf16_gate_value():
+    """Every one of the 65536 bf16 bit patterns as the gate (NaNs, infinities,
+    subnormals, both zeros included) against the oracle, with two up values:
+    the kernel pairs elements for its packed arithmetic, so each pattern is
+    checked in both lanes (even and odd positions)."""
+    g = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    g2 = np.concatenate([g, np.roll(g, 1)])  # each pattern at an even and an odd index
+    for u_val in (1.0, -2.5):
+        u = np.full(g2.shape, np.float32(u_val), dtype=np.float32)
+        ub = (u.view(np.uint32) >> 16).astype(np.uint16)
+        _, _, out = tbik.rope_swiglu(g=dev_bf16(g2), u=dev_bf16(ub))
+        ref = oracle.swiglu(g2, ub)
+        got = host_bits16(out)
+        same = (got == ref) | (np.isnan(synth.bf16_bits_to_f32(got)) & np.isnan(synth.bf16_bits_to_f32(ref)))
+        assert np.all(same), u_val
+
+
 def test_rope_swiglu_argument_errors():
     lib = tbik.load_library()
     a = tbik._binding.RopeSwigluArgs()
