@@ -268,7 +268,7 @@ struct LeafOps {
     bool final_;         // that value is the root of the tree over n leaves
 };
 
-__device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
+__host__ __device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
     LeafOps o;
     o.n1 = o.n2 = o.nm = o.nb = 0;
     int lo = 0, sz = n, top = 1;
@@ -303,7 +303,7 @@ __device__ __forceinline__ LeafOps leaf_ops(int n, int j) {
 
 // The same operations for the left-to-right chain ((L0 + L1) + L2) + ... of
 // the non-invariant baseline: leaf j > 0 pops the running sum of j leaves.
-__device__ __forceinline__ LeafOps seq_leaf_ops(int n, int j) {
+__host__ __device__ __forceinline__ LeafOps seq_leaf_ops(int n, int j) {
     LeafOps o;
     o.n1 = o.n2 = o.nm = o.nb = 0;
     if (j == 1)
@@ -319,19 +319,19 @@ __device__ __forceinline__ LeafOps seq_leaf_ops(int n, int j) {
     return o;
 }
 
-__device__ __forceinline__ int leaf_pops(const LeafOps& o) { return o.n1 + o.n2 + o.nm + o.nb; }
+__host__ __device__ __forceinline__ int leaf_pops(const LeafOps& o) { return o.n1 + o.n2 + o.nm + o.nb; }
 
 // A leaf's operations packed in 16 bits, so a table built once per CTA replaces
 // the walk (which costs several hundred cycles of dependent branches):
 // bit 0 pop of a single leaf, bit 1 pop of a 2-leaf value, bit 2 pop of a 3-4
 // leaf value, bits 3-7 pops of >= 5 leaf values, bits 8-9 size class of the
 // pushed value (0: 1 leaf, 1: 2, 2: 3-4, 3: >= 5), bit 10 final.
-__device__ __forceinline__ uint16_t encode_leaf_ops(const LeafOps& o) {
+__host__ __device__ __forceinline__ uint16_t encode_leaf_ops(const LeafOps& o) {
     const int cls = o.push_size == 1 ? 0 : (o.push_size == 2 ? 1 : (o.push_size <= 4 ? 2 : 3));
     return (uint16_t)(o.n1 | (o.n2 << 1) | (o.nm << 2) | (o.nb << 3) | (cls << 8) | ((o.final_ ? 1 : 0) << 10));
 }
 
-__device__ __forceinline__ int code_pops(uint32_t code) {
+__host__ __device__ __forceinline__ int code_pops(uint32_t code) {
     return (code & 1) + ((code >> 1) & 1) + ((code >> 2) & 1) + ((code >> 3) & 31);
 }
 

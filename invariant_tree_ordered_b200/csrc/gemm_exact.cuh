@@ -9,7 +9,10 @@
 // 4*ty + {0..3} and 64 + 4*ty + {0..3}, columns 4*tx + {0..3} and
 // 64 + 4*tx + {0..3}), so each k step reads four 16-byte shared-memory
 // vectors (two of A broadcast to the 16 threads of a row group, two of B) for
-// 64 fmas: the fp32 pipe, not shared memory, sets the pace.  K is staged 16
+// 64 fmas: the fp32 pipe, not shared memory, sets the pace.  The fmas run two
+// columns per instruction (packed f32x2: each lane is the IEEE fmaf of that
+// column, so every output is still one scalar fmaf chain), which halves the
+// instructions the scheduler issues per k step.  K is staged 16
 // deep through shared memory as fp32 (bf16 widening is exact), double
 // buffered: the next chunk's global loads are in flight while the current one
 // is computed, one barrier per chunk.  The tree stack lives in per-thread local
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
     __shared__ __align__(16) float Bs[2][EX_KC][EX_BN];
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    float stk[EX_MAXD][64];
+    f2x stk[EX_MAXD][8][4];
 
     for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
         const int tiles = p.tiles_m * p.tiles_n;
@@ -127,9 +130,14 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
         const int n = p.nl[f];
         const int kbeg = p.lo[f] * p.leaf;
         const int kend = kbeg + n * p.leaf;
-        float acc[64];
+        // acc[i][q]: row i (4*ty + i, then 64 + 4*ty + i - 4) and the column
+        // pair q (4*tx + 2q, +1, then 64 + 4*tx + 2q - 4, +1), one packed
+        // f32x2 register pair; every lane is the same fmaf chain as a scalar.
+        f2x acc[8][4];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[i][q] = 0ull;  // (+0.0f, +0.0f)
         int sp = 0, j = 0;
         int next_b = kbeg + p.leaf;
         float fa[8], fb[8];
@@ -141,18 +149,20 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
             const bool more = k0 + EX_KC < kend;
             if (more) ex_load_chunk<B_NK, VEC>(p, m0, n0, k0 + EX_KC, kend, fa, fb);
             const int kc = min(EX_KC, kend - k0);
-            // one k step: acc[i][c] = fma(A[row i][k], B[k][col c], acc[i][c])
+            // one k step: acc[i][c] = fma(A[row i][k], B[k][col c], acc[i][c]), two columns per instruction
             auto kstep = [&](int kk) {
                 const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
                 const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
                 const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
                 const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
                 const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                const f2x b[4] = {pk2(b0.x, b0.y), pk2(b0.z, b0.w), pk2(b1.x, b1.y), pk2(b1.z, b1.w)};
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 8; ++i) {
+                    const f2x ai = pk2(a[i], a[i]);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[i * 8 + c] = __fmaf_rn(a[i], b[c], acc[i * 8 + c]);
+                    for (int q = 0; q < 4; ++q) acc[i][q] = fma2(ai, b[q], acc[i][q]);
+                }
             };
             int kk = 0;
             if (kc == EX_KC && next_b - k0 >= EX_KC) {
@@ -167,30 +177,41 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
 #pragma unroll 4
                 for (; kk < seg; ++kk) kstep(kk);
                 if (k0 + kk == next_b) {
-                    // leaf j complete: apply the tree
+                    // leaf j complete: apply the tree (stack value + this value, per lane)
                     const LeafOps ops = leaf_ops(n, j);
                     for (int i = 0; i < leaf_pops(ops); ++i) {
                         --sp;
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) acc[e] = __fadd_rn(stk[sp][e], acc[e]);
+                        for (int r = 0; r < 8; ++r)
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) acc[r][q] = add2(stk[sp][r][q], acc[r][q]);
                     }
                     if (ops.final_) {
                         void* dst = p.direct ? p.out : (void*)(p.partials + (size_t)f * p.M * p.N);
                         const int bf = p.direct ? p.out_bf16 : 0;
                         const uint16_t* res = p.direct ? p.residual : nullptr;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
+                        for (int r = 0; r < 8; ++r)
 #pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                ex_store(dst, bf, p.M, p.N, m0 + (i >> 2) * 64 + ty * 4 + (i & 3),
-                                         n0 + (c >> 2) * 64 + tx * 4 + (c & 3), acc[i * 8 + c], res);
+                            for (int q = 0; q < 4; ++q) {
+                                float lo, hi;
+                                upk2(acc[r][q], lo, hi);
+                                const int row = m0 + (r >> 2) * 64 + ty * 4 + (r & 3);
+                                const int col = n0 + (q >> 1) * 64 + tx * 4 + (q & 1) * 2;
+                                ex_store(dst, bf, p.M, p.N, row, col, lo, res);
+                                ex_store(dst, bf, p.M, p.N, row, col + 1, hi, res);
+                            }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) stk[sp][e] = acc[e];
+                        for (int r = 0; r < 8; ++r)
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) stk[sp][r][q] = acc[r][q];
                         ++sp;
                     }
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) acc[e] = 0.0f;
+                    for (int r = 0; r < 8; ++r)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) acc[r][q] = 0ull;
                     ++j;
                     next_b += p.leaf;
                 }
