@@ -5,17 +5,15 @@
 // reference mode of the library; it also yields the non-invariant baseline
 // (one leaf per shard) and the logits of the exact logprob mode.
 //
-// 128x128 output tile per CTA, 256 threads, 8x8 outputs per thread (rows
-// 4*ty + {0..3} and 64 + 4*ty + {0..3}, columns 4*tx + {0..3} and
-// 64 + 4*tx + {0..3}), so each k step reads four 16-byte shared-memory
-// vectors (two of A broadcast to the 16 threads of a row group, two of B) for
-// 64 fmas: the fp32 pipe, not shared memory, sets the pace.  The fmas run two
-// columns per instruction (packed f32x2: each lane is the IEEE fmaf of that
-// column, so every output is still one scalar fmaf chain), which halves the
-// instructions the scheduler issues per k step.  K is staged 16
-// deep through shared memory as fp32 (bf16 widening is exact), double
-// buffered: the next chunk's global loads are in flight while the current one
-// is computed, one barrier per chunk.  The tree stack lives in per-thread local
+// 128x128 output tile per CTA, 512 threads (16 warps per SM), 8x4 outputs per
+// thread: rows 4*ty + {0..3} and 64 + 4*ty + {0..3}, columns 4*tx + {0..3}
+// (tx = lane, ty = warp), so each k step reads two 16-byte vectors of A (the
+// same for the whole warp: broadcast) and one of B for 32 fmas.  The fmas run
+// two columns per instruction (packed f32x2: each lane is the IEEE fmaf of
+// that column, so every output is still one scalar fmaf chain).  K is staged
+// 16 deep through shared memory as fp32 (bf16 widening is exact), double
+// buffered, with the global loads two chunks ahead (held as raw bf16 until
+// they are widened into shared memory), one barrier per chunk.  The tree stack lives in per-thread local
 // memory (touched once per leaf).
 #pragma once
 
@@ -26,7 +24,7 @@ namespace tbik {
 constexpr int EX_BM = 128;
 constexpr int EX_BN = 128;
 constexpr int EX_KC = 16;
-constexpr int EX_THREADS = 256;
+constexpr int EX_THREADS = 512;
 constexpr int EX_MAXD = 16;
 constexpr int EX_MAX_F = 64;
 
@@ -58,68 +56,81 @@ __device__ __forceinline__ void ex_store(void* out, int bf16, int M, int N, int 
         reinterpret_cast<float*>(out)[off] = v;
 }
 
-// Eight consecutive bf16 of one row, widened; elements at or past `lim` (or a
-// row past the matrix) read as 0.  VEC: one 16-byte load (the caller
-// guarantees 16-byte alignment and that the row holds all eight when p < lim).
+// Four consecutive bf16 of one row as raw 16-bit patterns in a uint2 (widened
+// only when stored to shared memory); elements at or past `lim` (or a row past
+// the matrix) read as 0.  VEC: one 8-byte load (the caller guarantees 8-byte
+// alignment and that the row holds all four when k < lim).
 template <int VEC>
-__device__ __forceinline__ void ld8(const uint16_t* row_base, bool row_ok, int k, int lim, float (&f)[8]) {
-    if (VEC && row_ok && k + 8 <= lim) {
-        unpack8(__ldg(reinterpret_cast<const uint4*>(row_base + k)), f);
-        return;
-    }
+__device__ __forceinline__ uint2 ld4raw(const uint16_t* row_base, bool row_ok, int k, int lim) {
+    if (VEC && row_ok && k + 4 <= lim) return __ldg(reinterpret_cast<const uint2*>(row_base + k));
+    uint32_t h[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = (row_ok && k + e < lim) ? bf2f(row_base[k + e]) : 0.0f;
+    for (int e = 0; e < 4; ++e) h[e] = (row_ok && k + e < lim) ? (uint32_t)row_base[k + e] : 0u;
+    return make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
 }
 
-// One 16-deep K chunk [k0, k0+16) of the unit, cut at kend, into registers:
-// thread t holds 8 values of A (row t/2, k offsets 8*(t%2)..) and 8 of B.
+__device__ __forceinline__ void widen4(uint2 w, float (&f)[4]) {
+    f[0] = __uint_as_float(w.x << 16);
+    f[1] = __uint_as_float(w.x & 0xffff0000u);
+    f[2] = __uint_as_float(w.y << 16);
+    f[3] = __uint_as_float(w.y & 0xffff0000u);
+}
+
+// The operands of one 16-deep K chunk [k0, k0+16) of the unit, cut at kend:
+// thread t holds 4 values of A (row t/4, k offsets 4*(t%4)..) and 4 of B.
+struct ExChunk {
+    uint2 a, b;
+};
+
 template <int B_NK, int VEC>
-__device__ __forceinline__ void ex_load_chunk(const ExParams& p, int m0, int n0, int k0, int kend, float (&fa)[8],
-                                              float (&fb)[8]) {
+__device__ __forceinline__ ExChunk ex_load_chunk(const ExParams& p, int m0, int n0, int k0, int kend) {
     const int t = threadIdx.x;
+    ExChunk c;
     {
-        const int r = t >> 1, kk = (t & 1) * 8, gm = m0 + r;
-        ld8<VEC>(p.A + (size_t)gm * p.K, gm < p.M, k0 + kk, kend, fa);
+        const int r = t >> 2, kk = (t & 3) * 4, gm = m0 + r;
+        c.a = ld4raw<VEC>(p.A + (size_t)gm * p.K, gm < p.M, k0 + kk, kend);
     }
     if (B_NK) {
-        const int c = t >> 1, kk = (t & 1) * 8, gn = n0 + c;
-        ld8<VEC>(p.B + (size_t)gn * p.K, gn < p.N, k0 + kk, kend, fb);
+        const int col = t >> 2, kk = (t & 3) * 4, gn = n0 + col;
+        c.b = ld4raw<VEC>(p.B + (size_t)gn * p.K, gn < p.N, k0 + kk, kend);
     } else {
-        const int kk = t >> 4, c = (t & 15) * 8, gk = k0 + kk;
-        ld8<VEC>(p.B + (size_t)gk * p.N + n0, gk < kend, c, p.N - n0, fb);
+        const int kk = t >> 5, col = (t & 31) * 4, gk = k0 + kk;
+        c.b = ld4raw<VEC>(p.B + (size_t)gk * p.N + n0, gk < kend, col, p.N - n0);
     }
+    return c;
 }
 
 template <int B_NK>
-__device__ __forceinline__ void ex_store_chunk(float (*As)[EX_BM], float (*Bs)[EX_BN], const float (&fa)[8],
-                                               const float (&fb)[8]) {
+__device__ __forceinline__ void ex_store_chunk(float (*As)[EX_BM], float (*Bs)[EX_BN], const ExChunk& c) {
     const int t = threadIdx.x;
+    float fa[4], fb[4];
+    widen4(c.a, fa);
+    widen4(c.b, fb);
     {
-        const int r = t >> 1, kk = (t & 1) * 8;
+        const int r = t >> 2, kk = (t & 3) * 4;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) As[kk + e][r] = fa[e];
+        for (int e = 0; e < 4; ++e) As[kk + e][r] = fa[e];
     }
     if (B_NK) {
-        const int c = t >> 1, kk = (t & 1) * 8;
+        const int col = t >> 2, kk = (t & 3) * 4;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) Bs[kk + e][c] = fb[e];
+        for (int e = 0; e < 4; ++e) Bs[kk + e][col] = fb[e];
     } else {
-        const int kk = t >> 4, c = (t & 15) * 8;
-        *reinterpret_cast<float4*>(&Bs[kk][c]) = make_float4(fb[0], fb[1], fb[2], fb[3]);
-        *reinterpret_cast<float4*>(&Bs[kk][c + 4]) = make_float4(fb[4], fb[5], fb[6], fb[7]);
+        const int kk = t >> 5, col = (t & 31) * 4;
+        *reinterpret_cast<float4*>(&Bs[kk][col]) = make_float4(fb[0], fb[1], fb[2], fb[3]);
     }
 }
 
 // VEC = 1 needs K % 8 == 0, the leaf length % 8 == 0 (chunk starts are then
-// multiples of 8 elements) and, for [K,N] B, N % 8 == 0: every 16-byte load is
+// multiples of 8 elements) and, for [K,N] B, N % 8 == 0: every 8-byte load is
 // then aligned.  VEC = 0 loads element by element.  Same arithmetic either way.
 template <int B_NK, int VEC>
 __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_constant__ ExParams p) {
     __shared__ __align__(16) float As[2][EX_KC][EX_BM];
     __shared__ __align__(16) float Bs[2][EX_KC][EX_BN];
     const int tid = threadIdx.x;
-    const int tx = tid & 15, ty = tid >> 4;
-    f2x stk[EX_MAXD][8][4];
+    const int tx = tid & 31, ty = tid >> 5;
+    f2x stk[EX_MAXD][8][2];
 
     for (int u = blockIdx.x; u < p.total_units; u += gridDim.x) {
         const int tiles = p.tiles_m * p.tiles_n;
@@ -131,37 +142,39 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
         const int kbeg = p.lo[f] * p.leaf;
         const int kend = kbeg + n * p.leaf;
         // acc[i][q]: row i (4*ty + i, then 64 + 4*ty + i - 4) and the column
-        // pair q (4*tx + 2q, +1, then 64 + 4*tx + 2q - 4, +1), one packed
-        // f32x2 register pair; every lane is the same fmaf chain as a scalar.
-        f2x acc[8][4];
+        // pair q (4*tx + 2q, +1), one packed f32x2 register pair; every lane is
+        // the same fmaf chain as a scalar.
+        f2x acc[8][2];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) acc[i][q] = 0ull;  // (+0.0f, +0.0f)
+            for (int q = 0; q < 2; ++q) acc[i][q] = 0ull;  // (+0.0f, +0.0f)
         int sp = 0, j = 0;
         int next_b = kbeg + p.leaf;
-        float fa[8], fb[8];
-        ex_load_chunk<B_NK, VEC>(p, m0, n0, kbeg, kend, fa, fb);
-        ex_store_chunk<B_NK>(As[0], Bs[0], fa, fb);
+        // Two chunks in flight: chunk i+1's operands were loaded while chunk
+        // i-1 was computed, chunk i+2's are loaded while chunk i is computed.
+        ex_store_chunk<B_NK>(As[0], Bs[0], ex_load_chunk<B_NK, VEC>(p, m0, n0, kbeg, kend));
+        ExChunk next = {make_uint2(0u, 0u), make_uint2(0u, 0u)};
+        if (kbeg + EX_KC < kend) next = ex_load_chunk<B_NK, VEC>(p, m0, n0, kbeg + EX_KC, kend);
         __syncthreads();
         int buf = 0;
         for (int k0 = kbeg; k0 < kend; k0 += EX_KC) {
             const bool more = k0 + EX_KC < kend;
-            if (more) ex_load_chunk<B_NK, VEC>(p, m0, n0, k0 + EX_KC, kend, fa, fb);
+            ExChunk after = {make_uint2(0u, 0u), make_uint2(0u, 0u)};
+            if (k0 + 2 * EX_KC < kend) after = ex_load_chunk<B_NK, VEC>(p, m0, n0, k0 + 2 * EX_KC, kend);
             const int kc = min(EX_KC, kend - k0);
             // one k step: acc[i][c] = fma(A[row i][k], B[k][col c], acc[i][c]), two columns per instruction
             auto kstep = [&](int kk) {
                 const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
                 const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
                 const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
-                const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
                 const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const f2x b[4] = {pk2(b0.x, b0.y), pk2(b0.z, b0.w), pk2(b1.x, b1.y), pk2(b1.z, b1.w)};
+                const f2x b[2] = {pk2(b0.x, b0.y), pk2(b0.z, b0.w)};
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const f2x ai = pk2(a[i], a[i]);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) acc[i][q] = fma2(ai, b[q], acc[i][q]);
+                    for (int q = 0; q < 2; ++q) acc[i][q] = fma2(ai, b[q], acc[i][q]);
                 }
             };
             int kk = 0;
@@ -184,7 +197,7 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
 #pragma unroll
                         for (int r = 0; r < 8; ++r)
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) acc[r][q] = add2(stk[sp][r][q], acc[r][q]);
+                            for (int q = 0; q < 2; ++q) acc[r][q] = add2(stk[sp][r][q], acc[r][q]);
                     }
                     if (ops.final_) {
                         void* dst = p.direct ? p.out : (void*)(p.partials + (size_t)f * p.M * p.N);
@@ -193,11 +206,11 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
 #pragma unroll
                         for (int r = 0; r < 8; ++r)
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
+                            for (int q = 0; q < 2; ++q) {
                                 float lo, hi;
                                 upk2(acc[r][q], lo, hi);
                                 const int row = m0 + (r >> 2) * 64 + ty * 4 + (r & 3);
-                                const int col = n0 + (q >> 1) * 64 + tx * 4 + (q & 1) * 2;
+                                const int col = n0 + tx * 4 + q * 2;
                                 ex_store(dst, bf, p.M, p.N, row, col, lo, res);
                                 ex_store(dst, bf, p.M, p.N, row, col + 1, hi, res);
                             }
@@ -205,20 +218,21 @@ __global__ void __launch_bounds__(EX_THREADS, 1) gemm_exact_kernel(const __grid_
 #pragma unroll
                         for (int r = 0; r < 8; ++r)
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) stk[sp][r][q] = acc[r][q];
+                            for (int q = 0; q < 2; ++q) stk[sp][r][q] = acc[r][q];
                         ++sp;
                     }
 #pragma unroll
                     for (int r = 0; r < 8; ++r)
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) acc[r][q] = 0ull;
+                        for (int q = 0; q < 2; ++q) acc[r][q] = 0ull;
                     ++j;
                     next_b += p.leaf;
                 }
             }
-            if (more) ex_store_chunk<B_NK>(As[buf ^ 1], Bs[buf ^ 1], fa, fb);
+            if (more) ex_store_chunk<B_NK>(As[buf ^ 1], Bs[buf ^ 1], next);
             __syncthreads();
             buf ^= 1;
+            next = after;
         }
     }
 }
