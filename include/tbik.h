@@ -355,7 +355,7 @@ TBIK_API tbik_status tbik_logprob_combine(const float* parts, const int32_t* tar
  *    more scratch than TBIK_NOALLOC_SCRATCH_BYTES (that is, when
  *    tbik_logprob_workspace() for the same arguments is larger).  For the
  *    151936 x 4096 lm_head with leaf 256 on a 148-SM B200 this allows up to
- *    1251 rows per call.
+ *    997 rows per call.
  *  - Returns TBIK_ERR_ARG for any mode without TBIK_TC or with TBIK_EXACT;
  *    otherwise the status tbik_logprob would return for the same arguments
  *    (TBIK_ERR_ARG, _SHAPE, _CUDA, _UNSUPPORTED) before the size check.

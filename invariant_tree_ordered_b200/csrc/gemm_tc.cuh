@@ -4,39 +4,48 @@
 // Sizes That Eliminates Training-Inference Mismatch" (TBIK summary page),
 // sections 核心思路 / 技术框架: the K reduction is one hierarchical binary
 // tree shared by the local and the cross-GPU steps.  Here each K leaf is a
-// chain of 256x128x16 bf16 MMAs into an fp32 TMEM accumulator that restarts
+// chain of 256xBNx16 bf16 MMAs into an fp32 TMEM accumulator that restarts
 // from zero; the leaves are then combined by the halving tree in fp32 in the
 // epilogue.  The MMA sequence of a leaf depends only on the leaf's K range,
 // never on M, N or T, so a row's bits are the same for every batch size and
-// every shard count.
+// every shard count (and, as measured, for either tile width).
 //
-// CTA pairs (clusters of 2, cta_group::2): a pair computes a 256 x 128 tile;
-// CTA r holds rows [128r, 128r+128) of A and rows/columns [64r, 64r+64) of B
-// in its shared memory and its own 128 x 128 fp32 accumulators in TMEM.  The
-// leader (rank 0) issues the MMAs; commits arrive on both CTAs' barriers.
-// Each CTA (352 threads, one per SM, persistent over work units):
+// CTA pairs (clusters of 2, cta_group::2): a pair computes a 256 x BN tile,
+// BN = 128 when B is [K,N] and 192 when B is [N,K]; CTA r holds rows
+// [128r, 128r+128) of A and rows/columns [BN/2 r, BN/2 (r+1)) of B in its
+// shared memory and its own 128 x BN fp32 accumulators in TMEM.  The leader
+// (rank 0) issues the MMAs; commits arrive on both CTAs' barriers.  Each CTA
+// (one per SM, persistent over work units):
 //   warp 0     TMA producer: its A and B halves, 128 deep (two 64-wide
 //              128-byte-swizzle slices), into a ring of 3 stages (up to 8
 //              when M is small and only the valid A rows are copied)
 //   warp 1     TMEM allocator (both CTAs) + MMA issuer (leader, lane 0)
-//   warps 2-9  epilogue: drain each leaf from TMEM and apply the tree; warp w
-//              reads TMEM lanes 32*(w%4).. (its row quadrant) and the 64
-//              columns of half (w-2)/4 of the tile
-//   warp 10    waiter (leader): performs every mbarrier wait the issuer needs
+//   warps 2..  epilogue (8 warps for BN = 128, 12 for 192): drain each leaf
+//              from TMEM and apply the tree; warp w reads TMEM lanes
+//              32*(w%4).. (its row quadrant) and 64 columns of the tile
+//   next warp  waiter (leader): performs every mbarrier wait the issuer needs
 //              (stage landed, accumulator drained), then meets the MMA warp on
 //              a named barrier.  A barrier wait in the issuing thread costs the
 //              tensor pipe a few hundred cycles even when the barrier is
 //              already complete; a named barrier between two warps costs
 //              nothing, so the issuer only issues MMAs and commits.
-// TMEM (512 columns): three leaf accumulators (columns 0, 128, 256) and a slot
-// at column 384.  Pending subtree results wait by size: a single leaf stays in
-// its own accumulator (it is always consumed by the next leaf); 2 leaves in
-// the TMEM slot; 3-4 leaves in one shared-memory slot; >= 5 leaves in a
-// per-CTA fp32 scratch in global memory that stays in L2.  At most one value
-// of each of the first three classes is pending at a time.  The epilogue
-// handles a leaf in two phases: it first drains the leaf (and the single leaf
-// it pops) into registers and releases both accumulators, then does the other
-// pops and the push, so the MMA never waits on the rest of the tree work.
+// Pending subtree results wait by size (at most one value per on-chip class,
+// checked by a host replay of the leaf operation codes for every leaf count
+// up to 1100; values of >= 5 leaves go to a per-CTA fp32 scratch stack in
+// global memory that stays in L2):
+//   BN = 128: TMEM (512 columns) holds three leaf accumulators (columns 0,
+//     128, 256) and a 2-leaf slot (384); a single leaf stays in its own
+//     accumulator (the next leaf always consumes it); 3-4 leaves in a
+//     shared-memory slot.
+//   BN = 192: two accumulators (columns 0 and 256); a pending 2-leaf value
+//     stays in the epilogue's registers R (64 per thread); the 3-4 leaf slot
+//     is the spare TMEM columns [192, 256) and [448, 512) for column groups 0
+//     and 1 plus 32 KiB of shared memory for group 2; a single leaf goes to R
+//     when R is free, else to the slot when that is free, else it stays in its
+//     accumulator (then the MMA waits for the next leaf's first phase).
+// The epilogue handles a leaf in two phases: it first drains the leaf (and the
+// single leaf it pops) and releases the accumulators, then does the other pops
+// and the push, so the MMA does not wait on the rest of the tree work.
 // A work unit is (m tile, n tile, frontier node f): the node's subtree of
 // leaves is reduced by this pair; with more than one frontier node per tile the
 // subtree results go to fp32 partial buffers that a combine kernel reduces
@@ -49,26 +58,45 @@ namespace tbik {
 
 constexpr int TC_BM = 128;        // rows per CTA
 constexpr int TC_PAIR_M = 256;    // rows per CTA pair (one MMA tile)
-constexpr int TC_BN = 128;
-constexpr int TC_BK = 128;                // K per ring stage
-constexpr int TC_KSLICES = TC_BK / 64;    // 64-wide (128-byte) swizzle slices per stage
-constexpr int TC_KSTEPS = TC_BK / 16;     // MMAs (K = 16) per stage
-constexpr int TC_STAGES = 3;       // ring stages when A fills its 128 rows
-constexpr int TC_MAX_STAGES = 8;   // ring stages when the A copies are small (small M)
-constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;        // this CTA's A rows
-constexpr int TC_B_BYTES = (TC_BN / 2) * TC_BK * 2;  // this CTA's half of B
-constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quadrant, each owning 64 columns
-constexpr int TC_WAITER_WARP = 2 + TC_EPI_WARPS;
-constexpr int TC_THREADS = 32 * (TC_WAITER_WARP + 1);
+constexpr int TC_BN = 128;        // columns per pair tile when B is [K,N]
+constexpr int TC_BN_WIDE = 192;   // columns per pair tile when B is [N,K]
+constexpr int TC_MAX_STAGES = 8;  // ring stages when the A copies are small (small M)
 constexpr int TC_BAR_EPI = 1;      // named barrier: the epilogue warps
 constexpr int TC_BAR_HANDOFF = 2;  // named barrier: waiter warp + MMA warp, lockstep
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_MAX_F = 64;
-constexpr int TC_SLOT_FLOATS = TC_BM * TC_BN;
 constexpr int TC_TAB_MAX = 1024;  // leaves per subtree covered by the shared-memory op table
-constexpr int TC_RING_BYTES = TC_STAGES * (TC_A_BYTES + TC_B_BYTES);
-constexpr size_t TC_SMEM_BYTES = (size_t)TC_RING_BYTES + TC_SLOT_FLOATS * 4 +
-                                 2 * TC_TAB_MAX * 2 /*op tables*/ + 1024 /*align*/ + 256 /*barriers*/;
+
+// Per tile width: the 128-column tile keeps three leaf accumulators and a
+// 2-leaf slot in TMEM and its 3-4 leaf slot in shared memory.  The
+// 192-column tile keeps two accumulators (columns 0 and 256), holds a pending
+// 2-leaf value in the epilogue's registers (12 epilogue warps of 64 columns
+// each; 16 warps in all, so a thread may use 128 registers) and splits its
+// 3-4 leaf slot: column groups 0 and 1 in the spare TMEM columns [192, 256)
+// and [448, 512), group 2 in shared memory.
+template <int BN>
+struct TcCfg {
+    static constexpr bool kWide = BN != TC_BN;
+    static constexpr int BK = 128;                // K per ring stage
+    static constexpr int KSLICES = BK / 64;       // 64-wide (128-byte) swizzle slices per stage
+    static constexpr int KSTEPS = BK / 16;        // MMAs (K = 16) per stage
+    static constexpr int STAGES = 3;              // ring stages when A fills its 128 rows
+    static constexpr int EPI_WARPS = BN / 16;     // BN/64 column groups per TMEM lane quadrant
+    static constexpr int WAITER_WARP = 2 + EPI_WARPS;
+    static constexpr int THREADS = kWide ? 512 : 32 * (WAITER_WARP + 1);
+    static constexpr int NACC = kWide ? 2 : 3;    // leaf accumulators in TMEM
+    static constexpr int ACC_STRIDE = kWide ? 256 : 128;
+    static constexpr int A_BYTES = TC_BM * BK * 2;        // this CTA's A rows
+    static constexpr int B_BYTES = (BN / 2) * BK * 2;     // this CTA's half of B
+    static constexpr int RING_BYTES = STAGES * (A_BYTES + B_BYTES);
+    static constexpr int SLOT_FLOATS = TC_BM * BN;                      // one pending value (L2 stack slot)
+    static constexpr int SMEM_SLOT_FLOATS = kWide ? TC_BM * 64 : SLOT_FLOATS;  // its shared-memory part
+    static constexpr uint32_t TMEM_SPARE0 = 192, TMEM_SPARE1 = 448;    // wide: slot columns of groups 0, 1
+    static constexpr size_t SMEM_BYTES = (size_t)RING_BYTES + SMEM_SLOT_FLOATS * 4 + 2 * TC_TAB_MAX * 2 /*op tables*/ +
+                                         1024 /*align*/ + 256 /*barriers*/;
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    static_assert(THREADS / 32 > WAITER_WARP, "warp roles");
+};
 
 // EPI_TREE_RES: EPI_TREE whose direct tiles add the bf16 residual to the fp32
 // root before the output rounding (a separate instantiation, so the plain
@@ -87,7 +115,7 @@ struct TcParams {
     void* out;        // C [M,N]
     const uint16_t* residual;  // EPI_TREE_RES: bf16 [M,N] added to the root before the rounding (direct only)
     float* partials;  // [F][M][N]
-    float* scratch;   // [gridDim.x][gs][128*128], layout per slot [col/4][row][4]
+    float* scratch;   // [gridDim.x][gs][128*BN], layout per slot [col/4][row][4]
     int gs;           // global stack slots per CTA (pending subtrees of >= 5 leaves)
     int b_mn;         // 1: B is [K,N] (MN-major operand)
     // logprob epilogue
@@ -101,9 +129,9 @@ struct TcParams {
     unsigned long long wait_cycles;  // bound of every device-side wait, in SM cycles
     int seq;                         // 1: the leaves form the left-to-right chain, not the tree
     int a_box_rows;                  // rows per A copy: 128, or M rounded up to 8 when M <= 128
-    // Ring layout: stage s at s * stage_bytes holds two A slices of a_slice
-    // bytes (a_box_rows rows of 128 bytes) and then the two 8 KiB B slices;
-    // stages = TC_RING_BYTES / stage_bytes, at most TC_MAX_STAGES.
+    // Ring layout: stage s at s * stage_bytes holds the A slices of a_slice
+    // bytes (a_box_rows rows of 128 bytes) and then the B slices;
+    // stages = RING_BYTES / stage_bytes, at most TC_MAX_STAGES.
     int stages;
     uint32_t stage_bytes, a_slice;
     int tab_n[2];                    // the (at most two) subtree sizes of the frontier nodes
@@ -124,8 +152,9 @@ __device__ __forceinline__ void tc_decode(const TcParams& p, int u, int& tm, int
     tn = r / gm;
 }
 
+template <int BN>
 __device__ __forceinline__ float* scratch_slot(const TcParams& p, int slot) {
-    return p.scratch + ((size_t)blockIdx.x * p.gs + slot) * TC_SLOT_FLOATS;
+    return p.scratch + ((size_t)blockIdx.x * p.gs + slot) * TcCfg<BN>::SLOT_FLOATS;
 }
 
 // 32 columns (chunk c) of one row of a scratch slot; coalesced across the warp.
@@ -144,6 +173,18 @@ __device__ __forceinline__ void scratch_st(float* base, int c, int row, const fl
     for (int q = 0; q < 8; ++q)
         *reinterpret_cast<float4*>(base + ((size_t)(c * 8 + q) * TC_BM + row) * 4) =
             make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// 16 columns (chunk q) of one row of a slot, as raw bits (the layout of scratch_ld).
+__device__ __forceinline__ void scratch_ld16(const float* base, int q, int row, uint32_t (&w)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float4 x = *reinterpret_cast<const float4*>(base + ((size_t)(q * 4 + i) * TC_BM + row) * 4);
+        w[4 * i + 0] = __float_as_uint(x.x);
+        w[4 * i + 1] = __float_as_uint(x.y);
+        w[4 * i + 2] = __float_as_uint(x.z);
+        w[4 * i + 3] = __float_as_uint(x.w);
+    }
 }
 
 // Row `row` (global), columns [col0, col0+32) of the output; N % 8 == 0.
@@ -185,20 +226,78 @@ __device__ __forceinline__ void add_residual32(const uint16_t* R, int M, int N, 
     }
 }
 
-template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
+// Logprob epilogue of one warp's 64 columns, one vocab leaf (index vleaf,
+// first column c0 of this call's vocabulary): the max, then the sum of
+// exp(z - max) = 2^(z*log2e - max*log2e) as two interleaved partial sums (even
+// and odd columns, each ascending) added at the end; (max, sum) go to
+// stats[vleaf][row] and the target's logit to zt[row].  Hardware exponential:
+// this mode is checked by tolerance; the order is fixed, so the bits are the
+// same for every T and M.  v is the fp32 root of the K tree for the 64 columns.
+__device__ __forceinline__ void logprob_leaf_stats(const TcParams& p, float (&v)[2][32], int row, int c0,
+                                                   int vleaf) {
+    if (c0 < p.V) {
+        // target column relative to this call's first vocabulary column
+        const long long tgt = (row < p.M) ? (long long)p.targets[row] - p.v0 : -1;
+        const int ncol = min(64, p.V - c0);
+        const long long kt = tgt - c0;  // target column within this leaf
+        const bool have_t = kt >= 0 && kt < ncol;
+        const int kti = have_t ? (int)kt : -1;
+        float zval = 0.0f;
+        if (have_t) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                if (k == kti) zval = v[0][k];
+                if (k + 32 == kti) zval = v[1][k];
+            }
+        }
+        if (ncol < 64) {  // the last vocab leaf: columns past V add nothing
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                if (k >= ncol) v[0][k] = -INFINITY;
+                if (k + 32 >= ncol) v[1][k] = -INFINITY;
+            }
+        }
+        float m = v[0][0];
+#pragma unroll
+        for (int k = 1; k < 32; ++k) m = fmaxf(m, v[0][k]);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) m = fmaxf(m, v[1][k]);
+        const float log2e = 0x1.715476p+0f;
+        const float ml = -__fmul_rn(m, log2e);
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+            for (int k = 0; k < 32; k += 2) {
+                s0 = __fadd_rn(s0, ex2_hw(__fmaf_rn(v[cc][k], log2e, ml)));
+                s1 = __fadd_rn(s1, ex2_hw(__fmaf_rn(v[cc][k + 1], log2e, ml)));
+            }
+        const float s = __fadd_rn(s0, s1);
+        if (row < p.M) {
+            *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
+            if (have_t) {
+                p.zt[row] = zval;
+                if (p.zflag) p.zflag[row] = 1;
+            }
+        }
+    }
+}
+
+template <int EPI, int BN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ TcParams p) {
+    using Cfg = TcCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* ring = smem;
-    float* sSlot = reinterpret_cast<float*>(smem + TC_RING_BYTES);  // pending 3-4 leaf subtree
-    uint16_t* leaf_tab = reinterpret_cast<uint16_t*>(sSlot + TC_SLOT_FLOATS);  // [2][TC_TAB_MAX]
+    float* sSlot = reinterpret_cast<float*>(smem + Cfg::RING_BYTES);  // pending 3-4 leaf subtree
+    uint16_t* leaf_tab = reinterpret_cast<uint16_t*>(sSlot + Cfg::SMEM_SLOT_FLOATS);  // [2][TC_TAB_MAX]
     uint64_t* bars = reinterpret_cast<uint64_t*>(leaf_tab + 2 * TC_TAB_MAX);
     uint64_t* full = bars;                          // [stages] both CTAs' copies landed (leader's)
     uint64_t* empty = bars + TC_MAX_STAGES;         // [stages] MMAs done reading (both CTAs)
-    uint64_t* acc_full = bars + 2 * TC_MAX_STAGES;  // [3] leaf accumulator ready (both CTAs)
-    uint64_t* acc_empty = acc_full + 3;         // [3] leaf accumulator drained by both CTAs (leader's)
+    uint64_t* acc_full = bars + 2 * TC_MAX_STAGES;  // [NACC] leaf accumulator ready (both CTAs)
+    uint64_t* acc_empty = acc_full + 3;         // [NACC] leaf accumulator drained by both CTAs (leader's)
     uint64_t* done = acc_empty + 3;             // all MMAs retired (both CTAs)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -219,9 +318,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 3; ++b) {
+        for (int b = 0; b < Cfg::NACC; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 2 * TC_EPI_WARPS);
+            mbar_init(&acc_empty[b], 2 * Cfg::EPI_WARPS);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -257,31 +356,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
                 const int k0 = p.lo[f] * p.leaf;
-                const int nkb = (p.nl[f] * p.leaf + TC_BK - 1) / TC_BK;
+                const int nkb = (p.nl[f] * p.leaf + Cfg::BK - 1) / Cfg::BK;
                 const int arow = tm * TC_PAIR_M + TC_BM * rank;
-                const int brow = tn * TC_BN + (TC_BN / 2) * rank;
+                const int brow = tn * BN + (BN / 2) * rank;
                 // A CTA whose 128 rows are all past M copies no A: the MMA
                 // then reads stale shared memory for rows whose results are
                 // never stored (rows of an MMA are independent).  Small M also
                 // copies only a_box_rows rows.
                 const int rows_pair = p.M - tm * TC_PAIR_M;
                 const bool a_mine = rows_pair - TC_BM * (int)rank > 0;
-                const uint32_t a_copy = p.a_slice * TC_KSLICES;  // bytes per CTA and stage
-                const uint32_t tx = a_copy * (rows_pair > TC_BM ? 2u : 1u) + 2u * TC_B_BYTES;
+                const uint32_t a_copy = p.a_slice * Cfg::KSLICES;  // bytes per CTA and stage
+                const uint32_t tx = a_copy * (rows_pair > TC_BM ? 2u : 1u) + 2u * Cfg::B_BYTES;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, wait_lim)) goto producer_out;
                     const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
-                    const int kx = k0 + kb * TC_BK;
+                    const int kx = k0 + kb * Cfg::BK;
                     uint8_t* sA = ring + (size_t)s * p.stage_bytes;
                     uint8_t* sB = sA + a_copy;
 #pragma unroll
-                    for (int h = 0; h < TC_KSLICES; ++h) {
+                    for (int h = 0; h < Cfg::KSLICES; ++h) {
                         if (a_mine) tma_load_2d_pair(sA + h * p.a_slice, &tmA, bar, kx + 64 * h, arow);
                         if (!b_mn)
-                            tma_load_2d_pair(sB + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar, kx + 64 * h, brow);
+                            tma_load_2d_pair(sB + h * (Cfg::B_BYTES / Cfg::KSLICES), &tmB, bar, kx + 64 * h, brow);
                         else
-                            tma_load_2d_pair(sB + h * (TC_B_BYTES / TC_KSLICES), &tmB, bar, brow, kx + 64 * h);
+                            tma_load_2d_pair(sB + h * (Cfg::B_BYTES / Cfg::KSLICES), &tmB, bar, brow, kx + 64 * h);
                     }
                     ++q;
                     if (++s == stages) {
@@ -296,30 +395,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 for (uint32_t i = (q > (uint32_t)stages ? q - stages : 0u); i < q; ++i)
                     mbar_drain(&full[i % stages], (i / stages) & 1, wait_lim);
         }
-    } else if (warp == 1 || warp == TC_WAITER_WARP) {
+    } else if (warp == 1 || warp == Cfg::WAITER_WARP) {
         // ------------------------------------------------ MMA issuer + waiter (leader)
         // Both warps walk the same sequence of k-steps.  A hand-off happens
         // where the issuer needs a condition: a stage start (its copies landed)
         // or a leaf start (its accumulator buffer drained).  The waiter checks
         // the condition(s), stores its verdict, and both warps bar.sync; the
         // issuer then reads the verdict, so the two always stop together.
-        // One 128-deep stage carries 8 MMAs of K = 16; descriptors are built
-        // once per stage and advanced through the start-address field.
+        // One stage carries BK/16 MMAs of K = 16; descriptors are built once
+        // per stage and advanced through the start-address field.
         const bool is_mma = warp == 1;
         if (rank == 0) {
-            const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, TC_BN, 0, p.b_mn);
+            const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, BN, 0, p.b_mn);
             const bool b_mn = p.b_mn != 0;
-            // MN-major B (a [K,N] operand): each CTA's 64 columns are one
-            // 128-byte swizzle atom wide, so the leading (MN) offset spans the
-            // whole half tile and the stride between 8-deep K groups is 1024 B.
-            constexpr uint32_t b_lbo = (uint32_t)TC_B_BYTES, b_sbo = 1024u;
+            // MN-major B (a [K,N] operand, 128-column tile only): each CTA's
+            // 64 columns are one 128-byte swizzle atom wide, so the leading
+            // (MN) offset spans the whole half tile and the stride between
+            // 8-deep K groups is 1024 B.
+            constexpr uint32_t b_lbo = (uint32_t)Cfg::B_BYTES, b_sbo = 1024u;
             const uint32_t ring_u = smem_u32(ring);
             const uint32_t stage_bytes = p.stage_bytes, a_slice = p.a_slice;
             const int stages = p.stages;
             const int spl = p.leaf / 16;  // MMAs per leaf
             const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
-            const bool aligned = (spl % TC_KSTEPS) == 0;  // leaf is a whole number of stages
-            const int kb_per_leaf = spl / TC_KSTEPS;
+            const bool aligned = (spl % Cfg::KSTEPS) == 0;  // leaf is a whole number of stages
+            const int kb_per_leaf = spl / Cfg::KSTEPS;
             uint32_t a = 0, hc = 0, ph = 0;  // ph: phase of the ring (flips when stage 0 comes round)
             int s = 0;
             // The hand-off: waiter lane 0 waits (bounded) for what the issuer needs.
@@ -331,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                         bool ok = true;
                         if (need_full) ok = mbar_wait(&full[s], ph, abort_flag, wait_lim);
                         if (ok && need_acc)
-                            ok = mbar_wait(&acc_empty[abuf], ((acount / 3) & 1) ^ 1, abort_flag, wait_lim);
+                            ok = mbar_wait(&acc_empty[abuf], ((acount / Cfg::NACC) & 1) ^ 1, abort_flag, wait_lim);
                         *verdict = ok ? 1 : 0;
                     }
                     __syncwarp();
@@ -347,12 +447,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 const int nsteps = p.nl[f] * spl;
                 uint32_t buf = 0;
                 int in_leaf = 0, kb_in_leaf = 0;
-                for (int st = 0; st < nsteps; st += TC_KSTEPS) {
+                for (int st = 0; st < nsteps; st += Cfg::KSTEPS) {
                     // The A slices of a small-M stage are a_box_rows rows apart;
                     // the MMA's other rows read whatever follows (results never
                     // stored), always inside this CTA's shared memory.
                     const uint32_t sa = ring_u + (uint32_t)s * stage_bytes;
-                    const uint32_t sb = sa + a_slice * TC_KSLICES;
+                    const uint32_t sb = sa + a_slice * Cfg::KSLICES;
                     const uint64_t adesc = smem_desc_sw128(sa, 16, 1024);
                     const uint64_t bdesc = b_mn ? smem_desc_sw128(sb, b_lbo, b_sbo) : smem_desc_sw128(sb, 16, 1024);
                     // k-step ks: slice ks/4 (advance by a slice's bytes >> 4), step ks%4 within it
@@ -360,16 +460,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                         return adesc + (uint64_t)((ks >> 2) * (a_slice >> 4) + (ks & 3) * 2);
                     };
                     auto b_at = [&](int ks) {
-                        return bdesc + (uint64_t)((ks >> 2) * ((TC_B_BYTES / TC_KSLICES) >> 4)) + b_step * (ks & 3);
+                        return bdesc + (uint64_t)((ks >> 2) * ((Cfg::B_BYTES / Cfg::KSLICES) >> 4)) + b_step * (ks & 3);
                     };
                     if (aligned) {
-                        if (kb_in_leaf == 0) buf = a % 3;
+                        if (kb_in_leaf == 0) buf = a % Cfg::NACC;
                         if (!handoff(true, kb_in_leaf == 0, buf, a)) goto mma_out;
                         if (is_mma && lane == 0) {
-                            const uint32_t d = tmem_base + buf * TC_BN;
+                            const uint32_t d = tmem_base + buf * Cfg::ACC_STRIDE;
                             tc_mma_pair(d, a_at(0), b_at(0), idesc, kb_in_leaf != 0 ? 1u : 0u);
 #pragma unroll
-                            for (int ks = 1; ks < TC_KSTEPS; ++ks) tc_mma_pair(d, a_at(ks), b_at(ks), idesc, 1u);
+                            for (int ks = 1; ks < Cfg::KSTEPS; ++ks) tc_mma_pair(d, a_at(ks), b_at(ks), idesc, 1u);
                             if (kb_in_leaf + 1 == kb_per_leaf) tc_commit_pair(&acc_full[buf]);
                         }
                         if (++kb_in_leaf == kb_per_leaf) {
@@ -377,13 +477,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                             kb_in_leaf = 0;
                         }
                     } else {
-                        const int nk = min(TC_KSTEPS, nsteps - st);
+                        const int nk = min(Cfg::KSTEPS, nsteps - st);
                         for (int ks = 0; ks < nk; ++ks) {
-                            if (in_leaf == 0) buf = a % 3;
+                            if (in_leaf == 0) buf = a % Cfg::NACC;
                             if (ks == 0 || in_leaf == 0)
                                 if (!handoff(ks == 0, in_leaf == 0, buf, a)) goto mma_out;
                             if (is_mma && lane == 0) {
-                                tc_mma_pair(tmem_base + buf * TC_BN, a_at(ks), b_at(ks), idesc, in_leaf != 0 ? 1u : 0u);
+                                tc_mma_pair(tmem_base + buf * Cfg::ACC_STRIDE, a_at(ks), b_at(ks), idesc,
+                                            in_leaf != 0 ? 1u : 0u);
                                 if (in_leaf + 1 == spl) tc_commit_pair(&acc_full[buf]);
                             }
                             if (++in_leaf == spl) {
@@ -405,8 +506,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             if (is_mma && lane == 0) tc_commit_pair(done);
         }
         if (is_mma && lane == 0) mbar_drain(done, 0, wait_lim);
-    } else {
+    } else if (warp < 2 + Cfg::EPI_WARPS) {
         // ------------------------------------------------ epilogue (both CTAs)
+      if constexpr (!Cfg::kWide) {
         const int ew = warp & 3;           // TMEM lane quadrant = rows 32*ew .. 32*ew+31
         const int half = (warp - 2) >> 2;  // columns [64*half, 64*half+64)
         const int rt = ew * 32 + lane;     // row within this CTA's 128
@@ -425,7 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 // One warp polls the accumulator barrier; the other epilogue
                 // warps wait on a hardware barrier, so nothing else polls.
                 if (warp == 2) mbar_wait(&acc_full[buf], (a / 3) & 1, abort_flag, wait_lim);
-                named_barrier_sync(TC_BAR_EPI, 32 * TC_EPI_WARPS);
+                named_barrier_sync(TC_BAR_EPI, 32 * Cfg::EPI_WARPS);
                 if (*abort_flag) goto epi_out;
                 ++a;
                 const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(p.seq ? seq_leaf_ops(n, j) : leaf_ops(n, j));
@@ -443,8 +545,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = half * 2 + cc;
                     uint32_t r0[32], r1[32];
-                    tmem_ld32_nowait(tl + buf * TC_BN + c * 32, r0);
-                    if (p1) tmem_ld32_nowait(tl + prev * TC_BN + c * 32, r1);
+                    tmem_ld32_nowait(tl + buf * Cfg::ACC_STRIDE + c * 32, r0);
+                    if (p1) tmem_ld32_nowait(tl + prev * Cfg::ACC_STRIDE + c * 32, r1);
                     tmem_wait_ld(r0);
                     if (p1) {
                         tie32(r1);
@@ -483,7 +585,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                     }
                 }
                 for (int i = 0; i < nb; ++i) {
-                    const float* sl = scratch_slot(p, gsp - 1 - i);
+                    const float* sl = scratch_slot<BN>(p, gsp - 1 - i);
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         float w[32];
@@ -503,14 +605,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                         else if (cls == 2)
                             scratch_st(sSlot, c, rt, v[cc]);
                         else
-                            scratch_st(scratch_slot(p, g_after), c, rt, v[cc]);
+                            scratch_st(scratch_slot<BN>(p, g_after), c, rt, v[cc]);
                     }
                     if (cls == 1) tmem_wait_st();
                 } else if (EPI == EPI_TREE && p.swiglu) {
                     // this warp's 64 columns: gate features f0..f0+31 (chunk 0)
                     // and the up values of the same features (chunk 1)
                     if (row < p.M) {
-                        const int f0 = tn * (TC_BN / 2) + half * 32;
+                        const int f0 = tn * (BN / 2) + half * 32;
                         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
                                                               (size_t)row * (p.N / 2) + f0);
 #pragma unroll
@@ -524,7 +626,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                 } else if (EPI != EPI_LOGPROB) {
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
-                        const int col = tn * TC_BN + (half * 2 + cc) * 32;
+                        const int col = tn * BN + (half * 2 + cc) * 32;
                         if (p.direct) {
                             if (EPI == EPI_TREE_RES) add_residual32(p.residual, p.M, p.N, row, col, v[cc]);
                             store_row32(p.out, p.out_bf16, p.M, p.N, row, col, v[cc]);
@@ -532,64 +634,191 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                             store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row, col, v[cc]);
                     }
                 } else {
-                    // Logprob: this warp's 64 columns are one vocab leaf.  The
-                    // max, then the sum of exp(z - max) = 2^(z*log2e - max*log2e)
-                    // as two interleaved partial sums (even and odd columns, each
-                    // ascending) added at the end.  Hardware exponential: this
-                    // mode is checked by tolerance; the order is fixed, so the
-                    // bits are the same for every T and M.
-                    const int c0 = tn * TC_BN + half * 64;
-                    const int vleaf = 2 * tn + half;
-                    if (c0 < p.V) {
-                        // target column relative to this call's first vocabulary column
-                        const long long tgt = (row < p.M) ? (long long)p.targets[row] - p.v0 : -1;
-                        const int ncol = min(64, p.V - c0);
-                        const long long kt = tgt - c0;  // target column within this leaf
-                        const bool have_t = kt >= 0 && kt < ncol;
-                        const int kti = have_t ? (int)kt : -1;
-                        float zval = 0.0f;
-                        if (have_t) {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                if (k == kti) zval = v[0][k];
-                                if (k + 32 == kti) zval = v[1][k];
-                            }
-                        }
-                        if (ncol < 64) {  // the last vocab leaf: columns past V add nothing
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                if (k >= ncol) v[0][k] = -INFINITY;
-                                if (k + 32 >= ncol) v[1][k] = -INFINITY;
-                            }
-                        }
-                        float m = v[0][0];
-#pragma unroll
-                        for (int k = 1; k < 32; ++k) m = fmaxf(m, v[0][k]);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) m = fmaxf(m, v[1][k]);
-                        const float log2e = 0x1.715476p+0f;
-                        const float ml = -__fmul_rn(m, log2e);
-                        float s0 = 0.0f, s1 = 0.0f;
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                            for (int k = 0; k < 32; k += 2) {
-                                s0 = __fadd_rn(s0, ex2_hw(__fmaf_rn(v[cc][k], log2e, ml)));
-                                s1 = __fadd_rn(s1, ex2_hw(__fmaf_rn(v[cc][k + 1], log2e, ml)));
-                            }
-                        const float s = __fadd_rn(s0, s1);
-                        if (row < p.M) {
-                            *reinterpret_cast<float2*>(p.stats + ((size_t)vleaf * p.M + row) * 2) = make_float2(m, s);
-                            if (have_t) {
-                                p.zt[row] = zval;
-                                if (p.zflag) p.zflag[row] = 1;
-                            }
-                        }
-                    }
+                    logprob_leaf_stats(p, v, row, tn * BN + half * 64, 2 * tn + half);
                 }
             }
         }
     epi_out:;
+      } else {
+        // 192-column tile: warp w reads TMEM lanes 32*(w%4).. and owns the 64
+        // columns of group (w-2)/4.  R holds this thread's 64 values of the
+        // working value, of a pending 2-leaf value, or of a stashed single
+        // leaf; the tree-walk replay checks that these never overlap.
+        const int ew = warp & 3;
+        const int grp = (warp - 2) >> 2;  // columns [64*grp, 64*grp+64)
+        const int rt = ew * 32 + lane;
+        const uint32_t tl = tmem_base + ((uint32_t)(ew * 32) << 16) + (uint32_t)(grp * 64);
+        // this warp's part of the 3-4 leaf slot in TMEM (groups 0, 1; group 2 uses shared memory)
+        const uint32_t tslot =
+            tmem_base + ((uint32_t)(ew * 32) << 16) + (grp == 0 ? Cfg::TMEM_SPARE0 : Cfg::TMEM_SPARE1);
+        float R[2][32];
+        uint32_t a = 0;
+        for (int u = pair; u < p.total_units; u += npairs) {
+            int tm, tn, f;
+            tc_decode(p, u, tm, tn, f);
+            const int n = p.nl[f];
+            const int row = tm * TC_PAIR_M + TC_BM * rank + rt;
+            const uint16_t* tab = leaf_tab + (n == p.tab_n[0] ? 0 : TC_TAB_MAX);
+            int gsp = 0;
+            for (int j = 0; j < n; ++j) {
+                const uint32_t buf = a & 1;
+                const uint32_t prev = buf ^ 1;  // accumulator of leaf j-1
+                if (warp == 2) mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim);
+                named_barrier_sync(TC_BAR_EPI, 32 * Cfg::EPI_WARPS);
+                if (*abort_flag) goto wepi_out;
+                ++a;
+                const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(p.seq ? seq_leaf_ops(n, j) : leaf_ops(n, j));
+                const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
+                const int nb = (code >> 3) & 31;
+                const int cls = (code >> 8) & 3;
+                const bool final_ = (code >> 10) & 1, c2p = (code >> 11) & 1, mp = (code >> 12) & 1;
+                const bool single = !final_ && cls == 0;
+                // A single leaf goes to R when R is free, else to the 3-4 leaf
+                // slot when that is free, else it stays in its accumulator and
+                // the next leaf pops it from there.
+                if (single && c2p && mp) continue;
+                tc_fence_after();
+                const uint32_t acc = tl + buf * Cfg::ACC_STRIDE;
+                const bool s_tm = p1 && c2p && mp;   // popped single in TMEM (accumulator prev)
+                const bool s_slot = p1 && c2p && !mp;  // popped single in the slot
+                if (single && c2p) {
+                    // park the single in the slot (TMEM spare columns or shared memory)
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t w[32];
+                        tmem_ld32_nowait(acc + cc * 32, w);
+                        tmem_wait_ld(w);
+                        if (grp < 2) {
+                            float f[32];
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) f[k] = __uint_as_float(w[k]);
+                            tmem_st32_nowait(tslot + cc * 32, f);
+                        } else {
+                            float f[32];
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) f[k] = __uint_as_float(w[k]);
+                            scratch_st(sSlot, cc, rt, f);
+                        }
+                    }
+                    if (grp < 2) tmem_wait_st();
+                } else if (s_tm || s_slot) {
+                    // R = R + (single + leaf), 16 columns at a time
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t l[16], sv[16];
+                        tmem_ld16_nowait(acc + q * 16, l);
+                        if (s_tm)
+                            tmem_ld16_nowait(tl + prev * Cfg::ACC_STRIDE + q * 16, sv);
+                        else if (grp < 2)
+                            tmem_ld16_nowait(tslot + q * 16, sv);
+                        else
+                            scratch_ld16(sSlot, q, rt, sv);
+                        tmem_wait_ld16(l);
+                        tie16(sv);
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            R[q >> 1][(q & 1) * 16 + k] = __fadd_rn(
+                                R[q >> 1][(q & 1) * 16 + k], __fadd_rn(__uint_as_float(sv[k]), __uint_as_float(l[k])));
+                    }
+                } else if (p1 || p2) {
+                    // R holds the left operand (a single or the 2-leaf value): R = R + leaf
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t l[32];
+                        tmem_ld32_nowait(acc + cc * 32, l);
+                        tmem_wait_ld(l);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) R[cc][k] = __fadd_rn(R[cc][k], __uint_as_float(l[k]));
+                    }
+                } else {
+                    // R = leaf (a single going to R, or a leaf whose pops are all below)
+                    uint32_t l[64];
+                    tmem_ld64_nowait(acc, l);
+                    tmem_wait_ld64(l);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        R[0][k] = __uint_as_float(l[k]);
+                        R[1][k] = __uint_as_float(l[32 + k]);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0 && !(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) {
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[buf]), 0));
+                    if (s_tm) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[prev]), 0));
+                }
+                if (single) continue;  // held in R or the slot until the next leaf
+                // Phase 2: the 3-4 leaf value, then the L2 stack from its top.
+                if (pm) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float w[32];
+                        if (grp < 2)
+                            tmem_ld32(tslot + cc * 32, w);
+                        else
+                            scratch_ld(sSlot, cc, rt, w);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) R[cc][k] = __fadd_rn(w[k], R[cc][k]);
+                    }
+                }
+                for (int i = 0; i < nb; ++i) {
+                    const float* sl = scratch_slot<BN>(p, gsp - 1 - i);
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        float w[32];
+                        scratch_ld(sl, grp * 2 + cc, rt, w);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) R[cc][k] = __fadd_rn(w[k], R[cc][k]);
+                    }
+                }
+                const int g_after = gsp - nb;
+                gsp = g_after + ((!final_ && cls == 3) ? 1 : 0);
+                if (!final_) {
+                    // a 2-leaf value stays in R
+                    if (cls == 2) {
+                        if (grp < 2) {
+#pragma unroll
+                            for (int cc = 0; cc < 2; ++cc) tmem_st32_nowait(tslot + cc * 32, R[cc]);
+                            tmem_wait_st();
+                        } else {
+#pragma unroll
+                            for (int cc = 0; cc < 2; ++cc) scratch_st(sSlot, cc, rt, R[cc]);
+                        }
+                    } else if (cls == 3) {
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) scratch_st(scratch_slot<BN>(p, g_after), grp * 2 + cc, rt, R[cc]);
+                    }
+                } else if (EPI == EPI_TREE && p.swiglu) {
+                    // gate features f0..f0+31 (R[0]) and their up values (R[1])
+                    if (row < p.M) {
+                        const int f0 = tn * (BN / 2) + grp * 32;
+                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                                              (size_t)row * (p.N / 2) + f0);
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            float o[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) o[e] = swiglu1(R[0][8 * q8 + e], R[1][8 * q8 + e]);
+                            if (f0 + 8 * q8 < p.N / 2) dst[q8] = pack8(o);
+                        }
+                    }
+                } else if (EPI != EPI_LOGPROB) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int col = tn * BN + (grp * 2 + cc) * 32;
+                        if (p.direct) {
+                            if (EPI == EPI_TREE_RES) add_residual32(p.residual, p.M, p.N, row, col, R[cc]);
+                            store_row32(p.out, p.out_bf16, p.M, p.N, row, col, R[cc]);
+                        } else
+                            store_row32(p.partials + (size_t)f * p.M * p.N, 0, p.M, p.N, row, col, R[cc]);
+                    }
+                } else {
+                    logprob_leaf_stats(p, R, row, tn * BN + grp * 64, (BN / 64) * tn + grp);
+                }
+            }
+        }
+    wepi_out:;
+      }
     }
 
     // A CTA that gave up tells its peer, so the peer's waits end too.

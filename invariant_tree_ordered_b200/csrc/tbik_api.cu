@@ -55,12 +55,13 @@ tbik_status device_info(int& dev, DeviceInfo*& info) {
     info = &d;
     if (!d.ok) return TBIK_ERR_UNSUPPORTED;
     if (!d.attrs_set) {
-        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TC_SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE_RES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TC_SMEM_BYTES) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_tc_kernel<EPI_LOGPROB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TC_SMEM_BYTES) != cudaSuccess)
+        const int s128 = (int)TcCfg<TC_BN>::SMEM_BYTES, s192 = (int)TcCfg<TC_BN_WIDE>::SMEM_BYTES;
+        const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        if (cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE, TC_BN>, attr, s128) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE_RES, TC_BN>, attr, s128) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE, TC_BN_WIDE>, attr, s192) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE_RES, TC_BN_WIDE>, attr, s192) != cudaSuccess ||
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_LOGPROB, TC_BN_WIDE>, attr, s192) != cudaSuccess)
             return TBIK_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -139,13 +140,21 @@ int a_box_rows(int M) { return M >= TC_BM ? TC_BM : ((M + 7) / 8) * 8; }
 
 // Ring of the tensor-core kernel: with a small A copy (small M) the same
 // shared memory holds more stages of B, i.e. more bytes in flight.
+template <int BN>
 void set_ring(TcParams& prm, int a_box) {
+    using Cfg = TcCfg<BN>;
     prm.a_box_rows = a_box;
     prm.a_slice = (uint32_t)a_box * 128u;
-    prm.stage_bytes = 2u * prm.a_slice + (uint32_t)TC_B_BYTES;
-    const int st = (int)(TC_RING_BYTES / prm.stage_bytes);
+    prm.stage_bytes = (uint32_t)Cfg::KSLICES * prm.a_slice + (uint32_t)Cfg::B_BYTES;
+    const int st = (int)(Cfg::RING_BYTES / prm.stage_bytes);
     prm.stages = st < TC_MAX_STAGES ? st : TC_MAX_STAGES;
 }
+
+// Pair-tile width of the tensor-core GEMM: 192 columns when B is [N,K]
+// (K-major; its TMA box of 96 rows has no swizzle-atom constraint), 128 when
+// B is [K,N].  It depends on the operand layout only, never on M, N or T.
+int tc_tile_n(bool b_nk) { return b_nk ? TC_BN_WIDE : TC_BN; }
+size_t tc_slot_bytes(int bn) { return (size_t)TC_BM * bn * sizeof(float); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -190,6 +199,7 @@ struct GemmPlan {
     int M = 0, N = 0, K = 0, T = 1, leaf = 1;
     int L = 0, D = 0, F = 1;
     int tiles_m = 0, tiles_n = 0, units = 0, grid = 0, gs = 0;
+    int bn = 0;  // output columns per tile (pair tile in TC mode)
     bool direct = true;
     std::vector<std::pair<int, int>> nodes;  // (first leaf, leaves) per frontier node
     int leaf_eff = 1;                        // K elements per leaf as launched
@@ -213,7 +223,8 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
     p.M = M, p.N = N, p.K = K, p.T = T, p.leaf = leaf;
     p.L = K / leaf;
     if (p.L % T) return TBIK_ERR_SHAPE;
-    const int bm = tc ? TC_PAIR_M : EX_BM, bn = tc ? TC_BN : EX_BN;
+    const int bm = tc ? TC_PAIR_M : EX_BM, bn = tc ? tc_tile_n(p.b_nk) : EX_BN;
+    p.bn = bn;
     if (tc) {
         if (N % 8 || K % 8) return TBIK_ERR_SHAPE;
         if (p.noninv ? (K / T) % 16 : leaf % 16) return TBIK_ERR_SHAPE;
@@ -273,7 +284,7 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
     }
     if (tc && p.gs > 0) {
         p.off_scratch = off;
-        off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
+        off = align256(off + (size_t)p.grid * p.gs * tc_slot_bytes(bn));
     }
     p.fused = p.swiglu && tc && p.direct;
     if (p.swiglu && !p.fused) {  // fp32 gate/up roots, then the SwiGLU kernel
@@ -353,12 +364,16 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         CUtensorMap ta, tb;
         const int a_box = a_box_rows(p.M);
         if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
-        bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, 64, TC_BN / 2)
-                          : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, TC_BN / 2, 64);
+        const bool wide = p.bn == TC_BN_WIDE;  // B is [N,K]
+        bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, 64, (uint32_t)p.bn / 2)
+                          : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, (uint32_t)p.bn / 2, 64);
         if (!okb) return TBIK_ERR_CUDA;
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
-        set_ring(prm, a_box);
+        if (wide)
+            set_ring<TC_BN_WIDE>(prm, a_box);
+        else
+            set_ring<TC_BN>(prm, a_box);
         prm.M = p.M, prm.N = p.N, prm.K = p.K;
         prm.leaf = p.leaf_eff;
         prm.F = p.F;
@@ -381,10 +396,16 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
             prm.nl[f] = (short)p.nodes[f].second;
             if (prm.nl[f] != prm.tab_n[0]) prm.tab_n[1] = prm.nl[f];
         }
-        if (prm.residual)
-            gemm_tc_kernel<EPI_TREE_RES><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+        using W = TcCfg<TC_BN_WIDE>;
+        using Nw = TcCfg<TC_BN>;
+        if (wide && prm.residual)
+            gemm_tc_kernel<EPI_TREE_RES, TC_BN_WIDE><<<p.grid, W::THREADS, W::SMEM_BYTES, s>>>(ta, tb, prm);
+        else if (wide)
+            gemm_tc_kernel<EPI_TREE, TC_BN_WIDE><<<p.grid, W::THREADS, W::SMEM_BYTES, s>>>(ta, tb, prm);
+        else if (prm.residual)
+            gemm_tc_kernel<EPI_TREE_RES, TC_BN><<<p.grid, Nw::THREADS, Nw::SMEM_BYTES, s>>>(ta, tb, prm);
         else
-            gemm_tc_kernel<EPI_TREE><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+            gemm_tc_kernel<EPI_TREE, TC_BN><<<p.grid, Nw::THREADS, Nw::SMEM_BYTES, s>>>(ta, tb, prm);
     } else {
         ExParams prm;
         memset(&prm, 0, sizeof(prm));
@@ -473,7 +494,7 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
         p.Lv = p.Vpad / VLEAF;
     }
     p.nvl = (V + VLEAF - 1) / VLEAF;        // vocab leaves holding columns
-    p.nvt = (V + TC_BN - 1) / TC_BN;        // 128-column GEMM tiles (two vocab leaves each)
+    p.nvt = (V + TC_BN_WIDE - 1) / TC_BN_WIDE;  // 192-column GEMM tiles (three vocab leaves each)
     // The baseline's logits: T chains over H/T each, summed left to right.
     if (p.noninv && (H % T || (tc && (H / T) % 16))) return TBIK_ERR_SHAPE;
     p.Lk = p.noninv ? T : H / leaf;
@@ -497,7 +518,7 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
     off = align256(off + (size_t)T * M * 2 * sizeof(float));
     if (tc && p.gs > 0) {
         p.off_scratch = off;
-        off = align256(off + (size_t)p.grid * p.gs * TC_SLOT_FLOATS * sizeof(float));
+        off = align256(off + (size_t)p.grid * p.gs * tc_slot_bytes(TC_BN_WIDE));
     }
     if (p.part) {  // which rows' targets fall in this shard
         p.off_zflag = off;
@@ -533,10 +554,10 @@ tbik_status run_logprob(const LogprobPlan& p, const uint16_t* hidden, const uint
         CUtensorMap ta, tb;
         const int a_box = a_box_rows(M);
         if (!make_map(&ta, hidden, (uint64_t)H, (uint64_t)M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
-        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, 64, TC_BN / 2)) return TBIK_ERR_CUDA;
+        if (!make_map(&tb, W, (uint64_t)H, (uint64_t)V, 64, TC_BN_WIDE / 2)) return TBIK_ERR_CUDA;
         TcParams prm;
         memset(&prm, 0, sizeof(prm));
-        set_ring(prm, a_box);
+        set_ring<TC_BN_WIDE>(prm, a_box);
         prm.M = M, prm.N = V, prm.K = H;
         prm.leaf = p.noninv ? H / T : leaf;
         prm.seq = p.noninv ? 1 : 0;
@@ -559,7 +580,8 @@ tbik_status run_logprob(const LogprobPlan& p, const uint16_t* hidden, const uint
         prm.lo[0] = 0;
         prm.nl[0] = (short)p.Lk;
         prm.tab_n[0] = prm.tab_n[1] = prm.nl[0];
-        gemm_tc_kernel<EPI_LOGPROB><<<p.grid, TC_THREADS, TC_SMEM_BYTES, s>>>(ta, tb, prm);
+        gemm_tc_kernel<EPI_LOGPROB, TC_BN_WIDE>
+            <<<p.grid, TcCfg<TC_BN_WIDE>::THREADS, TcCfg<TC_BN_WIDE>::SMEM_BYTES, s>>>(ta, tb, prm);
         if ((st = launch_status()) != TBIK_OK) return st;
     } else if (V > 0) {
         float* z = reinterpret_cast<float*>(w8 + p.off_z);

@@ -17,25 +17,27 @@ from tests.gpu_util import dev_bf16, host_f32, u32  # noqa: E402
 import invariant_tree_ordered_b200 as tbik  # noqa: E402
 
 
-def test_withheld_arrive_times_out_and_context_survives():
-    # 148 output tiles, 16 leaves each: every CTA streams more than two leaves,
-    # so the MMA issuer has to wait for a drained accumulator.
+@pytest.mark.parametrize("b_nk", [False, True])  # the 128- and 192-column tile kernels
+def test_withheld_arrive_times_out_and_context_survives(b_nk):
+    # 148 (99) output tiles, 16 leaves each: every CTA streams more than two
+    # leaves, so the MMA issuer has to wait for a drained accumulator.
     M, N, K, leaf = 128, 128 * 148, 256, 16
     a = dev_bf16(synth.normal_bf16(400, (M, K)))
-    b = dev_bf16(synth.normal_bf16(401, (K, N), std=0.05))
-    good = host_f32(tbik.gemm(a, b, T=1, leaf=leaf, tc=True))
+    bh = synth.normal_bf16(401, (K, N), std=0.05)
+    b = dev_bf16(np.ascontiguousarray(bh.T) if b_nk else bh)
+    good = host_f32(tbik.gemm(a, b, T=1, leaf=leaf, tc=True, b_nk=b_nk))
     assert tbik.get_error() == tbik.TBIK_OK
     try:
         tbik.debug_set(tbik.DEBUG_WITHHOLD_ACC_ARRIVE, 50_000_000)  # 50 ms per wait
         t0 = time.time()
-        tbik.gemm(a, b, T=1, leaf=leaf, tc=True)
+        tbik.gemm(a, b, T=1, leaf=leaf, tc=True, b_nk=b_nk)
         status = tbik.get_error()
         elapsed = time.time() - t0
     finally:
         tbik.debug_set(0, 0)
     assert status == tbik.TBIK_ERR_TIMEOUT
     assert elapsed < 10.0
-    again = host_f32(tbik.gemm(a, b, T=1, leaf=leaf, tc=True))
+    again = host_f32(tbik.gemm(a, b, T=1, leaf=leaf, tc=True, b_nk=b_nk))
     assert tbik.get_error() == tbik.TBIK_OK
     assert np.array_equal(u32(again), u32(good))
     assert torch.cuda.synchronize() is None

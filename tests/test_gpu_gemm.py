@@ -186,6 +186,22 @@ def test_down_proj_tc_invariance_over_T_and_M(down_proj):
     assert rel_frob(full[1][rows], c64) <= 2e-5
 
 
+def test_down_proj_tile_widths_agree_bitwise(down_proj):
+    """The [N,K] operand runs the 192-column tile kernel (two TMEM accumulators,
+    the pending 2-leaf value in registers, a split 3-4 leaf slot), the [K,N]
+    operand the 128-column one (three accumulators, TMEM and shared-memory
+    slots): different storage plans for the same 56-leaf tree.  Both must give
+    the same bits, at T = 1 and T = 8 and for a shifted batch."""
+    a, b = down_proj
+    bt = np.ascontiguousarray(b.T)
+    for T in (1, 8):
+        kn = run(a, b, T=T, leaf=256, tc=True)
+        nk = run(a, bt, T=T, leaf=256, tc=True, b_nk=True)
+        assert np.array_equal(u32(kn), u32(nk)), T
+    sub = run(a[7:300], bt, T=2, leaf=256, tc=True, b_nk=True)
+    assert np.array_equal(u32(sub), u32(kn[7:300]))
+
+
 def test_down_proj_exact_sampled_rows_full_M(down_proj):
     """64 seeded rows (tile edges included) of the exact-mode 4096-row launch at
     T = 8, bit-exact to the oracle."""

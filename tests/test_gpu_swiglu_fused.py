@@ -48,20 +48,23 @@ def test_fused_exact_bitwise_vs_oracle(M, K, F, leaf, b_nk):
 
 
 @pytest.mark.parametrize("M", [16, 1024])  # 16: frontier-split (unfused) path; 1024: fused epilogue
-def test_fused_tc_equals_tc_roots_then_swiglu(M):
+@pytest.mark.parametrize("b_nk", [False, True])  # 128-column tiles; 192-column tiles (ragged last tile)
+def test_fused_tc_equals_tc_roots_then_swiglu(M, b_nk):
     K, F = 2048, 2048
     a = dev_bf16(synth.normal_bf16(720, (M, K)))
     wg, wu = weights(730, K, F)
-    b = dev_bf16(interleave_gate_up(wg, wu))
-    fused = host_bits16(tbik.gemm(a, b, T=1, leaf=256, tc=True, swiglu=True))
-    roots = host_f32(tbik.gemm(a, b, T=1, leaf=256, tc=True))
+    bh = interleave_gate_up(wg, wu)
+    b = dev_bf16(np.ascontiguousarray(bh.T) if b_nk else bh)
+    fused = host_bits16(tbik.gemm(a, b, T=1, leaf=256, tc=True, swiglu=True, b_nk=b_nk))
+    roots = host_f32(tbik.gemm(a, b, T=1, leaf=256, tc=True, b_nk=b_nk))
     g, u = split_roots(roots, F)
     _, _, sep = tbik.rope_swiglu(g=dev_f32(g), u=dev_f32(u))
     assert np.array_equal(fused, host_bits16(sep))
     for T in (2, 8):
-        assert np.array_equal(host_bits16(tbik.gemm(a, b, T=T, leaf=256, tc=True, swiglu=True)), fused), T
+        assert np.array_equal(host_bits16(tbik.gemm(a, b, T=T, leaf=256, tc=True, swiglu=True, b_nk=b_nk)),
+                              fused), T
     if M > 1:
-        part = host_bits16(tbik.gemm(a[3:M - 2].contiguous(), b, T=4, leaf=256, tc=True, swiglu=True))
+        part = host_bits16(tbik.gemm(a[3:M - 2].contiguous(), b, T=4, leaf=256, tc=True, swiglu=True, b_nk=b_nk))
         assert np.array_equal(part, fused[3:M - 2])
     assert tbik.get_error() == tbik.TBIK_OK
 

@@ -92,7 +92,7 @@ def test_noalloc_refuses_arguments_beyond_its_scratch():
     V, H, leaf, T = 151936, 4096, 256, 8
     m_max = _largest_fitting_rows(lib, V, H, T, leaf)
     if torch.cuda.get_device_properties(0).multi_processor_count == 148:
-        assert m_max == 1251  # the limit stated in tbik.h for the 151936 x 4096 lm_head
+        assert m_max == 997  # the limit stated in tbik.h for the 151936 x 4096 lm_head
     big = m_max + 1
     # The size check comes before any pointer is used: small stand-in buffers.
     dummy = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
