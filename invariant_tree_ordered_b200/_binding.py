@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             "tbik_logprob_workspace": (sz, [i32, i32, i32, i32, i32, u32]),
             "tbik_logprob": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, u32, vp, sz, vp]),
             "tbik_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
+            "tbik_attention_tc_workspace": (sz, [i32, i32, i32, i32, i32]),
+            "tbik_attention_tc": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, sz, vp]),
             "tbik_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp]),
             "tbik_transpose": (i32, [vp, vp, i32, i32, vp]),
             "tbik_tree_combine": (i32, [vp, vp, ctypes.c_longlong, i32, u32, vp, vp]),
@@ -300,9 +302,18 @@ def rope_swiglu(*, q=None, k=None, pos=None, table=None, q_out=None, k_out=None,
     return q_out, k_out, out
 
 
-def attention(q, k, v, *, out=None, chunk: int = 64, stream=None):
-    """Causal attention with the key reduction in tree order (see tbik_attention);
-    q, k, v bf16 [batch, seq, heads, head_dim]."""
+def attention_tc_workspace(batch, seq, heads, head_dim, chunk=64) -> int:
+    n = load_library().tbik_attention_tc_workspace(batch, seq, heads, head_dim, chunk)
+    if n == (1 << 64) - 1:
+        raise TbikError(TBIK_ERR_SHAPE, "tbik_attention_tc_workspace: unsupported shape")
+    return n
+
+
+def attention(q, k, v, *, out=None, chunk: int = 64, tc: bool = False, workspace=None, stream=None):
+    """Causal attention with the key reduction in tree order; q, k, v bf16
+    [batch, seq, heads, head_dim].  tc=False: tbik_attention (exact order on
+    the CUDA cores); tc=True: tbik_attention_tc (tensor cores; a workspace is
+    allocated when none is given)."""
     torch = _torch()
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -313,8 +324,16 @@ def attention(q, k, v, *, out=None, chunk: int = 64, stream=None):
     if out is None:
         out = torch.empty_like(q)
     _need_out(out, torch.bfloat16, q.shape)
-    _check(lib.tbik_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, NH, D, chunk, _stream_handle(stream)),
-           "tbik_attention")
+    if not tc:
+        _check(lib.tbik_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, NH, D, chunk, _stream_handle(stream)),
+               "tbik_attention")
+        return out
+    need = attention_tc_workspace(B, S, NH, D, chunk)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wsp, wsn = (_ptr(workspace), workspace.numel() * workspace.element_size()) if workspace is not None else (None, 0)
+    _check(lib.tbik_attention_tc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, S, NH, D, chunk, wsp, wsn,
+                                 _stream_handle(stream)), "tbik_attention_tc")
     return out
 
 

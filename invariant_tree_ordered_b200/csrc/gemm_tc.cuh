@@ -525,10 +525,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
                 const uint32_t buf = a % 3;
                 const uint32_t prev = (a + 2) % 3;  // accumulator of leaf j-1 (a retained single leaf)
                 // One warp polls the accumulator barrier; the other epilogue
-                // warps wait on a hardware barrier, so nothing else polls.
-                if (warp == 2) mbar_wait(&acc_full[buf], (a / 3) & 1, abort_flag, wait_lim);
-                named_barrier_sync(TC_BAR_EPI, 32 * Cfg::EPI_WARPS);
-                if (*abort_flag) goto epi_out;
+                // warps wait on a hardware barrier, so nothing else polls.  The
+                // barrier's OR reduction makes the decision to give up common
+                // to all epilogue warps.
+                bool ok = true;
+                if (warp == 2) ok = mbar_wait(&acc_full[buf], (a / 3) & 1, abort_flag, wait_lim);
+                if (named_barrier_or(TC_BAR_EPI, 32 * Cfg::EPI_WARPS, !ok || *abort_flag != 0)) goto epi_out;
                 ++a;
                 const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(p.seq ? seq_leaf_ops(n, j) : leaf_ops(n, j));
                 const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
@@ -663,9 +665,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
             for (int j = 0; j < n; ++j) {
                 const uint32_t buf = a & 1;
                 const uint32_t prev = buf ^ 1;  // accumulator of leaf j-1
-                if (warp == 2) mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim);
-                named_barrier_sync(TC_BAR_EPI, 32 * Cfg::EPI_WARPS);
-                if (*abort_flag) goto wepi_out;
+                bool ok = true;  // as in the 128-column epilogue: one poller, a common decision
+                if (warp == 2) ok = mbar_wait(&acc_full[buf], (a >> 1) & 1, abort_flag, wait_lim);
+                if (named_barrier_or(TC_BAR_EPI, 32 * Cfg::EPI_WARPS, !ok || *abort_flag != 0)) goto wepi_out;
                 ++a;
                 const uint32_t code = use_tab ? tab[j] : encode_leaf_ops(p.seq ? seq_leaf_ops(n, j) : leaf_ops(n, j));
                 const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;

@@ -14,6 +14,7 @@
 #include "device_common.cuh"
 #include "gemm_exact.cuh"
 #include "gemm_tc.cuh"
+#include "attention_tc.cuh"
 #include "logprob.cuh"
 #include "attention.cuh"
 #include "reduce.cuh"
@@ -61,7 +62,8 @@ tbik_status device_info(int& dev, DeviceInfo*& info) {
             cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE_RES, TC_BN>, attr, s128) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE, TC_BN_WIDE>, attr, s192) != cudaSuccess ||
             cudaFuncSetAttribute(gemm_tc_kernel<EPI_TREE_RES, TC_BN_WIDE>, attr, s192) != cudaSuccess ||
-            cudaFuncSetAttribute(gemm_tc_kernel<EPI_LOGPROB, TC_BN_WIDE>, attr, s192) != cudaSuccess)
+            cudaFuncSetAttribute(gemm_tc_kernel<EPI_LOGPROB, TC_BN_WIDE>, attr, s192) != cudaSuccess ||
+            cudaFuncSetAttribute(attention_tc_kernel, attr, (int)ATC_SMEM_BYTES) != cudaSuccess)
             return TBIK_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -98,6 +100,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 [batch][seq][heads][head_dim] tensor (head_dim contiguous) as a 4-D map
+// {head_dim, heads, seq, batch}; box = 64 dims x 1 head x `rows` positions x 1
+// batch, 128-byte swizzle, zero OOB fill.
+bool make_map_bshd(CUtensorMap* m, const void* base, int batch, int seq, int heads, int hd, uint32_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)hd, (cuuint64_t)heads, (cuuint64_t)seq, (cuuint64_t)batch};
+    cuuint64_t strides[3] = {(cuuint64_t)hd * 2, (cuuint64_t)heads * hd * 2, (cuuint64_t)seq * heads * hd * 2};
+    cuuint32_t box[4] = {64, 1, rows, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -747,6 +764,72 @@ tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const uint16_t*
         attention_kernel<4><<<(int)blocks, ATT_WARPS * 32, 0, s>>>(q, k, v, out, batch, seq, heads, scale);
     else
         attention_kernel<2><<<(int)blocks, ATT_WARPS * 32, 0, s>>>(q, k, v, out, batch, seq, heads, scale);
+    return launch_status();
+}
+
+// Tensor-core mode of the attention: shapes, grid and scratch.
+struct AttTcPlan {
+    int tiles = 0, grid = 0, gs = 0;
+    size_t bytes = 0;
+};
+
+tbik_status plan_attention_tc(int batch, int seq, int heads, int head_dim, int chunk, int sms, AttTcPlan& p) {
+    if (batch < 0 || seq < 0 || heads <= 0) return TBIK_ERR_ARG;
+    if (head_dim != ATC_HD || chunk != ATC_CH || seq % ATC_BM || seq > 256 * ATC_CH) return TBIK_ERR_SHAPE;
+    const long long tiles = (long long)batch * heads * (seq / ATC_BM);
+    if (tiles > 0x7fffffffLL) return TBIK_ERR_SHAPE;
+    p.tiles = (int)tiles;
+    p.grid = p.tiles < sms ? p.tiles : sms;
+    // the deepest L2 stack over the chunk trees of every row length
+    p.gs = 0;
+    for (int n = 1; n <= seq / ATC_CH; ++n) {
+        const int g = max_big_pending(n);
+        if (g > p.gs) p.gs = g;
+    }
+    p.bytes = (size_t)p.grid * p.gs * (ATC_VAL_FLOATS + 2 * ATC_BM) * sizeof(float);
+    return TBIK_OK;
+}
+
+size_t tbik_attention_tc_workspace(int batch, int seq, int heads, int head_dim, int chunk) {
+    int dev;
+    DeviceInfo* info;
+    if (device_info(dev, info) != TBIK_OK) return (size_t)-1;
+    AttTcPlan p;
+    if (plan_attention_tc(batch, seq, heads, head_dim, chunk, info->sms, p) != TBIK_OK) return (size_t)-1;
+    return p.bytes;
+}
+
+tbik_status tbik_attention_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int batch,
+                              int seq, int heads, int head_dim, int chunk, void* workspace, size_t ws_bytes,
+                              void* stream) {
+    int dev;
+    DeviceInfo* info;
+    tbik_status st = device_info(dev, info);
+    if (st != TBIK_OK) return st;
+    AttTcPlan p;
+    if ((st = plan_attention_tc(batch, seq, heads, head_dim, chunk, info->sms, p)) != TBIK_OK) return st;
+    if (p.tiles == 0) return TBIK_OK;
+    if (!q || !k || !v || !out) return TBIK_ERR_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return TBIK_ERR_ALIGN;
+    if (p.bytes > 0 && (!workspace || ws_bytes < p.bytes)) return TBIK_ERR_WORKSPACE;
+    if (p.bytes > 0 && !aligned16(workspace)) return TBIK_ERR_ALIGN;
+    CUtensorMap tq, tk, tv;
+    if (!make_map_bshd(&tq, q, batch, seq, heads, head_dim, ATC_BM) ||
+        !make_map_bshd(&tk, k, batch, seq, heads, head_dim, ATC_CH) ||
+        !make_map_bshd(&tv, v, batch, seq, heads, head_dim, ATC_CH))
+        return TBIK_ERR_CUDA;
+    AttTcParams prm;
+    memset(&prm, 0, sizeof(prm));
+    prm.batch = batch, prm.seq = seq, prm.heads = heads;
+    prm.ntq = seq / ATC_BM;
+    prm.tiles = p.tiles;
+    prm.scale = (float)(1.0 / std::sqrt((double)head_dim));
+    prm.out = out;
+    prm.stack = reinterpret_cast<float*>(workspace);
+    prm.gs = p.gs;
+    prm.wait_cycles = wait_cycles(info);
+    attention_tc_kernel<<<p.grid, ATC_THREADS, ATC_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv,
+                                                                                                           prm);
     return launch_status();
 }
 

@@ -51,7 +51,7 @@ class Decoder:
         return self._tables[key]
 
     def forward(self, ids, targets, pos, *, T: int = 1, tc: bool = True, noninv: bool = False,
-                fuse_residual: bool = False, stream=None):
+                fuse_residual: bool = False, attention_tc: bool = False, stream=None):
         """ids, targets: device int32 [batch, seq]; pos: device int32 [batch*seq]
         (the position of each token).  Returns fp32 logprobs [batch, seq].
 
@@ -59,7 +59,10 @@ class Decoder:
         bf16 residual stream h in their last step (tbik_gemm_residual, one
         rounding: h = bf16(root + h)) and each RMSNorm normalises h with no
         residual input; otherwise the projection output is rounded to bf16
-        and the RMSNorm adds it to the residual in fp32."""
+        and the RMSNorm adds it to the residual in fp32.
+
+        attention_tc: the attention on the tensor cores (tbik_attention_tc,
+        head_dim 128, seq a multiple of 128); otherwise the exact-order kernel."""
         torch = tb._torch()
         c = self.cfg
         B, S = ids.shape
@@ -95,7 +98,7 @@ class Decoder:
             q3, k3 = q.view(n, c.heads, c.head_dim), k.view(n, c.heads, c.head_dim)
             tb.rope_swiglu(q=q3, k=k3, pos=pos, table=table, q_out=q3, k_out=k3, stream=stream)
             o = tb.attention(q.view(B, S, c.heads, c.head_dim), k.view(B, S, c.heads, c.head_dim),
-                             v.view(B, S, c.heads, c.head_dim), stream=stream)
+                             v.view(B, S, c.heads, c.head_dim), tc=attention_tc, stream=stream)
             y, res = add_norm(L["wo"], o.view(n, c.d), c.leaf, res)
             act = torch.empty((n, c.ffn), dtype=bf, device=dev)
             tb.gemm(y, L["wgu"], T=1, leaf=c.leaf, tc=tc, swiglu=True, out=act, stream=stream)

@@ -1,0 +1,99 @@
+"""Tensor-core mode of the tree-ordered causal attention (tbik_attention_tc).
+
+Not bit-exact to the oracle (the dot products run on the tensor cores and the
+softmax weights are rounded to bf16 before P V), so it is checked against the
+binary64 definition with a bound derived from that arithmetic:
+  the weights of a row are p_j rounded to bf16 (relative error <= 2^-9) and
+  the sum s uses the same rounded weights, so the output is an exact weighted
+  average of the v_j with each normalised weight moved by at most about
+  2 * 2^-9 of itself: |o/s - exact| <= 2^-8 * max_j |v_j - exact| <= 2^-7 * max|v|;
+  the output rounding to bf16 adds 2^-9 |out| (2^-8 here, with margin); the
+  fp32 score and combine arithmetic is orders of magnitude below these.
+It must also be bitwise independent of the batch composition and of how the
+heads are split, and agree with the exact mode to the same bound.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+from tests.gpu_util import dev_bf16, host_bits16  # noqa: E402
+
+import invariant_tree_ordered_b200 as tbik  # noqa: E402
+
+
+def qkv(seed, shape, std=1.0):
+    return [synth.normal_bf16(seed + i, shape, std=std) for i in range(3)]
+
+
+def f32(bits16):
+    return (np.asarray(bits16).astype(np.uint32) << 16).view(np.float32)
+
+
+def within_bound(got, ref, v):
+    vmax = float(np.abs(f32(v)).max())
+    return np.abs(got - ref) <= 2.0 ** -7 * vmax + 2.0 ** -8 * np.abs(ref)
+
+
+@pytest.mark.parametrize("B,S,NH", [(1, 128, 1), (2, 256, 3), (1, 1024, 2), (1, 2048, 1)])
+def test_tc_attention_vs_binary64(B, S, NH):
+    # 1024 and 2048 positions: 16 and 32 chunks, so pending summaries reach the L2 stack
+    q, k, v = qkv(500 + S, (B, S, NH, 128))
+    got = f32(host_bits16(tbik.attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), tc=True)))
+    assert tbik.get_error() == tbik.TBIK_OK
+    ref = oracle.attention_f64(q, k, v)
+    assert np.all(np.isfinite(got))
+    assert np.all(within_bound(got, ref, v))
+    assert float(np.mean(np.abs(got - ref))) <= 1e-3
+    exact = f32(oracle.attention(q, k, v, chunk=64))
+    assert np.all(within_bound(got, exact, v))
+
+
+def test_tc_attention_large_scores():
+    # std-4 queries and keys: a wide score range, so the chunk maxima and the
+    # exp(m - M) factors of the tree combine matter
+    q, k, v = qkv(530, (2, 384, 2, 128), std=4.0)
+    got = f32(host_bits16(tbik.attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), tc=True)))
+    ref = oracle.attention_f64(q, k, v)
+    assert np.all(np.isfinite(got)) and np.all(within_bound(got, ref, v))
+
+
+def test_tc_attention_batch_and_head_split_invariance():
+    B, S, NH = 3, 512, 4
+    q, k, v = (dev_bf16(a) for a in qkv(540, (B, S, NH, 128)))
+    full = host_bits16(tbik.attention(q, k, v, tc=True))
+    one = host_bits16(tbik.attention(q[1:2].contiguous(), k[1:2].contiguous(), v[1:2].contiguous(), tc=True))
+    assert np.array_equal(one[0], full[1])
+    for T in (2, 4):
+        w = NH // T
+        for t in range(T):
+            sl = slice(t * w, (t + 1) * w)
+            part = host_bits16(tbik.attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(),
+                                              v[:, :, sl].contiguous(), tc=True))
+            assert np.array_equal(part, full[:, :, sl]), (T, t)
+    perm = [2, 0, 1]
+    shuf = host_bits16(tbik.attention(q[perm].contiguous(), k[perm].contiguous(), v[perm].contiguous(), tc=True))
+    assert np.array_equal(shuf, full[perm])
+    assert tbik.get_error() == tbik.TBIK_OK
+
+
+def test_tc_attention_argument_errors():
+    lib = tbik.load_library()
+    s = torch.cuda.current_stream().cuda_stream
+    x = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
+    p = x.data_ptr()
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 200, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_SHAPE  # seq % 128
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 64, 64, None, 0, s) == tbik.TBIK_ERR_SHAPE   # head_dim
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 128, 32, None, 0, s) == tbik.TBIK_ERR_SHAPE  # chunk
+    assert lib.tbik_attention_tc(p + 2, p, p, p, 1, 256, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_ALIGN
+    assert lib.tbik_attention_tc_workspace(1, 200, 2, 128, 64) == (1 << 64) - 1
+    need = lib.tbik_attention_tc_workspace(1, 2048, 2, 128, 64)
+    assert need > 0  # 32 chunks: the tree has pending values of >= 5 chunks
+    big = torch.zeros((1, 2048, 2, 128), dtype=torch.bfloat16, device="cuda")
+    b = big.data_ptr()
+    assert lib.tbik_attention_tc(b, b, b, b, 1, 2048, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_WORKSPACE
+    assert tbik.get_error() == tbik.TBIK_OK

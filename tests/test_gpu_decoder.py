@@ -108,6 +108,23 @@ def test_full_config_tc_invariant_over_T_and_batch(full):
     assert tbik.get_error() == tbik.TBIK_OK
 
 
+def test_full_config_tc_attention_invariant_and_close(full):
+    """The attention on the tensor cores (tbik_attention_tc): the decoder stays
+    bitwise identical across T and batch compositions, and its logprobs stay
+    close to those with the exact-order attention (the per-layer bf16
+    activations differ by about one rounding, 2^-8 relative)."""
+    cfg, dec, ids, tg = full
+    base = run(dec, ids, tg, T=1, tc=True, attention_tc=True)
+    assert np.all(np.isfinite(base))
+    for T in (2, 8):
+        assert np.array_equal(u32(run(dec, ids, tg, T=T, tc=True, attention_tc=True)), u32(base)), T
+    sub = run(dec, ids[[5, 2]].copy(), tg[[5, 2]].copy(), T=4, tc=True, attention_tc=True)
+    assert np.array_equal(u32(sub), u32(base[[5, 2]]))
+    ref = run(dec, ids, tg, T=1, tc=True)
+    assert float(np.mean(np.abs(base - ref))) < 2e-2
+    assert tbik.get_error() == tbik.TBIK_OK
+
+
 def test_full_config_noninv_baseline_diverges_over_T(full):
     cfg, dec, ids, tg = full
     outs = {T: run(dec, ids, tg, T=T, tc=True, noninv=True) for T in (1, 2, 4, 8)}
