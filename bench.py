@@ -61,8 +61,8 @@ def parse():
     ap.add_argument("--impl", default="tbik", choices=["tbik", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decoder", action="store_true", help="skip the end-to-end decoder component")
-    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "gemm-exact", "attention", "swiglu",
-                                               "rmsnorm"],
+    ap.add_argument("--profile-case", choices=["logprob", "gemm", "gemm-t8", "gemm-exact", "attention",
+                                               "attention-tc", "swiglu", "rmsnorm"],
                     default=None,
                     help="run only one call of the path, `--steps` times, for ncu captures (no JSON line)")
     ap.add_argument("--tokens", type=int, default=M_TOK, help="tokens per call in --profile-case")
@@ -580,8 +580,9 @@ def decoder_component(dev, stream):
     """The end-to-end decoder (4 layers, d 2048, 16 heads of 128, ffn 5632,
     vocab 32000, batch 8 x seq 2048): forward + target logprobs in tensor-core
     mode at T = 1 (tokens/s, CUDA events), the same with the residual add fused
-    into the o and down projections, the attention kernel alone, the bitwise
-    checks against T = 8, and the non-invariant baseline's divergence."""
+    into the o and down projections, the same with the attention on the tensor
+    cores, the attention kernels alone (exact order and tensor cores), the
+    bitwise checks against T = 8, and the non-invariant baseline's divergence."""
     import torch
 
     import invariant_tree_ordered_b200 as tbik
@@ -621,6 +622,14 @@ def decoder_component(dev, stream):
     b.record(stream)
     torch.cuda.synchronize()
     ms_fused = a.elapsed_time(b) / n
+    tca = fwd(T=1, tc=True, attention_tc=True)  # attention on the tensor cores
+    a.record(stream)
+    for _ in range(n):
+        fwd(T=1, tc=True, attention_tc=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_tca = a.elapsed_time(b) / n
+    tca8 = fwd(T=8, tc=True, attention_tc=True)
     fused8 = fwd(T=8, tc=True, fuse_residual=True)
     t8 = fwd(T=8, tc=True)
     non1, non8 = fwd(T=1, tc=True, noninv=True), fwd(T=8, tc=True, noninv=True)
@@ -633,6 +642,16 @@ def decoder_component(dev, stream):
     b.record(stream)
     torch.cuda.synchronize()
     att_ms = a.elapsed_time(b) / n
+    aws = torch.empty(tbik.attention_tc_workspace(B, S, cfg["heads"], cfg["head_dim"]), dtype=torch.uint8,
+                      device=dev)
+    tbik.attention(q, q, q, tc=True, workspace=aws, stream=stream)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        tbik.attention(q, q, q, tc=True, workspace=aws, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    att_tc_ms = a.elapsed_time(b) / n
     att_flop = 4.0 * B * cfg["heads"] * cfg["head_dim"] * (S * (S + 1) / 2)
     status = tbik.get_error(stream)
     return {"workload": "4 layers, d 2048, 16x128 heads, ffn 5632, vocab 32000, batch 8 x seq 2048, TC, T=1",
@@ -642,6 +661,11 @@ def decoder_component(dev, stream):
             "fused_residual_bitwise_T1_vs_T8": bool(torch.equal(fused.view(torch.int32), fused8.view(torch.int32))),
             "noninv_max_abs_dlogprob_T8_vs_T1": float((non8 - non1).abs().max()),
             "attention_ms_per_layer": att_ms, "attention_tflops": att_flop / (att_ms * 1e-3) / 1e12,
+            "tc_attention": {"tokens_per_s": B * S / (ms_tca * 1e-3), "ms_per_forward": ms_tca,
+                             "bitwise_T1_vs_T8": bool(torch.equal(tca.view(torch.int32), tca8.view(torch.int32))),
+                             "mean_abs_dlogprob_vs_exact_attention": float((tca - base).abs().mean()),
+                             "attention_ms_per_layer": att_tc_ms,
+                             "attention_tflops": att_flop / (att_tc_ms * 1e-3) / 1e12},
             "status": int(status)}
 
 
@@ -653,13 +677,17 @@ def run_profile_case(args):
 
     dev = torch.device("cuda", 0)
     M = args.tokens
-    if args.profile_case == "attention":
+    if args.profile_case in ("attention", "attention-tc"):
         # decoder attention: sequences of 2048 positions, 16 heads of 128; --tokens = batch * 2048
         S, NH, D = 2048, 16, 128
         Bq = max(1, M // S)
         qkv = [synth.as_torch_bf16(synth.normal_bf16(450 + i, (Bq, S, NH, D))).to(dev) for i in range(3)]
         out = torch.empty_like(qkv[0])
-        call = lambda: tbik.attention(*qkv, out=out)  # noqa: E731
+        if args.profile_case == "attention":
+            call = lambda: tbik.attention(*qkv, out=out)  # noqa: E731
+        else:
+            aws = torch.empty(tbik.attention_tc_workspace(Bq, S, NH, D), dtype=torch.uint8, device=dev)
+            call = lambda: tbik.attention(*qkv, out=out, tc=True, workspace=aws)  # noqa: E731
     elif args.profile_case in ("swiglu", "rmsnorm"):
         d = synth.reduction_inputs(M, F=F)
         t = {k: synth.as_torch_bf16(d[k]).to(dev) for k in ("x", "res", "gamma", "g", "u")}
