@@ -592,12 +592,14 @@ def decoder_component(dev, stream):
     w = synth.decoder_weights(cfg)
     up = lambda a: synth.as_torch_bf16(a).to(dev)  # noqa: E731
     layers = []
+    tr = lambda a: np.ascontiguousarray(a.T)  # noqa: E731  weights stored [out, in], as in nn.Linear
     for L in w["layers"]:
-        dl = {k: up(L[k]) for k in ("wq", "wk", "wv", "wo", "wd")}
-        dl["wgu"] = up(interleave_gate_up(L["wg"], L["wu"]))
+        dl = {k: up(tr(L[k])) for k in ("wq", "wk", "wv", "wo", "wd")}
+        dl["wgu"] = up(tr(interleave_gate_up(L["wg"], L["wu"])))
         layers.append(dl)
     dc = DecoderConfig(d=cfg["d"], heads=cfg["heads"], head_dim=cfg["head_dim"], ffn=cfg["ffn"],
-                       vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"])
+                       vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"],
+                       w_out_in=True)
     dec = Decoder(dc, up(w["emb"]), up(w["lm_head"]), up(w["gamma"]), layers)
     ids_h, tg_h = synth.decoder_tokens(cfg)
     B, S = ids_h.shape
@@ -654,7 +656,8 @@ def decoder_component(dev, stream):
     att_tc_ms = a.elapsed_time(b) / n
     att_flop = 4.0 * B * cfg["heads"] * cfg["head_dim"] * (S * (S + 1) / 2)
     status = tbik.get_error(stream)
-    return {"workload": "4 layers, d 2048, 16x128 heads, ffn 5632, vocab 32000, batch 8 x seq 2048, TC, T=1",
+    return {"workload": "4 layers, d 2048, 16x128 heads, ffn 5632, vocab 32000, batch 8 x seq 2048, TC, T=1, "
+                        "projection weights stored [out, in]",
             "tokens_per_s": B * S / (ms * 1e-3), "ms_per_forward": ms,
             "bitwise_T1_vs_T8": bool(torch.equal(base.view(torch.int32), t8.view(torch.int32))),
             "ms_per_forward_fused_residual": ms_fused,

@@ -32,13 +32,16 @@ class DecoderConfig:
     layers: int
     leaf: int = 256       # K leaf of the d-wide GEMMs
     leaf_ffn: int = 176   # K leaf of the down projection (ffn wide)
+    w_out_in: bool = False  # projection weights stored [out, in] (the GEMMs' [N,K] operand) instead of [in, out]
 
 
 class Decoder:
     """Weights are device bf16 tensors: ``emb`` and ``lm_head`` [vocab, d],
     ``gamma`` [d], and per layer ``wq wk wv wo`` [d, d], ``wgu`` [d, 2 ffn]
     (gate and up interleaved, see `interleave_gate_up`), ``wd`` [ffn, d]
-    ([in, out] row-major)."""
+    ([in, out] row-major), or each of them transposed ([out, in]) when
+    ``cfg.w_out_in``: the same products, run by the tensor-core GEMM's
+    192-column tiles, with the same bits."""
 
     def __init__(self, cfg: DecoderConfig, emb, lm_head, gamma, layers):
         self.cfg, self.emb, self.lm_head, self.gamma, self.layers = cfg, emb, lm_head, gamma, layers
@@ -70,15 +73,18 @@ class Decoder:
         dev = ids.device
         bf = torch.bfloat16
 
+        nk = c.w_out_in
+
         def dense(a, w, leaf, shards=1, baseline=False):
-            out = torch.empty((a.shape[0], w.shape[1]), dtype=bf, device=dev)
-            tb.gemm(a, w, T=shards, leaf=leaf, tc=tc, noninv=baseline, out_bf16=True, out=out, stream=stream)
+            out = torch.empty((a.shape[0], w.shape[0] if nk else w.shape[1]), dtype=bf, device=dev)
+            tb.gemm(a, w, T=shards, leaf=leaf, tc=tc, noninv=baseline, out_bf16=True, b_nk=nk, out=out,
+                    stream=stream)
             return out
 
         def add_norm(w, a, leaf, res):
             """(y, res) after the row-parallel projection a @ w and its residual add."""
             if fuse_residual:  # res is the stream h, updated in place
-                tb.gemm(a, w, T=T, leaf=leaf, tc=tc, noninv=noninv, residual=res, out=res, stream=stream)
+                tb.gemm(a, w, T=T, leaf=leaf, tc=tc, noninv=noninv, residual=res, out=res, b_nk=nk, stream=stream)
                 y, _ = tb.rmsnorm_residual(res, None, self.gamma, eps=1e-6, T=1, want_res_out=False, stream=stream)
                 return y, res
             return tb.rmsnorm_residual(dense(a, w, leaf, T, noninv), res, self.gamma, eps=1e-6, T=1, stream=stream)
@@ -101,7 +107,7 @@ class Decoder:
                              v.view(B, S, c.heads, c.head_dim), tc=attention_tc, stream=stream)
             y, res = add_norm(L["wo"], o.view(n, c.d), c.leaf, res)
             act = torch.empty((n, c.ffn), dtype=bf, device=dev)
-            tb.gemm(y, L["wgu"], T=1, leaf=c.leaf, tc=tc, swiglu=True, out=act, stream=stream)
+            tb.gemm(y, L["wgu"], T=1, leaf=c.leaf, tc=tc, swiglu=True, b_nk=nk, out=act, stream=stream)
             y, res = add_norm(L["wd"], act, c.leaf_ffn, res)
         lp = tb.logprob(y, self.lm_head, targets.reshape(-1), T=T, leaf=c.leaf, tc=tc, noninv=noninv, stream=stream)
         return lp.view(B, S)

@@ -20,15 +20,18 @@ import invariant_tree_ordered_b200 as tbik  # noqa: E402
 from invariant_tree_ordered_b200.decoder import Decoder, DecoderConfig, interleave_gate_up, positions  # noqa: E402
 
 
-def build(cfg):
+def build(cfg, out_in=False):
+    """The decoder on device; out_in: projection weights stored [out, in]."""
     w = synth.decoder_weights(cfg)
+    lay = (lambda a: np.ascontiguousarray(a.T)) if out_in else (lambda a: a)  # noqa: E731
     layers = []
     for L in w["layers"]:
-        dl = {k: dev_bf16(L[k]) for k in ("wq", "wk", "wv", "wo", "wd")}
-        dl["wgu"] = dev_bf16(interleave_gate_up(L["wg"], L["wu"]))
+        dl = {k: dev_bf16(lay(L[k])) for k in ("wq", "wk", "wv", "wo", "wd")}
+        dl["wgu"] = dev_bf16(lay(interleave_gate_up(L["wg"], L["wu"])))
         layers.append(dl)
     dc = DecoderConfig(d=cfg["d"], heads=cfg["heads"], head_dim=cfg["head_dim"], ffn=cfg["ffn"],
-                       vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"])
+                       vocab=cfg["vocab"], layers=cfg["layers"], leaf=cfg["leaf"], leaf_ffn=cfg["leaf_ffn"],
+                       w_out_in=out_in)
     return w, Decoder(dc, dev_bf16(w["emb"]), dev_bf16(w["lm_head"]), dev_bf16(w["gamma"]), layers)
 
 
@@ -64,6 +67,20 @@ def test_small_fused_residual_exact_matches_oracle_decoder(small):
     for o in outs[1:]:
         assert np.array_equal(u32(o), u32(outs[0]))
     assert tbik.get_error() == tbik.TBIK_OK
+
+
+def test_small_out_in_weights_exact_and_tc_bits(small):
+    """Weights stored [out, in] (the tensor-core GEMM's 192-column tiles): exact
+    mode stays bit-exact to the oracle decoder, tensor-core mode gives the same
+    bits as the [in, out] layout."""
+    cfg, w, dec, ids, tg = small
+    _, dec_t = build(cfg, out_in=True)
+    ref = odec.forward(cfg, w, ids, tg, T=1)
+    assert np.array_equal(u32(run(dec_t, ids, tg, T=2, tc=False)), u32(ref))
+    for T in (1, 8):
+        assert np.array_equal(u32(run(dec_t, ids, tg, T=T, tc=True)), u32(run(dec, ids, tg, T=T, tc=True))), T
+    assert np.array_equal(u32(run(dec_t, ids, tg, T=1, tc=True, fuse_residual=True)),
+                          u32(run(dec, ids, tg, T=1, tc=True, fuse_residual=True)))
 
 
 def test_small_tc_invariant_and_close_to_oracle(small):
