@@ -53,6 +53,7 @@ constexpr int ATC_THREADS = 32 * (2 + ATC_EPI_WARPS);
 constexpr int ATC_TMEM_COLS = 512;
 constexpr uint32_t ATC_S_COL = 0, ATC_O_COL = 128, ATC_SLOT_COL = 384;
 constexpr int ATC_VAL_FLOATS = ATC_BM * ATC_HD;  // one pending o value of the tile
+constexpr int ATC_MAX_GS = 8;  // L2 stack depth bound (chunk trees of up to 256 chunks need 5)
 // shared memory (from a 1024-byte aligned base); V first, so that every
 // descriptor-addressed read stays inside the allocation
 constexpr int ATC_OFF_V = 0;             // [2] 64 keys x 128 dims bf16, two 8 KiB atoms
@@ -71,7 +72,7 @@ struct AttTcParams {
     int tiles;         // batch * heads * ntq
     float scale;
     uint16_t* out;     // [batch][seq][heads][128] bf16
-    float* stack;      // [gridDim.x][gs][ATC_VAL_FLOATS + 2 * ATC_BM]: pending >= 5-chunk values
+    float* stack;      // [gridDim.x][gs][ATC_VAL_FLOATS]: o of the pending >= 5-chunk values
     int gs;
     unsigned long long wait_cycles;
 };
@@ -258,7 +259,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         // on; the pair's barrier (OR reduction) then takes both warps out
         // together, so neither waits there for one that has left.
         bool ab = false;
-        float* stack = p.stack + (size_t)blockIdx.x * p.gs * (ATC_VAL_FLOATS + 2 * ATC_BM);
+        float* stack = p.stack + (size_t)blockIdx.x * p.gs * ATC_VAL_FLOATS;
+        // (m, s) of the L2 stack's values, per thread: both warps of a row
+        // quadrant hold the same values, but a shared copy would race (a leaf
+        // that pops a slot and pushes its result into it lets one warp write the
+        // new value before the other has read the old one)
+        float stk_m[ATC_MAX_GS], stk_s[ATC_MAX_GS];
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x) {
             int qt, bh;
             atc_tile(p, t, qt, bh);
@@ -427,9 +433,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         vm = M;
                     }
                     for (int q = 0; q < nb; ++q) {
-                        const float* sl = stack + (size_t)(gsp - 1 - q) * (ATC_VAL_FLOATS + 2 * ATC_BM);
+                        const int slot = gsp - 1 - q;
+                        const float* sl = stack + (size_t)slot * ATC_VAL_FLOATS;
                         float M, ea, eb;
-                        atc_factors(sl[ATC_VAL_FLOATS + r], vm, M, ea, eb);
+                        atc_factors(stk_m[slot], vm, M, ea, eb);
 #pragma unroll
                         for (int cc = 0; cc < 2; ++cc) {
                             float w[32];
@@ -438,7 +445,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                             for (int k = 0; k < 32; ++k)
                                 v[cc][k] = __fadd_rn(__fmul_rn(w[k], ea), __fmul_rn(v[cc][k], eb));
                         }
-                        vs = __fadd_rn(__fmul_rn(sl[ATC_VAL_FLOATS + ATC_BM + r], ea), __fmul_rn(vs, eb));
+                        vs = __fadd_rn(__fmul_rn(stk_s[slot], ea), __fmul_rn(vs, eb));
                         vm = M;
                     }
                     gsp -= nb;
@@ -455,11 +462,11 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                             m34 = vm;
                             s34 = vs;
                         } else {
-                            float* sl = stack + (size_t)gsp * (ATC_VAL_FLOATS + 2 * ATC_BM);
+                            float* sl = stack + (size_t)gsp * ATC_VAL_FLOATS;
 #pragma unroll
                             for (int cc = 0; cc < 2; ++cc) atc_st32(sl, 2 * half + cc, r, v[cc]);
-                            sl[ATC_VAL_FLOATS + r] = vm;  // both halves hold the same (m, s)
-                            sl[ATC_VAL_FLOATS + ATC_BM + r] = vs;
+                            stk_m[gsp] = vm;
+                            stk_s[gsp] = vs;
                             ++gsp;
                         }
                     } else if (i < p.seq) {

@@ -786,7 +786,8 @@ tbik_status plan_attention_tc(int batch, int seq, int heads, int head_dim, int c
         const int g = max_big_pending(n);
         if (g > p.gs) p.gs = g;
     }
-    p.bytes = (size_t)p.grid * p.gs * (ATC_VAL_FLOATS + 2 * ATC_BM) * sizeof(float);
+    if (p.gs > ATC_MAX_GS) return TBIK_ERR_SHAPE;  // cannot happen for seq <= 16384
+    p.bytes = (size_t)p.grid * p.gs * ATC_VAL_FLOATS * sizeof(float);
     return TBIK_OK;
 }
 

@@ -81,6 +81,21 @@ def test_tc_attention_batch_and_head_split_invariance():
     assert tbik.get_error() == tbik.TBIK_OK
 
 
+def test_tc_attention_repeat_runs_and_batch_subset_at_2048():
+    """Several 2048-position tiles per CTA (persistent grid) with chunk trees
+    deep enough for the L2 stack: repeated calls give the same bits, and so
+    does one sequence alone."""
+    B, S, NH = 4, 2048, 16
+    g = torch.Generator(device="cuda").manual_seed(5)
+    q, k, v = [torch.randn(B, S, NH, 128, device="cuda", generator=g).to(torch.bfloat16) for _ in range(3)]
+    runs = [host_bits16(tbik.attention(q, k, v, tc=True)) for _ in range(3)]
+    for r in runs[1:]:
+        assert np.array_equal(r, runs[0])
+    one = host_bits16(tbik.attention(q[2:3].contiguous(), k[2:3].contiguous(), v[2:3].contiguous(), tc=True))
+    assert np.array_equal(one[0], runs[0][2])
+    assert tbik.get_error() == tbik.TBIK_OK
+
+
 def test_tc_attention_argument_errors():
     lib = tbik.load_library()
     s = torch.cuda.current_stream().cuda_stream
