@@ -412,10 +412,14 @@ TBIK_API tbik_status tbik_get_error(void* stream);
  * Test hooks.  flags: TBIK_DEBUG_WITHHOLD_ACC_ARRIVE makes the tensor-core GEMM
  * epilogue withhold its "accumulator drained" arrive, so the MMA issuer's
  * bounded wait expires: the kernel must record TBIK_ERR_TIMEOUT, drain its own
- * copies in flight, free its TMEM and return.  wait_limit_ns bounds every
- * device-side wait (0 keeps the default of 2 s).
+ * copies in flight, free its TMEM and return.  TBIK_DEBUG_TILE128 runs every
+ * tensor-core GEMM on the 128-column pair tile (normally 192 columns unless B
+ * is [K,N] with N <= 128), so that tests can compare the two tile designs on
+ * the same operands.  wait_limit_ns bounds every device-side wait (0 keeps the
+ * default of 2 s).
  */
 #define TBIK_DEBUG_WITHHOLD_ACC_ARRIVE 0x1u
+#define TBIK_DEBUG_TILE128 0x2u
 TBIK_API tbik_status tbik_debug_set(unsigned flags, unsigned long long wait_limit_ns);
 
 #ifdef __cplusplus

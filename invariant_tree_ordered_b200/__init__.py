@@ -9,7 +9,7 @@ The computation lives in the C-ABI library ``libtbik.so`` (``include/tbik.h``);
 this package is its Python binding.
 """
 from ._binding import (  # noqa: F401
-    B_KN, B_NK, SWIGLU_OUT, DEBUG_WITHHOLD_ACC_ARRIVE, EXACT, NONINV, OUT_BF16, OUT_F32, T_MAX, TC,
+    B_KN, B_NK, SWIGLU_OUT, DEBUG_WITHHOLD_ACC_ARRIVE, DEBUG_TILE128, EXACT, NONINV, OUT_BF16, OUT_F32, T_MAX, TC,
     TBIK_ERR_ALIGN, TBIK_ERR_ARG, TBIK_ERR_CUDA, TBIK_ERR_POSITION, TBIK_ERR_SHAPE, TBIK_ERR_TARGET,
     TBIK_ERR_TIMEOUT, TBIK_ERR_UNSUPPORTED, TBIK_ERR_WORKSPACE, TBIK_OK, VOCAB_LEAF, TbikError, debug_set,
     attention, attention_tc_workspace, declared_functions, embedding, gemm, gemm_workspace, get_error, load_library, logprob, logprob_workspace,

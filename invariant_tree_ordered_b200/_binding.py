@@ -37,6 +37,7 @@ OUT_F32 = 0x000
 OUT_BF16 = 0x100
 SWIGLU_OUT = 0x200
 DEBUG_WITHHOLD_ACC_ARRIVE = 0x1
+DEBUG_TILE128 = 0x2
 VOCAB_LEAF = 64
 T_MAX = 8
 

@@ -669,6 +669,16 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     d |= (uint64_t)2 << 61;
     return d;
 }
+// The same with the 64-byte swizzle (mode 4): atoms of 8 rows x 64 bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;
+    return d;
+}
 
 // Instruction descriptor for kind::f16 (PTX ISA, "Instruction descriptor"):
 // D format f32 (bits 4-5 = 1), A and B bf16 (bits 7-9 = 1, 10-12 = 1),

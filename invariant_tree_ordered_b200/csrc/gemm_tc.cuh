@@ -379,8 +379,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
                         if (a_mine) tma_load_2d_pair(sA + h * p.a_slice, &tmA, bar, kx + 64 * h, arow);
                         if (!b_mn)
                             tma_load_2d_pair(sB + h * (Cfg::B_BYTES / Cfg::KSLICES), &tmB, bar, kx + 64 * h, brow);
-                        else
+                        else if (!Cfg::kWide)
                             tma_load_2d_pair(sB + h * (Cfg::B_BYTES / Cfg::KSLICES), &tmB, bar, brow, kx + 64 * h);
+                    }
+                    if (Cfg::kWide && b_mn) {
+                        // [K,N] B on the 192-column tile: this CTA's 96 columns as three
+                        // 32-column (64-byte swizzle) boxes of the stage's 128 K rows
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d_pair(sB + j * (Cfg::BK * 64), &tmB, bar, brow + 32 * j, kx);
                     }
                     ++q;
                     if (++s == stages) {
@@ -408,16 +415,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
         if (rank == 0) {
             const uint32_t idesc = idesc_bf16_f32(TC_PAIR_M, BN, 0, p.b_mn);
             const bool b_mn = p.b_mn != 0;
-            // MN-major B (a [K,N] operand, 128-column tile only): each CTA's
-            // 64 columns are one 128-byte swizzle atom wide, so the leading
-            // (MN) offset spans the whole half tile and the stride between
-            // 8-deep K groups is 1024 B.
-            constexpr uint32_t b_lbo = (uint32_t)Cfg::B_BYTES, b_sbo = 1024u;
+            // MN-major B (a [K,N] operand).  128-column tile: each CTA's 64
+            // columns are one 128-byte swizzle atom wide, so the leading (MN)
+            // offset spans the whole half tile and the stride between 8-deep K
+            // groups is 1024 B.  192-column tile: 64-byte swizzle, the CTA's 96
+            // columns are three 32-column atoms 128 K rows (8 KiB) apart, 8-deep
+            // K groups 512 B apart, 1 KiB per 16 K rows.
+            constexpr uint32_t b_lbo = Cfg::kWide ? (uint32_t)(Cfg::BK * 64) : (uint32_t)Cfg::B_BYTES;
+            constexpr uint32_t b_sbo = Cfg::kWide ? 512u : 1024u;
             const uint32_t ring_u = smem_u32(ring);
             const uint32_t stage_bytes = p.stage_bytes, a_slice = p.a_slice;
             const int stages = p.stages;
             const int spl = p.leaf / 16;  // MMAs per leaf
-            const uint64_t b_step = b_mn ? (2048u >> 4) : (32u >> 4);
+            const uint64_t b_step = b_mn ? ((Cfg::kWide ? 1024u : 2048u) >> 4) : (32u >> 4);
             const bool aligned = (spl % Cfg::KSTEPS) == 0;  // leaf is a whole number of stages
             const int kb_per_leaf = spl / Cfg::KSTEPS;
             uint32_t a = 0, hc = 0, ph = 0;  // ph: phase of the ring (flips when stage 0 comes round)
@@ -454,12 +464,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
                     const uint32_t sa = ring_u + (uint32_t)s * stage_bytes;
                     const uint32_t sb = sa + a_slice * Cfg::KSLICES;
                     const uint64_t adesc = smem_desc_sw128(sa, 16, 1024);
-                    const uint64_t bdesc = b_mn ? smem_desc_sw128(sb, b_lbo, b_sbo) : smem_desc_sw128(sb, 16, 1024);
+                    const uint64_t bdesc = !b_mn ? smem_desc_sw128(sb, 16, 1024)
+                                                 : (Cfg::kWide ? smem_desc_sw64(sb, b_lbo, b_sbo)
+                                                               : smem_desc_sw128(sb, b_lbo, b_sbo));
                     // k-step ks: slice ks/4 (advance by a slice's bytes >> 4), step ks%4 within it
                     auto a_at = [&](int ks) {
                         return adesc + (uint64_t)((ks >> 2) * (a_slice >> 4) + (ks & 3) * 2);
                     };
                     auto b_at = [&](int ks) {
+                        if (Cfg::kWide && b_mn) return bdesc + b_step * (uint64_t)ks;  // one 128-deep region
                         return bdesc + (uint64_t)((ks >> 2) * ((Cfg::B_BYTES / Cfg::KSLICES) >> 4)) + b_step * (ks & 3);
                     };
                     if (aligned) {

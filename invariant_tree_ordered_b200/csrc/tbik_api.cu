@@ -90,9 +90,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 row-major matrix with `inner` contiguous elements per row and `outer`
-// rows; box = box_inner x box_outer elements, 128-byte swizzle, zero OOB fill.
+// rows; box = box_inner x box_outer elements, 128-byte (or 64-byte) swizzle,
+// zero OOB fill.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
+              uint32_t box_outer, bool swizzle64 = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -100,8 +101,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // bf16 [batch][seq][heads][head_dim] tensor (head_dim contiguous) as a 4-D map
@@ -167,10 +168,14 @@ void set_ring(TcParams& prm, int a_box) {
     prm.stages = st < TC_MAX_STAGES ? st : TC_MAX_STAGES;
 }
 
-// Pair-tile width of the tensor-core GEMM: 192 columns when B is [N,K]
-// (K-major; its TMA box of 96 rows has no swizzle-atom constraint), 128 when
-// B is [K,N].  It depends on the operand layout only, never on M, N or T.
-int tc_tile_n(bool b_nk) { return b_nk ? TC_BN_WIDE : TC_BN; }
+// Pair-tile width of the tensor-core GEMM: 192 columns (a [K,N] B in
+// 64-byte-swizzle atoms of 32 columns), except for a [K,N] B of at most 128
+// columns, which fills one 128-column tile.  It depends on N and the operand
+// layout only, never on M or T (and both widths give the same bits).
+int tc_tile_n(bool b_nk, int N) {
+    if (g_debug_flags & TBIK_DEBUG_TILE128) return TC_BN;
+    return (b_nk || N > TC_BN) ? TC_BN_WIDE : TC_BN;
+}
 size_t tc_slot_bytes(int bn) { return (size_t)TC_BM * bn * sizeof(float); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -240,7 +245,7 @@ tbik_status plan_gemm(int M, int N, int K, int T, int leaf, unsigned mode, int s
     p.M = M, p.N = N, p.K = K, p.T = T, p.leaf = leaf;
     p.L = K / leaf;
     if (p.L % T) return TBIK_ERR_SHAPE;
-    const int bm = tc ? TC_PAIR_M : EX_BM, bn = tc ? tc_tile_n(p.b_nk) : EX_BN;
+    const int bm = tc ? TC_PAIR_M : EX_BM, bn = tc ? tc_tile_n(p.b_nk, N) : EX_BN;
     p.bn = bn;
     if (tc) {
         if (N % 8 || K % 8) return TBIK_ERR_SHAPE;
@@ -381,8 +386,9 @@ tbik_status run_gemm(const GemmPlan& p, const uint16_t* A, const uint16_t* B, vo
         CUtensorMap ta, tb;
         const int a_box = a_box_rows(p.M);
         if (!make_map(&ta, A, (uint64_t)p.K, (uint64_t)p.M, 64, (uint32_t)a_box)) return TBIK_ERR_CUDA;
-        const bool wide = p.bn == TC_BN_WIDE;  // B is [N,K]
-        bool okb = p.b_nk ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, 64, (uint32_t)p.bn / 2)
+        const bool wide = p.bn == TC_BN_WIDE;  // 192-column pair tiles
+        bool okb = p.b_nk  ? make_map(&tb, B, (uint64_t)p.K, (uint64_t)p.N, 64, (uint32_t)p.bn / 2)
+                   : wide ? make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, 32, TcCfg<TC_BN_WIDE>::BK, true)
                           : make_map(&tb, B, (uint64_t)p.N, (uint64_t)p.K, (uint32_t)p.bn / 2, 64);
         if (!okb) return TBIK_ERR_CUDA;
         TcParams prm;
@@ -1059,6 +1065,7 @@ tbik_status tbik_get_error(void* stream) {
 }
 
 tbik_status tbik_debug_set(unsigned flags, unsigned long long wait_limit_ns) {
+    if (flags & ~(TBIK_DEBUG_WITHHOLD_ACC_ARRIVE | TBIK_DEBUG_TILE128)) return TBIK_ERR_ARG;
     g_debug_flags = flags;
     g_wait_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;
     return TBIK_OK;

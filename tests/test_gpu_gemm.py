@@ -187,19 +187,27 @@ def test_down_proj_tc_invariance_over_T_and_M(down_proj):
 
 
 def test_down_proj_tile_widths_agree_bitwise(down_proj):
-    """The [N,K] operand runs the 192-column tile kernel (two TMEM accumulators,
-    the pending 2-leaf value in registers, a split 3-4 leaf slot), the [K,N]
-    operand the 128-column one (three accumulators, TMEM and shared-memory
-    slots): different storage plans for the same 56-leaf tree.  Both must give
-    the same bits, at T = 1 and T = 8 and for a shifted batch."""
+    """The 192-column tile kernel (two TMEM accumulators, the pending 2-leaf
+    value in registers, a split 3-4 leaf slot; B [K,N] in 64-byte-swizzle
+    atoms, B [N,K] K-major) and the 128-column one (three accumulators, TMEM
+    and shared-memory slots; the test hook forces it): different storage
+    plans and operand layouts for the same 56-leaf tree.  All must give the
+    same bits, at T = 1 and T = 8 and for a shifted batch."""
     a, b = down_proj
     bt = np.ascontiguousarray(b.T)
     for T in (1, 8):
         kn = run(a, b, T=T, leaf=256, tc=True)
         nk = run(a, bt, T=T, leaf=256, tc=True, b_nk=True)
+        try:
+            tbik.debug_set(tbik.DEBUG_TILE128, 0)
+            kn128 = run(a, b, T=T, leaf=256, tc=True)
+        finally:
+            tbik.debug_set(0, 0)
         assert np.array_equal(u32(kn), u32(nk)), T
-    sub = run(a[7:300], bt, T=2, leaf=256, tc=True, b_nk=True)
+        assert np.array_equal(u32(kn), u32(kn128)), T
+    sub = run(a[7:300], b, T=2, leaf=256, tc=True)
     assert np.array_equal(u32(sub), u32(kn[7:300]))
+    assert tbik.get_error() == tbik.TBIK_OK
 
 
 def test_down_proj_exact_sampled_rows_full_M(down_proj):
