@@ -11,7 +11,7 @@
 // every shard count (and, as measured, for either tile width).
 //
 // CTA pairs (clusters of 2, cta_group::2): a pair computes a 256 x BN tile,
-// BN = 128 when B is [K,N] and 192 when B is [N,K]; CTA r holds rows
+// BN = 192 (128 for a [K,N] B of at most 128 columns); CTA r holds rows
 // [128r, 128r+128) of A and rows/columns [BN/2 r, BN/2 (r+1)) of B in its
 // shared memory and its own 128 x BN fp32 accumulators in TMEM.  The leader
 // (rank 0) issues the MMAs; commits arrive on both CTAs' barriers.  Each CTA
@@ -58,8 +58,8 @@ namespace tbik {
 
 constexpr int TC_BM = 128;        // rows per CTA
 constexpr int TC_PAIR_M = 256;    // rows per CTA pair (one MMA tile)
-constexpr int TC_BN = 128;        // columns per pair tile when B is [K,N]
-constexpr int TC_BN_WIDE = 192;   // columns per pair tile when B is [N,K]
+constexpr int TC_BN = 128;        // columns per pair tile: narrow [K,N] operands (N <= 128)
+constexpr int TC_BN_WIDE = 192;   // columns per pair tile otherwise
 constexpr int TC_MAX_STAGES = 8;  // ring stages when the A copies are small (small M)
 constexpr int TC_BAR_EPI = 1;      // named barrier: the epilogue warps
 constexpr int TC_BAR_HANDOFF = 2;  // named barrier: waiter warp + MMA warp, lockstep
