@@ -205,7 +205,12 @@ typedef struct {
     /* SwiGLU group (skipped when g is NULL): out = bf16((g / (1 + exp(-g))) * u)
        in fp32 with the library's exp specification (Cody-Waite reduction by a
        split ln 2, degree-7 Taylor polynomial, correctly rounded scaling).
-       g/u bf16 or fp32 (in_f32 = 1) [n]; out bf16 [n]; n % 8 == 0. */
+       g/u bf16 or fp32 (in_f32 = 1) [n]; out bf16 [n]; n % 8 == 0.
+       With bf16 g, silu(g) = g / (1 + exp(-g)) is read from a table of its
+       fp32 value for every bf16 g (the same bits): the first such call on a
+       device builds the 256 KiB table on its stream and records an event that
+       later calls on any stream wait for; make that first call outside a
+       stream capture. */
     const void* g;
     const void* u;
     uint16_t* out;

@@ -173,6 +173,59 @@ __global__ void rope_kernel(const uint16_t* __restrict__ q, const uint16_t* __re
 }
 
 
+// SwiGLU of bf16 gates through a table: silu(g) = g / (1 + exp(-g)) depends
+// only on g's 16 bits, so g_silu_lut[bits] holds the fp32 result of exactly the
+// operations of swiglu1 for every bf16 value, and out = bf16(lut[g] * u) has
+// the same bits as the computed form (the GPU tests run all 65536 gates).
+// Built once per device (silu_lut_kernel) before the first table lookup.
+static __device__ float g_silu_lut[65536];
+
+__global__ void silu_lut_kernel() {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= 65536) return;
+    const float g = __uint_as_float((uint32_t)t << 16);
+    const float e = exp_spec(-g);
+    const float den = __fadd_rn(1.0f, e);
+    g_silu_lut[t] = __fdiv_rn(g, den);
+}
+
+// out = bf16(lut[g] * u) for bf16 g and u, 8 elements per thread per
+// iteration of a grid-stride loop (the next vector's loads in flight); the
+// table (256 KiB) is read through the read-only cache.
+template <typename IDX>
+__global__ void swiglu_lut_kernel(const uint16_t* __restrict__ g, const uint16_t* __restrict__ u, uint16_t* out,
+                                  long long n) {
+    const IDX nv = (IDX)(n >> 3);
+    const IDX stride = (IDX)gridDim.x * blockDim.x;
+    IDX i = (IDX)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= nv) return;
+    uint4 cg = __ldg(reinterpret_cast<const uint4*>(g) + i), cu = __ldg(reinterpret_cast<const uint4*>(u) + i);
+    while (true) {
+        const IDX inext = i + stride;
+        const bool more = inext < nv;
+        uint4 ng, nu;
+        if (more) {
+            ng = __ldg(reinterpret_cast<const uint4*>(g) + inext);
+            nu = __ldg(reinterpret_cast<const uint4*>(u) + inext);
+        }
+        const uint32_t gw[4] = {cg.x, cg.y, cg.z, cg.w};
+        float sg[8], uf[8], o[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sg[2 * e] = __ldg(g_silu_lut + (gw[e] & 0xffffu));
+            sg[2 * e + 1] = __ldg(g_silu_lut + (gw[e] >> 16));
+        }
+        unpack8(cu, uf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(sg[e], uf[e]);
+        reinterpret_cast<uint4*>(out)[i] = pack8(o);
+        if (!more) break;
+        i = inext;
+        cg = ng;
+        cu = nu;
+    }
+}
+
 // out = bf16((g / (1 + exp(-g))) * u), one 8-element vector per thread per
 // iteration of a grid-stride loop; the next iteration's inputs are loaded
 // before this one's arithmetic, so loads stay in flight during the (ALU-heavy)

@@ -36,6 +36,7 @@ struct DeviceInfo {
     int sms = 0;
     int clock_khz = 0;
     bool attrs_set = false;
+    cudaEvent_t lut_built = nullptr;  // the SwiGLU table's build, recorded on the stream that ran it
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -920,10 +921,25 @@ tbik_status tbik_rope_swiglu_fp32(const tbik_rope_swiglu_args* a, void* stream) 
             else
                 swiglu_kernel<1, long long><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
         } else {
+            // bf16 gates: the table, built on this device once (on the first
+            // caller's stream; later calls on any stream wait for its event)
+            {
+                std::lock_guard<std::mutex> lk(g_mu);
+                if (!info->lut_built) {
+                    silu_lut_kernel<<<65536 / 256, 256, 0, s>>>();
+                    cudaEvent_t ev;
+                    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return TBIK_ERR_CUDA;
+                    if (cudaEventRecord(ev, s) != cudaSuccess) return TBIK_ERR_CUDA;
+                    info->lut_built = ev;
+                }
+            }
+            if (cudaStreamWaitEvent(s, info->lut_built, 0) != cudaSuccess) return TBIK_ERR_CUDA;
+            const uint16_t* g16 = reinterpret_cast<const uint16_t*>(a->g);
+            const uint16_t* u16 = reinterpret_cast<const uint16_t*>(a->u);
             if (narrow)
-                swiglu_kernel<0, uint32_t><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+                swiglu_lut_kernel<uint32_t><<<(int)blocks, 256, 0, s>>>(g16, u16, a->out, a->n);
             else
-                swiglu_kernel<0, long long><<<(int)blocks, 256, 0, s>>>(a->g, a->u, a->out, a->n);
+                swiglu_lut_kernel<long long><<<(int)blocks, 256, 0, s>>>(g16, u16, a->out, a->n);
         }
         if ((st = launch_status()) != TBIK_OK) return st;
     }

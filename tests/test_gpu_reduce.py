@@ -123,6 +123,12 @@ def test_swiglu_every_bf16_gate_value():
         got = host_bits16(out)
         same = (got == ref) | (np.isnan(synth.bf16_bits_to_f32(got)) & np.isnan(synth.bf16_bits_to_f32(ref)))
         assert np.all(same), u_val
+        # bf16 gates read silu(g) from the library's table; the same values as
+        # fp32 inputs take the computed path: the two give the same bits
+        _, _, out32 = tbik.rope_swiglu(g=dev_f32(synth.bf16_bits_to_f32(g2)), u=dev_f32(synth.bf16_bits_to_f32(ub)))
+        got32 = host_bits16(out32)
+        same32 = (got == got32) | (np.isnan(synth.bf16_bits_to_f32(got)) & np.isnan(synth.bf16_bits_to_f32(got32)))
+        assert np.all(same32), u_val
 
 
 def test_rope_swiglu_argument_errors():
