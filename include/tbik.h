@@ -246,24 +246,29 @@ TBIK_API tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const 
 
 /*
  * The same attention in tensor-core mode (TBIK summary page, 技术框架: the
- * key reduction stays one fixed tree of 64-key chunks).  Per chunk:
+ * key reduction stays one fixed tree, here of 128-key leaves, each computed
+ * as two 64-key tensor-core chunks under one maximum).  Per leaf:
  *   s_j = fl(dot(q_i, k_j) * scale) with the dot product on the tensor cores
  *         (bf16 operands, fp32 accumulation in the hardware's fixed order);
- *   m = max over the chunk's keys j <= i; p_j = bf16(2^(s_j*log2e - m*log2e))
- *   (hardware exponential; 0 for j > i); s = (ascending sum of the rounded
- *   p_j over keys 0..31) + (the same over keys 32..63); o = sum of p_j * v_j
+ *   m = max over the leaf's keys j <= i; p_j = bf16(2^(s_j*log2e - m*log2e))
+ *   (hardware exponential; 0 for j > i); s = s_lo + s_hi over the rounded
+ *   p_j (keys 0..63 and 64..127 of the leaf, each (c0 + c1) + (c2 + c3) with
+ *   c_q the ascending sum over its keys k = q mod 4); o = sum of p_j * v_j
  *   on the tensor cores;
- * chunk summaries combined by TREE exactly as in tbik_attention (exp
- * specification for the combine factors), out[d] = bf16(o[d] / s).  Each
- * output row depends only on its query and the keys/values at positions <= i,
- * so it is bitwise the same for any batch composition and head split; it is
- * checked against the binary64 definition by tolerance.
+ * leaf summaries combined by TREE: M = max, e = exp(m - M) (the exp
+ * specification; 1 for the side holding M), s = fma(s', e', fl(s*e)),
+ * o = fma(o', e', fl(o*e)) (left operand's product rounded);
+ * out[d] = bf16(o[d] / s).  Each output row depends only on its query and
+ * the keys/values at positions <= i, so it is bitwise the same for any batch
+ * composition and head split; it is checked against the binary64 definition
+ * by tolerance.
  * q, k, v, out: bf16 [batch][seq][heads][head_dim], device memory, 16-byte
- * aligned; out may alias q but not k or v.  head_dim == 128, chunk == 64,
- * seq a multiple of 128 and <= 16384 (else TBIK_ERR_SHAPE); workspace: device
- * memory of at least tbik_attention_tc_workspace() bytes, 16-byte aligned
- * (TBIK_ERR_WORKSPACE / TBIK_ERR_ALIGN otherwise; may be NULL when that is 0),
- * owned by the caller and not used by concurrent calls.  No launch on error.
+ * aligned; out may alias q but not k or v.  head_dim == 128, chunk == 128
+ * (the leaf), seq a multiple of 128 and <= 16384 (else TBIK_ERR_SHAPE);
+ * workspace: device memory of at least tbik_attention_tc_workspace() bytes,
+ * 16-byte aligned (TBIK_ERR_WORKSPACE / TBIK_ERR_ALIGN otherwise; may be NULL
+ * when that is 0), owned by the caller and not used by concurrent calls.  No
+ * launch on error.
  */
 TBIK_API size_t tbik_attention_tc_workspace(int batch, int seq, int heads, int head_dim, int chunk);
 TBIK_API tbik_status tbik_attention_tc(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,

@@ -303,18 +303,26 @@ def rope_swiglu(*, q=None, k=None, pos=None, table=None, q_out=None, k_out=None,
     return q_out, k_out, out
 
 
-def attention_tc_workspace(batch, seq, heads, head_dim, chunk=64) -> int:
+# keys per tree leaf: the exact mode's chunk and the tensor-core mode's leaf (two 64-key MMA chunks)
+ATTENTION_CHUNK = 64
+ATTENTION_TC_LEAF = 128
+
+
+def attention_tc_workspace(batch, seq, heads, head_dim, chunk=ATTENTION_TC_LEAF) -> int:
     n = load_library().tbik_attention_tc_workspace(batch, seq, heads, head_dim, chunk)
     if n == (1 << 64) - 1:
         raise TbikError(TBIK_ERR_SHAPE, "tbik_attention_tc_workspace: unsupported shape")
     return n
 
 
-def attention(q, k, v, *, out=None, chunk: int = 64, tc: bool = False, workspace=None, stream=None):
+def attention(q, k, v, *, out=None, chunk=None, tc: bool = False, workspace=None, stream=None):
     """Causal attention with the key reduction in tree order; q, k, v bf16
     [batch, seq, heads, head_dim].  tc=False: tbik_attention (exact order on
-    the CUDA cores); tc=True: tbik_attention_tc (tensor cores; a workspace is
-    allocated when none is given)."""
+    the CUDA cores, leaves of `chunk` = 64 keys); tc=True: tbik_attention_tc
+    (tensor cores, leaves of 128 keys; a workspace is allocated when none is
+    given)."""
+    if chunk is None:
+        chunk = ATTENTION_TC_LEAF if tc else ATTENTION_CHUNK
     torch = _torch()
     lib = load_library()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):

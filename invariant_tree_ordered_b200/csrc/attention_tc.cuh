@@ -2,65 +2,72 @@
 //
 // Source: TBIK summary page, 技术框架 (one hierarchical binary tree for every
 // reduction, so the result does not depend on how the work is split).  The
-// structure is the exact mode's (attention.cuh): keys in chunks of 64
-// positions, each chunk reduced to a (max, sum, weighted value sum) summary,
-// the summaries of chunks 0..floor(i/64) combined by the halving tree.  What
-// differs is how one chunk is computed:
+// structure is the exact mode's (attention.cuh): keys in fixed leaves, each
+// leaf reduced to a (max, sum, weighted value sum) summary, the summaries of
+// the leaves 0..floor(i/128) combined by the halving tree.  What differs is
+// the leaf (128 keys, two 64-key tensor-core chunks under one maximum) and how
+// it is computed:
 //   scores  s_j = fl(S_ij * scale), S = Q K^T on the tensor cores (tcgen05,
 //           bf16 operands, fp32 accumulation in TMEM in the hardware's order);
-//   chunk   m = max over the chunk's keys j <= i;
+//   leaf    m = max over the leaf's keys j <= i;
 //           p_j = bf16(2^(s_j*log2e - m*log2e)) with the hardware exponential,
-//           0 for j > i; s = (ascending sum of p_j over keys 0..31) +
-//           (ascending sum over keys 32..63), of the rounded p_j;
-//           o = P V on the tensor cores (the bf16 p_j as A, V as B);
-//   combine the exact mode's rule: M = max, e = exp(m - M) by the library's
-//           exp specification (1 for the side holding M), s = s*e + s'*e',
-//           o = o*e + o'*e' (products rounded separately);
+//           0 for j > i; s = s_lo + s_hi over the rounded p_j, where s_lo
+//           covers keys 0..63 of the leaf and s_hi keys 64..127, each
+//           (c0 + c1) + (c2 + c3) with c_q the ascending sum over the keys
+//           k = q (mod 4) of that half;
+//           o = P V on the tensor cores (the bf16 p_j as A, V as B, K = 128);
+//   combine M = max, e = exp(m - M) by the library's exp specification (1 for
+//           the side holding M), s = fma(s', e', fl(s*e)),
+//           o = fma(o', e', fl(o*e)) (the left operand's product rounded);
 //   output  bf16(o[d] / s).
 // A row's result depends only on its query, the keys and values at positions
-// <= i and its fixed chunk tree, never on the batch composition, the other
+// <= i and its fixed leaf tree, never on the batch composition, the other
 // rows of its tile or how heads are split across devices.
 //
 // One CTA per SM, persistent over 128-row query tiles of one (batch, head),
 // the longest tiles first; 320 threads:
 //   warp 0     TMA producer: the Q tile (two 64-dim slices, K-major, 128-byte
-//              swizzle) and per chunk K (same layout, 64 rows) and V (MN-major:
-//              two 64-dim atoms of 64 keys) into a 2-stage ring
-//   warp 1     TMEM allocator + MMA issuer: S_c = Q K_c^T (M=128, N=64) into
-//              S[c%2], then O_{c-1} = P_{c-1} V_{c-1} (M=128, N=128, K=64)
-//              into O[(c-1)%2]
+//              swizzle), per leaf K (same layout, two 64-key chunks) and V
+//              (MN-major: per chunk two 64-dim atoms of 64 keys); K of the
+//              next leaf is requested as soon as the scores of the current
+//              one are done, before V of the current one
+//   warp 1     TMEM allocator + MMA issuer: S = Q K^T of the leaf's two chunks
+//              (M=128, N=64 each) into S[0], S[1], then O_{L-1} = P V of the
+//              previous leaf (M=128, N=128, K=128) into O[(L-1)%2]
 //   warps 2-9  epilogue: warp w owns rows 32*(w%4).. and half h = (w-2)/4:
-//              keys [32h, 32h+32) of each chunk's softmax and head dims
-//              [64h, 64h+64) of the tree.  Loop: softmax of chunk c (writes
-//              P_c), then the tree step of chunk c-1, so the MMA of O_c runs
-//              while the tree of chunk c-1 is evaluated.
-// A tile starts at a multiple of 128: its rows 0..63 have i0/64 + 1 chunks,
-// rows 64..127 one more, so the tree walk is the same for all lanes of a warp.
-// Pending chunk summaries wait by size: a single chunk in its O buffer (the
-// next chunk consumes it), 2 chunks in a TMEM slot, 3-4 in shared memory,
-// >= 5 in a per-CTA stack in global memory that stays in L2.
+//              the softmax of chunk h of each leaf (its maximum taken over
+//              both chunks) and head dims [64h, 64h+64) of the tree.  Loop:
+//              softmax of leaf L (writes P_L), then the tree step of leaf
+//              L-1, so the MMA of O_L runs while the tree of L-1 is evaluated.
+// A tile starts at a multiple of 128, so every row of it has the same leaves
+// (the tile's own block is the last, the diagonal one) and the tree walk is
+// the same for all lanes of a warp.  Pending leaf summaries wait by size: a
+// single leaf in its O buffer (the next leaf consumes it), 2 leaves in a TMEM
+// slot, 3-4 in shared memory, >= 5 in a per-CTA stack in global memory that
+// stays in L2.
 #pragma once
 
 #include "device_common.cuh"
 
 namespace tbik {
 
-constexpr int ATC_BM = 128;  // query rows per tile
-constexpr int ATC_CH = 64;   // keys per chunk
-constexpr int ATC_HD = 128;  // head dimension
+constexpr int ATC_BM = 128;    // query rows per tile
+constexpr int ATC_CH = 64;     // keys per tensor-core chunk
+constexpr int ATC_LEAF = 128;  // keys per tree leaf (two chunks)
+constexpr int ATC_HD = 128;    // head dimension
 constexpr int ATC_EPI_WARPS = 8;
 constexpr int ATC_THREADS = 32 * (2 + ATC_EPI_WARPS);
 constexpr int ATC_TMEM_COLS = 512;
 constexpr uint32_t ATC_S_COL = 0, ATC_O_COL = 128, ATC_SLOT_COL = 384;
 constexpr int ATC_VAL_FLOATS = ATC_BM * ATC_HD;  // one pending o value of the tile
-constexpr int ATC_MAX_GS = 8;  // L2 stack depth bound (chunk trees of up to 256 chunks need 5)
+constexpr int ATC_MAX_GS = 8;  // L2 stack depth bound (leaf trees of up to 256 leaves need 5)
 // shared memory (from a 1024-byte aligned base); V first, so that every
 // descriptor-addressed read stays inside the allocation
-constexpr int ATC_OFF_V = 0;             // [2] 64 keys x 128 dims bf16, two 8 KiB atoms
-constexpr int ATC_OFF_K = 32768;         // [2] 64 keys x 128 dims, two 8 KiB slices
+constexpr int ATC_OFF_V = 0;             // the leaf's 2 chunks x 64 keys x 128 dims bf16, two 8 KiB atoms each
+constexpr int ATC_OFF_K = 32768;         // the leaf's 2 chunks x 64 keys x 128 dims, two 8 KiB slices each
 constexpr int ATC_OFF_Q = 65536;         // 128 rows x 128 dims, two 16 KiB slices
-constexpr int ATC_OFF_P = 98304;         // [2] 128 rows x 64 keys bf16
-constexpr int ATC_OFF_SLOT = 131072;     // pending 3-4 chunk value, fp32 [dim/4][row][4]
+constexpr int ATC_OFF_P = 98304;         // [2 chunks] 128 rows x 64 keys bf16
+constexpr int ATC_OFF_SLOT = 131072;     // pending 3-4 leaf value, fp32 [dim/4][row][4]
 constexpr int ATC_OFF_X = 196608;        // [2][2][128] per-row sums exchanged between halves
 constexpr int ATC_OFF_BAR = 198656;
 constexpr size_t ATC_SMEM_BYTES = ATC_OFF_BAR + 256 + 1024;
@@ -72,7 +79,7 @@ struct AttTcParams {
     int tiles;         // batch * heads * ntq
     float scale;
     uint16_t* out;     // [batch][seq][heads][128] bf16
-    float* stack;      // [gridDim.x][gs][ATC_VAL_FLOATS]: o of the pending >= 5-chunk values
+    float* stack;      // [gridDim.x][gs][ATC_VAL_FLOATS]: o of the pending >= 5-leaf values
     int gs;
     unsigned long long wait_cycles;
 };
@@ -93,6 +100,26 @@ __device__ __forceinline__ void atc_st32(float* base, int c, int row, const floa
     for (int q = 0; q < 8; ++q)
         *reinterpret_cast<float4*>(base + ((size_t)(c * 8 + q) * ATC_BM + row) * 4) =
             make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+__device__ __forceinline__ float atc_f(float x) { return x; }
+__device__ __forceinline__ float atc_f(uint32_t x) { return __uint_as_float(x); }
+
+// out[k] = fma(b[k], eb, fl(a[k] * ea)): the left operand's product rounded,
+// the right one's fused into the add; two lanes per instruction (each lane the
+// IEEE result of the scalar operation).
+template <typename TA, typename TB>
+__device__ __forceinline__ void atc_comb(float (&out)[32], const TA (&a)[32], float ea, const TB (&b)[32], float eb) {
+    const f2x ea2 = pk2(ea, ea), eb2 = pk2(eb, eb);
+#pragma unroll
+    for (int k = 0; k < 32; k += 2) {
+        const f2x r = fma2(pk2(atc_f(b[k]), atc_f(b[k + 1])), eb2, mul2(pk2(atc_f(a[k]), atc_f(a[k + 1])), ea2));
+        upk2(r, out[k], out[k + 1]);
+    }
+}
+// The same rule for the running sums.
+__device__ __forceinline__ float atc_comb1(float a, float ea, float b, float eb) {
+    return __fmaf_rn(b, eb, __fmul_rn(a, ea));
 }
 
 // Combine factors of two summaries (a is the left operand): M and the two
@@ -121,14 +148,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ATC_OFF_BAR);
     uint64_t* q_full = bars;           // Q tile landed
     uint64_t* q_empty = bars + 1;      // the tile's last S MMA retired
-    uint64_t* kv_full = bars + 2;      // [2] K and V of a chunk landed
-    uint64_t* kv_empty = bars + 4;     // [2] the chunk's MMAs retired
-    uint64_t* s_full = bars + 6;       // [2] S of a chunk in TMEM
-    uint64_t* p_full = bars + 8;       // [2] P of a chunk written (S read) by the 8 epilogue warps
-    uint64_t* o_full = bars + 10;      // [2] O of a chunk in TMEM
-    uint64_t* o_empty = bars + 12;     // [2] O buffer released by the 8 epilogue warps
-    uint64_t* done = bars + 14;        // every MMA issued by this CTA retired
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+    uint64_t* k_full = bars + 2;       // K of a leaf landed
+    uint64_t* k_empty = bars + 3;      // the leaf's S MMAs retired
+    uint64_t* v_full = bars + 4;       // V of a leaf landed
+    uint64_t* v_empty = bars + 5;      // the leaf's P V MMAs retired
+    uint64_t* s_full = bars + 6;       // S of a leaf (both chunks) in TMEM
+    uint64_t* p_full = bars + 7;       // P of a leaf written (S read) by the 8 epilogue warps
+    uint64_t* o_full = bars + 8;       // [2] O of a leaf in TMEM
+    uint64_t* o_empty = bars + 10;     // [2] O buffer released by the 8 epilogue warps
+    uint64_t* done = bars + 12;        // every MMA issued by this CTA retired
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,11 +165,13 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
+        mbar_init(k_full, 1);
+        mbar_init(k_empty, 1);
+        mbar_init(v_full, 1);
+        mbar_init(v_empty, 1);
+        mbar_init(s_full, 1);
+        mbar_init(p_full, ATC_EPI_WARPS);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&kv_full[b], 1);
-            mbar_init(&kv_empty[b], 1);
-            mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], ATC_EPI_WARPS);
             mbar_init(&o_full[b], 1);
             mbar_init(&o_empty[b], ATC_EPI_WARPS);
         }
@@ -163,33 +194,42 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            uint32_t g = 0, nt = 0;  // chunks and tiles loaded so far by this CTA
+            uint32_t gk = 0, gv = 0, nt = 0;  // K leaves, V leaves and tiles loaded so far by this CTA
             for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++nt) {
                 int qt, bh;
                 atc_tile(p, t, qt, bh);
                 const int b = bh / p.heads, h = bh - b * p.heads;
                 const int i0 = qt * ATC_BM;
-                const int nc = i0 / ATC_CH + 2;
+                const int nl = qt + 1;  // leaves of the tile
                 if (nt > 0 && !mbar_wait(q_empty, (nt - 1) & 1, abort_flag, lim)) goto producer_out;
                 mbar_arrive_expect_tx(q_full, 2 * ATC_BM * 128);
                 for (int sl = 0; sl < 2; ++sl)
                     tma_load_4d(smem + ATC_OFF_Q + sl * 16384, &tmQ, q_full, 64 * sl, h, i0, b);
-                for (int c = 0; c < nc; ++c, ++g) {
-                    const int s = g & 1;
-                    if (g >= 2 && !mbar_wait(&kv_empty[s], ((g >> 1) - 1) & 1, abort_flag, lim)) goto producer_out;
-                    mbar_arrive_expect_tx(&kv_full[s], 2 * 2 * ATC_CH * 128);
-                    for (int sl = 0; sl < 2; ++sl) {
-                        tma_load_4d(smem + ATC_OFF_K + s * 16384 + sl * 8192, &tmK, &kv_full[s], 64 * sl, h,
-                                    ATC_CH * c, b);
-                        tma_load_4d(smem + ATC_OFF_V + s * 16384 + sl * 8192, &tmV, &kv_full[s], 64 * sl, h,
-                                    ATC_CH * c, b);
+                for (int l = 0; l <= nl; ++l) {
+                    if (l < nl) {  // K of leaf l
+                        if (gk >= 1 && !mbar_wait(k_empty, (gk - 1) & 1, abort_flag, lim)) goto producer_out;
+                        mbar_arrive_expect_tx(k_full, 2 * 2 * ATC_CH * 128);
+                        for (int ch = 0; ch < 2; ++ch)
+                            for (int sl = 0; sl < 2; ++sl)
+                                tma_load_4d(smem + ATC_OFF_K + ch * 16384 + sl * 8192, &tmK, k_full, 64 * sl, h,
+                                            ATC_LEAF * l + ATC_CH * ch, b);
+                        ++gk;
+                    }
+                    if (l >= 1) {  // V of leaf l - 1
+                        if (gv >= 1 && !mbar_wait(v_empty, (gv - 1) & 1, abort_flag, lim)) goto producer_out;
+                        mbar_arrive_expect_tx(v_full, 2 * 2 * ATC_CH * 128);
+                        for (int ch = 0; ch < 2; ++ch)
+                            for (int sl = 0; sl < 2; ++sl)
+                                tma_load_4d(smem + ATC_OFF_V + ch * 16384 + sl * 8192, &tmV, v_full, 64 * sl, h,
+                                            ATC_LEAF * (l - 1) + ATC_CH * ch, b);
+                        ++gv;
                     }
                 }
             }
         producer_out:
             // let the last copies land before the CTA can exit
-            if (g > 0) mbar_drain(&kv_full[(g - 1) & 1], ((g - 1) >> 1) & 1, lim);
-            if (g > 1) mbar_drain(&kv_full[(g - 2) & 1], ((g - 2) >> 1) & 1, lim);
+            if (gk > 0) mbar_drain(k_full, (gk - 1) & 1, lim);
+            if (gv > 0) mbar_drain(v_full, (gv - 1) & 1, lim);
             if (nt > 0) mbar_drain(q_full, (nt - 1) & 1, lim);
         }
     } else if (warp == 1) {
@@ -202,42 +242,54 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++nt) {
                 int qt, bh;
                 atc_tile(p, t, qt, bh);
-                const int nc = (qt * ATC_BM) / ATC_CH + 2;
+                const int nl = qt + 1;
                 if (!mbar_wait(q_full, nt & 1, abort_flag, lim)) goto mma_out;
-                for (int c = 0; c <= nc; ++c) {
-                    if (c < nc) {
-                        const uint32_t g = g0 + c, b = g & 1, ph = (g >> 1) & 1;
-                        if (!mbar_wait(&kv_full[b], ph, abort_flag, lim)) goto mma_out;
-                        // S[b] was read by the softmax of chunk g - 2
-                        if (g >= 2 && !mbar_wait(&p_full[b], ph ^ 1, abort_flag, lim)) goto mma_out;
+                for (int l = 0; l <= nl; ++l) {
+                    if (l < nl) {
+                        const uint32_t g = g0 + l;
+                        if (!mbar_wait(k_full, g & 1, abort_flag, lim)) goto mma_out;
+                        // S was read by the softmax of leaf g - 1
+                        if (g >= 1 && !mbar_wait(p_full, (g - 1) & 1, abort_flag, lim)) goto mma_out;
                         tc_fence_after();
                         const uint64_t adesc = smem_desc_sw128(q_u, 16, 1024);
-                        const uint64_t bdesc = smem_desc_sw128(smem_u32(smem + ATC_OFF_K + b * 16384), 16, 1024);
 #pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            tc_mma(tmem_base + ATC_S_COL + 64 * b,
-                                   adesc + (uint64_t)((ks >> 2) * (16384 >> 4) + (ks & 3) * 2),
-                                   bdesc + (uint64_t)((ks >> 2) * (8192 >> 4) + (ks & 3) * 2), idesc_s, ks ? 1u : 0u);
-                        tc_commit(&s_full[b]);
-                        if (c == nc - 1) tc_commit(q_empty);
+                        for (int ch = 0; ch < 2; ++ch) {
+                            const uint64_t bdesc =
+                                smem_desc_sw128(smem_u32(smem + ATC_OFF_K + ch * 16384), 16, 1024);
+#pragma unroll
+                            for (int ks = 0; ks < 8; ++ks)
+                                tc_mma(tmem_base + ATC_S_COL + 64 * ch,
+                                       adesc + (uint64_t)((ks >> 2) * (16384 >> 4) + (ks & 3) * 2),
+                                       bdesc + (uint64_t)((ks >> 2) * (8192 >> 4) + (ks & 3) * 2), idesc_s,
+                                       ks ? 1u : 0u);
+                        }
+                        tc_commit(s_full);
+                        tc_commit(k_empty);
+                        if (l == nl - 1) tc_commit(q_empty);
                     }
-                    if (c >= 1) {
-                        const uint32_t g = g0 + c - 1, b = g & 1, ph = (g >> 1) & 1;
-                        if (!mbar_wait(&p_full[b], ph, abort_flag, lim)) goto mma_out;
+                    if (l >= 1) {
+                        const uint32_t g = g0 + l - 1, b = g & 1, ph = (g >> 1) & 1;
+                        if (!mbar_wait(v_full, g & 1, abort_flag, lim)) goto mma_out;
+                        // P of leaf g: already awaited above unless no S was issued in this step
+                        if (l == nl && !mbar_wait(p_full, g & 1, abort_flag, lim)) goto mma_out;
                         if (g >= 2 && !mbar_wait(&o_empty[b], ph ^ 1, abort_flag, lim)) goto mma_out;
                         tc_fence_after();
-                        const uint64_t adesc = smem_desc_sw128(smem_u32(smem + ATC_OFF_P + b * 16384), 16, 1024);
-                        // V: MN-major, the two 64-dim atoms 8 KiB apart, 8-key groups 1 KiB apart
-                        const uint64_t bdesc = smem_desc_sw128(smem_u32(smem + ATC_OFF_V + b * 16384), 8192, 1024);
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc_mma(tmem_base + ATC_O_COL + 128 * b, adesc + (uint64_t)(ks * 2),
-                                   bdesc + (uint64_t)(ks * (2048 >> 4)), idesc_o, ks ? 1u : 0u);
+                        for (int ch = 0; ch < 2; ++ch) {
+                            const uint64_t adesc = smem_desc_sw128(smem_u32(smem + ATC_OFF_P + ch * 16384), 16, 1024);
+                            // V: MN-major, the two 64-dim atoms 8 KiB apart, 8-key groups 1 KiB apart
+                            const uint64_t bdesc =
+                                smem_desc_sw128(smem_u32(smem + ATC_OFF_V + ch * 16384), 8192, 1024);
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                tc_mma(tmem_base + ATC_O_COL + 128 * b, adesc + (uint64_t)(ks * 2),
+                                       bdesc + (uint64_t)(ks * (2048 >> 4)), idesc_o, (ch | ks) ? 1u : 0u);
+                        }
                         tc_commit(&o_full[b]);
-                        tc_commit(&kv_empty[b]);
+                        tc_commit(v_empty);
                     }
                 }
-                g0 += nc;
+                g0 += nl;
             }
         mma_out:
             // every MMA retires before TMEM is released
@@ -248,12 +300,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     } else {
         // ------------------------------------------------------ epilogue
         const int qd = warp & 3;          // row quadrant: rows 32*qd .. 32*qd+31
-        const int half = (warp - 2) >> 2;  // keys [32h, 32h+32), dims [64h, 64h+64)
+        const int half = (warp - 2) >> 2;  // chunk h of each leaf, dims [64h, 64h+64)
         const int r = qd * 32 + lane;     // row of the tile
         const uint32_t tl = tmem_base + ((uint32_t)(qd * 32) << 16);
         const float log2e = 0x1.715476p+0f;
         const int bar_pair = 3 + qd;      // named barrier of this quadrant's two warps
-        float cm0 = 0.f, cm1 = 0.f, cs0 = 0.f, cs1 = 0.f;  // (m, s) of the chunks in buffers 0 and 1
+        float cm0 = 0.f, cm1 = 0.f, cs0 = 0.f, cs1 = 0.f;  // (m, s) of the leaves in O buffers 0 and 1
         uint32_t g0 = 0;
         // A bounded wait that expires makes this warp skip its work from then
         // on; the pair's barrier (OR reduction) then takes both warps out
@@ -270,103 +322,126 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             atc_tile(p, t, qt, bh);
             const int bb = bh / p.heads, hh = bh - bb * p.heads;
             const int i0 = qt * ATC_BM;
-            const int i = i0 + r;                      // this row's query position
-            const int nc = i0 / ATC_CH + 2;            // chunks of the tile
-            const int ncr = (qd < 2) ? nc - 1 : nc;    // chunks of this row's tree
+            const int i = i0 + r;   // this row's query position
+            const int nl = qt + 1;  // leaves of every row of the tile
             // pending summaries: single (its O buffer), 2 (TMEM slot), 3-4 (shared), >= 5 (L2 stack)
             float m1 = 0.f, s1 = 0.f, m2 = 0.f, s2 = 0.f, m34 = 0.f, s34 = 0.f;
             uint32_t single_b = 0;
             int gsp = 0;
-            for (int c = 0; c <= nc; ++c) {
-                if (c < nc) {
-                    // ---------------- softmax of chunk c
-                    const uint32_t g = g0 + c, b = g & 1, ph = (g >> 1) & 1;
+            for (int l = 0; l <= nl; ++l) {
+                if (l < nl) {
+                    // ---------------- softmax of leaf l (this warp: chunk `half`)
+                    const uint32_t g = g0 + l, b = g & 1;
                     uint32_t okw = 1;
-                    if (lane == 0 && !ab) okw = mbar_wait(&s_full[b], ph, abort_flag, lim) ? 1u : 0u;
+                    if (lane == 0 && !ab) okw = mbar_wait(s_full, g & 1, abort_flag, lim) ? 1u : 0u;
                     ab = ab || __shfl_sync(0xffffffffu, okw, 0) == 0;
                     float* xs = sX + (b * 2) * ATC_BM;
+                    float m = -INFINITY;
                     if (!ab) {
                     tc_fence_after();
-                    uint32_t sr[64];
-                    tmem_ld64_nowait(tl + ATC_S_COL + 64 * b, sr);
-                    tmem_wait_ld64(sr);
-                    float m = -INFINITY, sh = 0.0f;
-                    uint32_t pk[16];  // this half's 32 bf16 p, packed in pairs
-                    if (c < ncr) {
-                        const int key0 = ATC_CH * c;
+                    const int key0 = ATC_LEAF * l;
+                    const int kh = key0 + ATC_CH * half;        // first key of this warp's chunk
+                    const int kx = key0 + ATC_CH * (half ^ 1);  // first key of the other chunk
+                    // every key of the leaf precedes every row of the tile: no mask
+                    const bool full = l < nl - 1;
+                    // the other chunk's maximum, on the raw scores: fl(x * scale) is
+                    // non-decreasing in x, so scaling the maximum gives the maximum of
+                    // the scaled scores exactly
+                    {
+                        uint32_t sx[64];
+                        tmem_ld64_nowait(tl + ATC_S_COL + 64 * (half ^ 1), sx);
+                        tmem_wait_ld64(sx);
+                        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                        for (int k = 0; k < 64; ++k) {
-                            const float sv = __fmul_rn(__uint_as_float(sr[k]), p.scale);
-                            sr[k] = __float_as_uint(sv);
-                            if (key0 + k <= i) m = fmaxf(m, sv);
-                        }
-                        const float ml = -__fmul_rn(m, log2e);
-                        const int kh = key0 + 32 * half;  // first key of this half
-#pragma unroll
-                        for (int k2 = 0; k2 < 16; ++k2) {
-                            float pv[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int j = 2 * k2 + e;
-                                const float sj = __uint_as_float(half ? sr[32 + j] : sr[j]);
-                                const float x = ex2_hw(__fmaf_rn(sj, log2e, ml));
-                                pv[e] = (kh + j <= i) ? bf2f(f2bf(x)) : 0.0f;
-                                sh = __fadd_rn(sh, pv[e]);
-                            }
-                            pk[k2] = pack_bf2(pv[0], pv[1]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int k2 = 0; k2 < 16; ++k2) pk[k2] = 0u;
+                        for (int k = 0; k < 64; ++k)
+                            if (full || kx + k <= i) mq[k & 3] = fmaxf(mq[k & 3], __uint_as_float(sx[k]));
+                        m = __fmul_rn(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), p.scale);
                     }
-                    // P row r, keys [32h, 32h+32): four 16-byte chunks at swizzled positions
-                    uint8_t* prow = smem + ATC_OFF_P + b * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+                    uint32_t so[64];
+                    tmem_ld64_nowait(tl + ATC_S_COL + 64 * half, so);
+                    tmem_wait_ld64(so);
+                    float vo[64];
+                    const f2x sc2 = pk2(p.scale, p.scale);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int ch = (4 * half + j) ^ (r & 7);
-                        *reinterpret_cast<uint4*>(prow + ch * 16) =
+                    for (int k = 0; k < 64; k += 2)
+                        upk2(mul2(pk2(__uint_as_float(so[k]), __uint_as_float(so[k + 1])), sc2), vo[k], vo[k + 1]);
+                    {
+                        float mq[4] = {m, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                        for (int k = 0; k < 64; ++k)
+                            if (full || kh + k <= i) mq[k & 3] = fmaxf(mq[k & 3], vo[k]);
+                        m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+                    }
+                    const float ml = -__fmul_rn(m, log2e);
+                    const f2x l2 = pk2(log2e, log2e), ml2 = pk2(ml, ml);
+                    float cq[4] = {0.f, 0.f, 0.f, 0.f};  // sums over the keys k = q (mod 4)
+                    uint32_t pk[32];                     // this chunk's 64 bf16 p, packed in pairs
+#pragma unroll
+                    for (int k2 = 0; k2 < 32; ++k2) {
+                        const int j = 2 * k2;
+                        float y0, y1;
+                        upk2(fma2(pk2(vo[j], vo[j + 1]), l2, ml2), y0, y1);
+                        // both weights rounded to bf16 in one conversion; the sums
+                        // take the rounded values (0 for a key after the row)
+                        uint32_t w = pack_bf2(ex2_hw(y0), ex2_hw(y1));
+                        if (!full) {
+                            if (kh + j > i) w &= 0xffff0000u;
+                            if (kh + j + 1 > i) w &= 0x0000ffffu;
+                        }
+                        pk[k2] = w;
+                        cq[j & 3] = __fadd_rn(cq[j & 3], __uint_as_float(w << 16));
+                        cq[(j + 1) & 3] = __fadd_rn(cq[(j + 1) & 3], __uint_as_float(w & 0xffff0000u));
+                    }
+                    // P of the previous leaf is read by its P V MMA, which is issued
+                    // after the scores of this leaf: wait for that MMA before
+                    // overwriting P (the same phase the tree step waits for later)
+                    if (g >= 1) {
+                        const uint32_t gp = g - 1;
+                        uint32_t okp = 1;
+                        if (lane == 0) okp = mbar_wait(&o_full[gp & 1], (gp >> 1) & 1, abort_flag, lim) ? 1u : 0u;
+                        ab = __shfl_sync(0xffffffffu, okp, 0) == 0;
+                    }
+                    if (!ab) {
+                    // P row r of this chunk: eight 16-byte pieces at swizzled positions
+                    uint8_t* prow = smem + ATC_OFF_P + half * 16384 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4*>(prow + ((j ^ (r & 7)) * 16)) =
                             make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-                    }
-                    xs[half * ATC_BM + r] = sh;
-                    if (b) cm1 = m; else cm0 = m;
+                    xs[half * ATC_BM + r] = __fadd_rn(__fadd_rn(cq[0], cq[1]), __fadd_rn(cq[2], cq[3]));
                     fence_proxy_async_smem();
                     tc_fence_before();
                     }
+                    }
                     if (named_barrier_or(bar_pair, 64, ab)) goto epi_out;
-                    const float s_c = __fadd_rn(xs[r], xs[ATC_BM + r]);  // keys 0..31, then 32..63
-                    if (b) cs1 = s_c; else cs0 = s_c;
+                    const float s_l = __fadd_rn(xs[r], xs[ATC_BM + r]);  // keys 0..63, then 64..127
+                    if (b) { cm1 = m; cs1 = s_l; } else { cm0 = m; cs0 = s_l; }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&p_full[b]);
+                    if (lane == 0) mbar_arrive(p_full);
                 }
-                if (c >= 1) {
-                    // ---------------- tree step of chunk c - 1
-                    const int c1 = c - 1;
-                    const uint32_t g = g0 + c1, b = g & 1, ph = (g >> 1) & 1;
+                if (l >= 1) {
+                    // ---------------- tree step of leaf l - 1
+                    const int l1 = l - 1;
+                    const uint32_t g = g0 + l1, b = g & 1, ph = (g >> 1) & 1;
                     uint32_t okw = 1;
                     if (lane == 0 && !ab) okw = mbar_wait(&o_full[b], ph, abort_flag, lim) ? 1u : 0u;
                     ab = ab || __shfl_sync(0xffffffffu, okw, 0) == 0;
                     if (ab) continue;  // left at the pair's next barrier (or at the end)
                     tc_fence_after();
-                    if (c1 >= ncr) {  // past this row's last chunk: release the buffer only
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&o_empty[b]);
-                        continue;
-                    }
-                    const uint32_t code = encode_leaf_ops(leaf_ops(ncr, c1));
+                    const uint32_t code = encode_leaf_ops(leaf_ops(nl, l1));
                     const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
                     const int nb = (code >> 3) & 31;
                     const int cls = (code >> 8) & 3;
                     const bool final_ = (code >> 10) & 1;
                     const uint32_t oc = tl + ATC_O_COL + 128 * b + 64 * half;  // this half's 64 dims
                     const float cmb = b ? cm1 : cm0, csb = b ? cs1 : cs0;
-                    if (!final_ && cls == 0) {  // a single chunk waits in its O buffer
+                    if (!final_ && cls == 0) {  // a single leaf waits in its O buffer
                         single_b = b;
                         m1 = cmb;
                         s1 = csb;
                         continue;
                     }
-                    // phase 1: the chunk (and the single it pops) into v; release the buffers
+                    // phase 1: the leaf (and the single it pops) into v; release the buffers
                     float v[2][32];
                     float vm = cmb, vs = csb;
                     if (p1) {
@@ -376,16 +451,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
 #pragma unroll
                         for (int cc = 0; cc < 2; ++cc) {
                             uint32_t ra[32], rb[32];
-                            tmem_ld32_nowait(os + 32 * cc, ra);
-                            tmem_ld32_nowait(oc + 32 * cc, rb);
-                            tmem_wait_ld(ra);
-                            tie32(rb);
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                v[cc][k] = __fadd_rn(__fmul_rn(__uint_as_float(ra[k]), ea),
-                                                     __fmul_rn(__uint_as_float(rb[k]), eb));
+                            tmem_ld32x2(os + 32 * cc, ra, oc + 32 * cc, rb);
+                            atc_comb(v[cc], ra, ea, rb, eb);
                         }
-                        vs = __fadd_rn(__fmul_rn(s1, ea), __fmul_rn(vs, eb));
+                        vs = atc_comb1(s1, ea, vs, eb);
                         vm = M;
                     } else {
                         uint32_t ro[64];
@@ -411,11 +480,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         for (int cc = 0; cc < 2; ++cc) {
                             float w[32];
                             tmem_ld32(tl + ATC_SLOT_COL + 64 * half + 32 * cc, w);
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                v[cc][k] = __fadd_rn(__fmul_rn(w[k], ea), __fmul_rn(v[cc][k], eb));
+                            atc_comb(v[cc], w, ea, v[cc], eb);
                         }
-                        vs = __fadd_rn(__fmul_rn(s2, ea), __fmul_rn(vs, eb));
+                        vs = atc_comb1(s2, ea, vs, eb);
                         vm = M;
                     }
                     if (pm) {
@@ -425,11 +492,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         for (int cc = 0; cc < 2; ++cc) {
                             float w[32];
                             atc_ld32(sSlot, 2 * half + cc, r, w);
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                v[cc][k] = __fadd_rn(__fmul_rn(w[k], ea), __fmul_rn(v[cc][k], eb));
+                            atc_comb(v[cc], w, ea, v[cc], eb);
                         }
-                        vs = __fadd_rn(__fmul_rn(s34, ea), __fmul_rn(vs, eb));
+                        vs = atc_comb1(s34, ea, vs, eb);
                         vm = M;
                     }
                     for (int q = 0; q < nb; ++q) {
@@ -441,11 +506,9 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         for (int cc = 0; cc < 2; ++cc) {
                             float w[32];
                             atc_ld32(sl, 2 * half + cc, r, w);
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                v[cc][k] = __fadd_rn(__fmul_rn(w[k], ea), __fmul_rn(v[cc][k], eb));
+                            atc_comb(v[cc], w, ea, v[cc], eb);
                         }
-                        vs = __fadd_rn(__fmul_rn(stk_s[slot], ea), __fmul_rn(vs, eb));
+                        vs = atc_comb1(stk_s[slot], ea, vs, eb);
                         vm = M;
                     }
                     gsp -= nb;
@@ -484,7 +547,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     }
                 }
             }
-            g0 += nc;
+            g0 += nl;
         }
     epi_out:;
     }

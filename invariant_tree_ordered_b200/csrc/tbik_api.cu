@@ -782,14 +782,14 @@ struct AttTcPlan {
 
 tbik_status plan_attention_tc(int batch, int seq, int heads, int head_dim, int chunk, int sms, AttTcPlan& p) {
     if (batch < 0 || seq < 0 || heads <= 0) return TBIK_ERR_ARG;
-    if (head_dim != ATC_HD || chunk != ATC_CH || seq % ATC_BM || seq > 256 * ATC_CH) return TBIK_ERR_SHAPE;
+    if (head_dim != ATC_HD || chunk != ATC_LEAF || seq % ATC_BM || seq > 128 * ATC_LEAF) return TBIK_ERR_SHAPE;
     const long long tiles = (long long)batch * heads * (seq / ATC_BM);
     if (tiles > 0x7fffffffLL) return TBIK_ERR_SHAPE;
     p.tiles = (int)tiles;
     p.grid = p.tiles < sms ? p.tiles : sms;
-    // the deepest L2 stack over the chunk trees of every row length
+    // the deepest L2 stack over the leaf trees of every row length
     p.gs = 0;
-    for (int n = 1; n <= seq / ATC_CH; ++n) {
+    for (int n = 1; n <= seq / ATC_LEAF; ++n) {
         const int g = max_big_pending(n);
         if (g > p.gs) p.gs = g;
     }

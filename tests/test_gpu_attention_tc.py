@@ -1,8 +1,9 @@
 """Tensor-core mode of the tree-ordered causal attention (tbik_attention_tc).
 
-Not bit-exact to the oracle (the dot products run on the tensor cores and the
-softmax weights are rounded to bf16 before P V), so it is checked against the
-binary64 definition with a bound derived from that arithmetic:
+Not bit-exact to the oracle (the dot products run on the tensor cores, the
+keys are reduced in 128-key leaves and the softmax weights are rounded to bf16
+before P V), so it is checked against the binary64 definition with a bound
+derived from that arithmetic:
   the weights of a row are p_j rounded to bf16 (relative error <= 2^-9) and
   the sum s uses the same rounded weights, so the output is an exact weighted
   average of the v_j with each normalised weight moved by at most about
@@ -39,9 +40,10 @@ def within_bound(got, ref, v):
     return np.abs(got - ref) <= 2.0 ** -7 * vmax + 2.0 ** -8 * np.abs(ref)
 
 
-@pytest.mark.parametrize("B,S,NH", [(1, 128, 1), (2, 256, 3), (1, 1024, 2), (1, 2048, 1)])
+@pytest.mark.parametrize("B,S,NH", [(1, 128, 1), (2, 256, 3), (1, 1024, 2), (1, 2048, 1), (1, 4096, 1)])
 def test_tc_attention_vs_binary64(B, S, NH):
-    # 1024 and 2048 positions: 16 and 32 chunks, so pending summaries reach the L2 stack
+    # 1024, 2048 and 4096 positions: 8, 16 and 32 leaves; from 2048 on, pending
+    # summaries of >= 5 leaves (8, then 16 and 8) use the L2 stack
     q, k, v = qkv(500 + S, (B, S, NH, 128))
     got = f32(host_bits16(tbik.attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), tc=True)))
     assert tbik.get_error() == tbik.TBIK_OK
@@ -82,7 +84,7 @@ def test_tc_attention_batch_and_head_split_invariance():
 
 
 def test_tc_attention_repeat_runs_and_batch_subset_at_2048():
-    """Several 2048-position tiles per CTA (persistent grid) with chunk trees
+    """Several 2048-position tiles per CTA (persistent grid) with leaf trees
     deep enough for the L2 stack: repeated calls give the same bits, and so
     does one sequence alone."""
     B, S, NH = 4, 2048, 16
@@ -101,14 +103,16 @@ def test_tc_attention_argument_errors():
     s = torch.cuda.current_stream().cuda_stream
     x = torch.zeros((1, 256, 2, 128), dtype=torch.bfloat16, device="cuda")
     p = x.data_ptr()
-    assert lib.tbik_attention_tc(p, p, p, p, 1, 200, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_SHAPE  # seq % 128
-    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 64, 64, None, 0, s) == tbik.TBIK_ERR_SHAPE   # head_dim
-    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 128, 32, None, 0, s) == tbik.TBIK_ERR_SHAPE  # chunk
-    assert lib.tbik_attention_tc(p + 2, p, p, p, 1, 256, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_ALIGN
-    assert lib.tbik_attention_tc_workspace(1, 200, 2, 128, 64) == (1 << 64) - 1
-    need = lib.tbik_attention_tc_workspace(1, 2048, 2, 128, 64)
-    assert need > 0  # 32 chunks: the tree has pending values of >= 5 chunks
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 200, 2, 128, 128, None, 0, s) == tbik.TBIK_ERR_SHAPE  # seq % 128
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 64, 128, None, 0, s) == tbik.TBIK_ERR_SHAPE   # head_dim
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_SHAPE   # leaf
+    assert lib.tbik_attention_tc(p, p, p, p, 1, 256, 2, 128, 32, None, 0, s) == tbik.TBIK_ERR_SHAPE   # leaf
+    assert lib.tbik_attention_tc(p + 2, p, p, p, 1, 256, 2, 128, 128, None, 0, s) == tbik.TBIK_ERR_ALIGN
+    assert lib.tbik_attention_tc_workspace(1, 200, 2, 128, 128) == (1 << 64) - 1
+    assert lib.tbik_attention_tc_workspace(1, 256, 2, 128, 128) == 0  # 2 leaves: nothing pending in L2
+    need = lib.tbik_attention_tc_workspace(1, 2048, 2, 128, 128)
+    assert need > 0  # 16 leaves: the tree has a pending value of 8 leaves
     big = torch.zeros((1, 2048, 2, 128), dtype=torch.bfloat16, device="cuda")
     b = big.data_ptr()
-    assert lib.tbik_attention_tc(b, b, b, b, 1, 2048, 2, 128, 64, None, 0, s) == tbik.TBIK_ERR_WORKSPACE
+    assert lib.tbik_attention_tc(b, b, b, b, 1, 2048, 2, 128, 128, None, 0, s) == tbik.TBIK_ERR_WORKSPACE
     assert tbik.get_error() == tbik.TBIK_OK
