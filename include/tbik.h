@@ -258,7 +258,7 @@ TBIK_API tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const 
  * leaf summaries combined by TREE: M = max, e = exp(m - M) (the exp
  * specification; 1 for the side holding M), s = fma(s', e', fl(s*e)),
  * o = fma(o', e', fl(o*e)) (left operand's product rounded);
- * out[d] = bf16(o[d] / s).  Each output row depends only on its query and
+ * out[d] = bf16(o[d] * fl(1/s)).  Each output row depends only on its query and
  * the keys/values at positions <= i, so it is bitwise the same for any batch
  * composition and head split; it is checked against the binary64 definition
  * by tolerance.

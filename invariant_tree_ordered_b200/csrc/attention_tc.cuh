@@ -19,7 +19,7 @@
 //   combine M = max, e = exp(m - M) by the library's exp specification (1 for
 //           the side holding M), s = fma(s', e', fl(s*e)),
 //           o = fma(o', e', fl(o*e)) (the left operand's product rounded);
-//   output  bf16(o[d] / s).
+//   output  bf16(o[d] * fl(1/s)).
 // A row's result depends only on its query, the keys and values at positions
 // <= i and its fixed leaf tree, never on the batch composition, the other
 // rows of its tile or how heads are split across devices.
@@ -352,10 +352,18 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         tmem_ld64_nowait(tl + ATC_S_COL + 64 * (half ^ 1), sx);
                         tmem_wait_ld64(sx);
                         float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                        if (full) {
 #pragma unroll
-                        for (int k = 0; k < 64; ++k)
-                            if (full || kx + k <= i) mq[k & 3] = fmaxf(mq[k & 3], __uint_as_float(sx[k]));
-                        m = __fmul_rn(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), p.scale);
+                            for (int k = 0; k < 64; k += 8)
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    mq[q] = fmax3(mq[q], __uint_as_float(sx[k + 2 * q]), __uint_as_float(sx[k + 2 * q + 1]));
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 64; ++k)
+                                if (kx + k <= i) mq[k & 3] = fmaxf(mq[k & 3], __uint_as_float(sx[k]));
+                        }
+                        m = __fmul_rn(fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]), p.scale);
                     }
                     uint32_t so[64];
                     tmem_ld64_nowait(tl + ATC_S_COL + 64 * half, so);
@@ -367,30 +375,48 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         upk2(mul2(pk2(__uint_as_float(so[k]), __uint_as_float(so[k + 1])), sc2), vo[k], vo[k + 1]);
                     {
                         float mq[4] = {m, -INFINITY, -INFINITY, -INFINITY};
+                        if (full) {
 #pragma unroll
-                        for (int k = 0; k < 64; ++k)
-                            if (full || kh + k <= i) mq[k & 3] = fmaxf(mq[k & 3], vo[k]);
-                        m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+                            for (int k = 0; k < 64; k += 8)
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], vo[k + 2 * q], vo[k + 2 * q + 1]);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 64; ++k)
+                                if (kh + k <= i) mq[k & 3] = fmaxf(mq[k & 3], vo[k]);
+                        }
+                        m = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]);
                     }
                     const float ml = -__fmul_rn(m, log2e);
                     const f2x l2 = pk2(log2e, log2e), ml2 = pk2(ml, ml);
                     float cq[4] = {0.f, 0.f, 0.f, 0.f};  // sums over the keys k = q (mod 4)
                     uint32_t pk[32];                     // this chunk's 64 bf16 p, packed in pairs
+                    // both weights of a pair rounded to bf16 in one conversion; the
+                    // sums take the rounded values (0 for a key after the row)
+                    if (full) {
 #pragma unroll
-                    for (int k2 = 0; k2 < 32; ++k2) {
-                        const int j = 2 * k2;
-                        float y0, y1;
-                        upk2(fma2(pk2(vo[j], vo[j + 1]), l2, ml2), y0, y1);
-                        // both weights rounded to bf16 in one conversion; the sums
-                        // take the rounded values (0 for a key after the row)
-                        uint32_t w = pack_bf2(ex2_hw(y0), ex2_hw(y1));
-                        if (!full) {
+                        for (int k2 = 0; k2 < 32; ++k2) {
+                            const int j = 2 * k2;
+                            float y0, y1;
+                            upk2(fma2(pk2(vo[j], vo[j + 1]), l2, ml2), y0, y1);
+                            const uint32_t w = pack_bf2(ex2_hw(y0), ex2_hw(y1));
+                            pk[k2] = w;
+                            cq[j & 3] = __fadd_rn(cq[j & 3], __uint_as_float(w << 16));
+                            cq[(j + 1) & 3] = __fadd_rn(cq[(j + 1) & 3], __uint_as_float(w & 0xffff0000u));
+                        }
+                    } else {
+#pragma unroll
+                        for (int k2 = 0; k2 < 32; ++k2) {
+                            const int j = 2 * k2;
+                            float y0, y1;
+                            upk2(fma2(pk2(vo[j], vo[j + 1]), l2, ml2), y0, y1);
+                            uint32_t w = pack_bf2(ex2_hw(y0), ex2_hw(y1));
                             if (kh + j > i) w &= 0xffff0000u;
                             if (kh + j + 1 > i) w &= 0x0000ffffu;
+                            pk[k2] = w;
+                            cq[j & 3] = __fadd_rn(cq[j & 3], __uint_as_float(w << 16));
+                            cq[(j + 1) & 3] = __fadd_rn(cq[(j + 1) & 3], __uint_as_float(w & 0xffff0000u));
                         }
-                        pk[k2] = w;
-                        cq[j & 3] = __fadd_rn(cq[j & 3], __uint_as_float(w << 16));
-                        cq[(j + 1) & 3] = __fadd_rn(cq[(j + 1) & 3], __uint_as_float(w & 0xffff0000u));
                     }
                     // P of the previous leaf is read by its P V MMA, which is issued
                     // after the scores of this leaf: wait for that MMA before
@@ -533,15 +559,16 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                             ++gsp;
                         }
                     } else if (i < p.seq) {
-                        // out[b][i][h][64h .. 64h+63] = bf16(o / s)
+                        // out[b][i][h][64h .. 64h+63] = bf16(o * fl(1/s))
                         uint16_t* orow = p.out + (((size_t)bb * p.seq + i) * p.heads + hh) * ATC_HD + 64 * half;
+                        const float rs = __frcp_rn(vs);
 #pragma unroll
                         for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
                             for (int q8 = 0; q8 < 4; ++q8) {
                                 float o8[8];
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) o8[e] = __fdiv_rn(v[cc][8 * q8 + e], vs);
+                                for (int e = 0; e < 8; ++e) o8[e] = __fmul_rn(v[cc][8 * q8 + e], rs);
                                 *reinterpret_cast<uint4*>(orow + 32 * cc + 8 * q8) = pack8(o8);
                             }
                     }

@@ -106,6 +106,14 @@ __device__ __forceinline__ float swiglu1(float g, float u) {
     return __fmul_rn(sg, u);
 }
 
+// Three-input maximum (max.f32 with three sources, sm_100): the largest of a,
+// b, c, exactly (no rounding), NaN inputs ignored as by fmaxf.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // ---- two lanes per instruction (packed f32x2 add / mul / fma, sm_100) ------
 // Each lane of a packed operation is the IEEE round-to-nearest-even result of
 // the scalar operation on that lane, so the paired forms below return exactly
