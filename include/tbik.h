@@ -255,8 +255,8 @@ TBIK_API tbik_status tbik_attention(const uint16_t* q, const uint16_t* k, const 
  *   p_j (keys 0..63 and 64..127 of the leaf, each (c0 + c1) + (c2 + c3) with
  *   c_q the ascending sum over its keys k = q mod 4); o = sum of p_j * v_j
  *   on the tensor cores;
- * leaf summaries combined by TREE: M = max, e = exp(m - M) (the exp
- * specification; 1 for the side holding M), s = fma(s', e', fl(s*e)),
+ * leaf summaries combined by TREE: M = max, e = 2^(fl(m - M)*log2e) (the
+ * hardware exponential; 1 for the side holding M), s = fma(s', e', fl(s*e)),
  * o = fma(o', e', fl(o*e)) (left operand's product rounded);
  * out[d] = bf16(o[d] * fl(1/s)).  Each output row depends only on its query and
  * the keys/values at positions <= i, so it is bitwise the same for any batch

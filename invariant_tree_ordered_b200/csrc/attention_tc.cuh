@@ -16,8 +16,8 @@
 //           (c0 + c1) + (c2 + c3) with c_q the ascending sum over the keys
 //           k = q (mod 4) of that half;
 //           o = P V on the tensor cores (the bf16 p_j as A, V as B, K = 128);
-//   combine M = max, e = exp(m - M) by the library's exp specification (1 for
-//           the side holding M), s = fma(s', e', fl(s*e)),
+//   combine M = max, e = 2^(fl(m - M)*log2e) by the hardware exponential (1
+//           for the side holding M), s = fma(s', e', fl(s*e)),
 //           o = fma(o', e', fl(o*e)) (the left operand's product rounded);
 //   output  bf16(o[d] * fl(1/s)).
 // A row's result depends only on its query, the keys and values at positions
@@ -123,12 +123,14 @@ __device__ __forceinline__ float atc_comb1(float a, float ea, float b, float eb)
 }
 
 // Combine factors of two summaries (a is the left operand): M and the two
-// exponentials of the exact mode's rule.
+// exponentials e = 2^(fl(m - M) * log2e) by the hardware exponential (1 for
+// the side holding M).
 __device__ __forceinline__ void atc_factors(float am, float bm, float& M, float& ea, float& eb) {
+    const float log2e = 0x1.715476p+0f;
     M = (bm > am) ? bm : am;
     const bool finite = M != INFINITY;
-    ea = (finite && am == M) ? 1.0f : exp_spec(__fsub_rn(am, M));
-    eb = (finite && bm == M) ? 1.0f : exp_spec(__fsub_rn(bm, M));
+    ea = (finite && am == M) ? 1.0f : ex2_hw(__fmul_rn(__fsub_rn(am, M), log2e));
+    eb = (finite && bm == M) ? 1.0f : ex2_hw(__fmul_rn(__fsub_rn(bm, M), log2e));
 }
 
 // Query tile t (longest first): position block qt and (batch, head) bh.
