@@ -257,23 +257,11 @@ __device__ __forceinline__ void logprob_leaf_stats(const TcParams& p, float (&v)
                 if (k + 32 >= ncol) v[1][k] = -INFINITY;
             }
         }
-        // the maximum (exact in any order): four running maxima of three inputs
-        float mq[4];
+        float m = v[0][0];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mq[q] = fmax3(v[0][q], v[0][4 + q], v[0][8 + q]);
+        for (int k = 1; k < 32; ++k) m = fmaxf(m, v[0][k]);
 #pragma unroll
-        for (int k = 12; k < 28; k += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], v[0][k + q], v[0][k + 4 + q]);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], v[0][28 + q], v[1][q]);
-#pragma unroll
-        for (int k = 4; k < 28; k += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], v[1][k + q], v[1][k + 4 + q]);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) mq[q] = fmaxf(mq[q], v[1][28 + q]);
-        const float m = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]);
+        for (int k = 0; k < 32; ++k) m = fmaxf(m, v[1][k]);
         const float log2e = 0x1.715476p+0f;
         const float ml = -__fmul_rn(m, log2e);
         float s0 = 0.0f, s1 = 0.0f;
