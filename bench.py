@@ -458,6 +458,27 @@ def run_tbik(args):
     except Exception as e:  # noqa: BLE001
         exact = {"error": f"{type(e).__name__}: {e}"[:300]}
         torch.cuda.synchronize()
+    try:  # the backward GEMMs of the down_proj (an extra measurement): dA = dY B^T with B read as [N', K']
+        # (K' = 4096 in leaves of 256), dB = A^T dY reducing over the 4096 tokens in leaves of 256
+        dY = hid  # any bf16 [M, 4096] gradient of the output
+        dA = torch.empty((M_TOK, F), dtype=torch.float32, device=dev)
+        dB = torch.empty((F, H), dtype=torch.float32, device=dev)
+        At = torch.empty((F, M_TOK), dtype=torch.bfloat16, device=dev)
+        wdx = torch.empty(max(tbik.gemm_workspace(M_TOK, F, H, 1, LEAF, tbik.TC | tbik.B_NK), 256),
+                          dtype=torch.uint8, device=dev)
+        wdw = torch.empty(max(tbik.gemm_workspace(F, H, M_TOK, 1, LEAF, tbik.TC), 256), dtype=torch.uint8,
+                          device=dev)
+        dx_ms = avg_ms(lambda: tbik.gemm(dY, B, T=1, leaf=LEAF, tc=True, b_nk=True, out=dA, workspace=wdx))
+        tr_ms = avg_ms(lambda: tbik.transpose(A, out=At))
+        dw_ms = avg_ms(lambda: tbik.gemm(At, dY, T=1, leaf=LEAF, tc=True, out=dB, workspace=wdw))
+        backward = {"dA_ms": dx_ms, "dA_tflops": GEMM_FLOP / (dx_ms * 1e-3) / 1e12,
+                    "dB_gemm_ms": dw_ms, "dB_gemm_tflops": GEMM_FLOP / (dw_ms * 1e-3) / 1e12,
+                    "transpose_A_ms": tr_ms, "transpose_A_gbs": 2 * M_TOK * F * 2 / (tr_ms * 1e-3) / 1e9,
+                    "fp32_outputs": True, "status": int(tbik.get_error(stream))}
+        del dA, dB, At, wdx, wdw
+    except Exception as e:  # noqa: BLE001
+        backward = {"error": f"{type(e).__name__}: {e}"[:300]}
+        torch.cuda.synchronize()
     pk = peaks()
     red8k = reductions_component(8192, dev, stream, gamma, table, pk["hbm"])
     dec = None
@@ -501,6 +522,7 @@ def run_tbik(args):
             "ms": comp_ms,
             "reductions_8192_tokens": dict(red8k, copy_peak_gbs=pk["hbm"], copy_peak_source=pk["src"]),
             "exact_mode": exact,
+            "backward_down_proj_tc": backward,
             "overhead_vs_noninv": {"gemm": g_inv / g_non - 1.0, "logprob": l_inv / l_non - 1.0,
                                    "gemm_ms": [g_inv, g_non], "logprob_ms": [l_inv, l_non]},
             "decoder_e2e": dec,

@@ -420,9 +420,10 @@ TBIK_API tbik_status tbik_get_error(void* stream);
 
 /*
  * Test hooks.  flags: TBIK_DEBUG_WITHHOLD_ACC_ARRIVE makes the tensor-core GEMM
- * epilogue withhold its "accumulator drained" arrive, so the MMA issuer's
- * bounded wait expires: the kernel must record TBIK_ERR_TIMEOUT, drain its own
- * copies in flight, free its TMEM and return.  TBIK_DEBUG_TILE128 runs every
+ * epilogue withhold its "accumulator drained" arrive (and the tensor-core
+ * attention's epilogue its "P written" arrive), so the MMA issuer's bounded
+ * wait expires: the kernel must record TBIK_ERR_TIMEOUT, drain its own copies
+ * in flight, free its TMEM and return.  TBIK_DEBUG_TILE128 runs every
  * tensor-core GEMM on the 128-column pair tile (normally 192 columns unless B
  * is [K,N] with N <= 128), so that tests can compare the two tile designs on
  * the same operands.  wait_limit_ns bounds every device-side wait (0 keeps the

@@ -82,6 +82,7 @@ struct AttTcParams {
     float* stack;      // [gridDim.x][gs][ATC_VAL_FLOATS]: o of the pending >= 5-leaf values
     int gs;
     unsigned long long wait_cycles;
+    unsigned debug;    // TBIK_DEBUG_* test hooks
 };
 
 // 32 dims (chunk c of 4) of one row of a pending value, [dim/4][row][4] layout.
@@ -445,7 +446,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     const float s_l = __fadd_rn(xs[r], xs[ATC_BM + r]);  // keys 0..63, then 64..127
                     if (b) { cm1 = m; cs1 = s_l; } else { cm0 = m; cs0 = s_l; }
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(p_full);
+                    if (lane == 0 && !(p.debug & TBIK_DEBUG_WITHHOLD_ACC_ARRIVE)) mbar_arrive(p_full);
                 }
                 if (l >= 1) {
                     // ---------------- tree step of leaf l - 1

@@ -836,6 +836,7 @@ tbik_status tbik_attention_tc(const uint16_t* q, const uint16_t* k, const uint16
     prm.stack = reinterpret_cast<float*>(workspace);
     prm.gs = p.gs;
     prm.wait_cycles = wait_cycles(info);
+    prm.debug = g_debug_flags;
     attention_tc_kernel<<<p.grid, ATC_THREADS, ATC_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(tq, tk, tv,
                                                                                                            prm);
     return launch_status();

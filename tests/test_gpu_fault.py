@@ -46,3 +46,31 @@ def test_withheld_arrive_times_out_and_context_survives(b_nk, tile128):
     assert tbik.get_error() == tbik.TBIK_OK
     assert np.array_equal(u32(again), u32(good))
     assert torch.cuda.synchronize() is None
+
+
+def test_attention_withheld_arrive_times_out_and_context_survives():
+    """The tensor-core attention with its epilogue's "P written" arrive
+    withheld: the MMA issuer's bounded wait expires, the producer and the
+    epilogue warps leave through their own bounded waits (the pair barrier
+    takes both warps of a quadrant out together), the copies in flight land
+    and TMEM is freed; the next call gives the same bits as before."""
+    B, S, NH = 2, 1024, 4
+    g = torch.Generator(device="cuda").manual_seed(9)
+    q, k, v = [torch.randn(B, S, NH, 128, device="cuda", generator=g).to(torch.bfloat16) for _ in range(3)]
+    try:
+        tbik.debug_set(0, 0)
+        good = tbik.attention(q, k, v, tc=True).view(torch.int16).cpu().numpy()
+        assert tbik.get_error() == tbik.TBIK_OK
+        tbik.debug_set(tbik.DEBUG_WITHHOLD_ACC_ARRIVE, 50_000_000)  # 50 ms per wait
+        t0 = time.time()
+        tbik.attention(q, k, v, tc=True)
+        status = tbik.get_error()
+        elapsed = time.time() - t0
+        tbik.debug_set(0, 0)
+        again = tbik.attention(q, k, v, tc=True).view(torch.int16).cpu().numpy()
+    finally:
+        tbik.debug_set(0, 0)
+    assert status == tbik.TBIK_ERR_TIMEOUT
+    assert elapsed < 10.0
+    assert tbik.get_error() == tbik.TBIK_OK
+    assert np.array_equal(again, good)
