@@ -233,7 +233,41 @@ __global__ void embedding_kernel(const int32_t* __restrict__ ids, const uint16_t
     }
 }
 
-// bf16 transpose through a 32 x 33 shared-memory tile (block 32 x 8).
+// bf16 transpose of rows, cols multiples of 8 with 16-byte aligned rows: a
+// 64 x 64 tile per CTA of 256 threads, read as 16-byte vectors of 8 columns
+// into shared memory (rows padded to 72 elements, so the 16-byte stores and
+// the column reads are free of bank conflicts) and written as 32-byte runs of
+// 16 consecutive rows of one column (full sectors).
+__global__ void __launch_bounds__(256) transpose_vec_kernel(const uint16_t* __restrict__ in, uint16_t* out,
+                                                            int rows, int cols) {
+    __shared__ __align__(16) uint16_t tile[64][72];
+    const int tid = threadIdx.x;
+    const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+        const int r = (tid >> 3) + 32 * pass, v = tid & 7;  // tile row, 8-column vector
+        if (r0 + r < rows && c0 + 8 * v < cols)
+            *reinterpret_cast<uint4*>(&tile[r][8 * v]) =
+                __ldg(reinterpret_cast<const uint4*>(in + (size_t)(r0 + r) * cols + c0) + v);
+    }
+    __syncthreads();
+    const int c = tid & 63, q = tid >> 6;  // output row c0 + c, input rows r0 + 16q .. r0 + 16q + 15
+    if (c0 + c < cols) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int rb = 16 * q + 8 * h;
+            if (r0 + rb < rows) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    w[e] = (uint32_t)tile[rb + 2 * e][c] | ((uint32_t)tile[rb + 2 * e + 1][c] << 16);
+                *reinterpret_cast<uint4*>(out + (size_t)(c0 + c) * rows + r0 + rb) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+    }
+}
+
+// bf16 transpose through a 32 x 33 shared-memory tile (block 32 x 8), any shape.
 __global__ void transpose_kernel(const uint16_t* __restrict__ in, uint16_t* out, int rows, int cols) {
     __shared__ uint16_t tile[32][33];
     const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;

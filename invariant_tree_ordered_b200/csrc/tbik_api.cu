@@ -851,6 +851,11 @@ tbik_status tbik_transpose(const uint16_t* in, uint16_t* out, int rows, int cols
     if (rows == 0 || cols == 0) return TBIK_OK;
     if (!in || !out) return TBIK_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 1u) return TBIK_ERR_ALIGN;
+    if (rows % 8 == 0 && cols % 8 == 0 && aligned16(in) && aligned16(out) && (rows + 63) / 64 <= 65535) {
+        transpose_vec_kernel<<<dim3((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64)), 256, 0,
+                               reinterpret_cast<cudaStream_t>(stream)>>>(in, out, rows, cols);
+        return launch_status();
+    }
     const long long gx = (cols + 31) / 32, gy = (rows + 31) / 32;
     if (gy > 65535) return TBIK_ERR_SHAPE;
     transpose_kernel<<<dim3((unsigned)gx, (unsigned)gy), dim3(32, 8), 0, reinterpret_cast<cudaStream_t>(stream)>>>(

@@ -19,7 +19,9 @@ import invariant_tree_ordered_b200 as tbik  # noqa: E402
 
 
 def test_transpose_exact():
-    for rows, cols in ((1, 1), (33, 70), (256, 128), (1000, 37)):
+    # (256, 128), (200, 136), (64, 8), (8, 640): the 16-byte vector path (both
+    # sizes multiples of 8), full and ragged 64 x 64 tiles; the rest element-wise
+    for rows, cols in ((1, 1), (33, 70), (256, 128), (1000, 37), (200, 136), (64, 8), (8, 640)):
         x = synth.normal_bf16(800 + rows, (rows, cols))
         got = host_bits16(tbik.transpose(dev_bf16(x)))
         assert np.array_equal(got, np.ascontiguousarray(x.T)), (rows, cols)
