@@ -175,6 +175,21 @@ __device__ __forceinline__ void scratch_st(float* base, int c, int row, const fl
             make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
+// A push onto the L2 stack (the layout of scratch_st), with an evict-last L2
+// policy: the lines are read back by the pop a few leaves later, and keeping
+// them resident avoids their write-back and re-read (measured 1-2 % faster).
+__device__ __forceinline__ void stack_push32(float* base, int c, int row, const float (&v)[32]) {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        float* a = base + ((size_t)(c * 8 + q) * TC_BM + row) * 4;
+        asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(a), "f"(v[4 * q]),
+                     "f"(v[4 * q + 1]), "f"(v[4 * q + 2]), "f"(v[4 * q + 3]), "l"(pol)
+                     : "memory");
+    }
+}
+
 // 16 columns (chunk q) of one row of a slot, as raw bits (the layout of scratch_ld).
 __device__ __forceinline__ void scratch_ld16(const float* base, int q, int row, uint32_t (&w)[16]) {
 #pragma unroll
@@ -620,7 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
                         else if (cls == 2)
                             scratch_st(sSlot, c, rt, v[cc]);
                         else
-                            scratch_st(scratch_slot<BN>(p, g_after), c, rt, v[cc]);
+                            stack_push32(scratch_slot<BN>(p, g_after), c, rt, v[cc]);
                     }
                     if (cls == 1) tmem_wait_st();
                 } else if (EPI == EPI_TREE && p.swiglu) {
@@ -801,7 +816,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
                         }
                     } else if (cls == 3) {
 #pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) scratch_st(scratch_slot<BN>(p, g_after), grp * 2 + cc, rt, R[cc]);
+                        for (int cc = 0; cc < 2; ++cc) stack_push32(scratch_slot<BN>(p, g_after), grp * 2 + cc, rt, R[cc]);
                     }
                 } else if (EPI == EPI_TREE && p.swiglu) {
                     // gate features f0..f0+31 (R[0]) and their up values (R[1])
