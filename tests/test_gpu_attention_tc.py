@@ -116,3 +116,19 @@ def test_tc_attention_argument_errors():
     b = big.data_ptr()
     assert lib.tbik_attention_tc(b, b, b, b, 1, 2048, 2, 128, 128, None, 0, s) == tbik.TBIK_ERR_WORKSPACE
     assert tbik.get_error() == tbik.TBIK_OK
+
+
+@pytest.mark.parametrize("tc", [True, False])
+def test_prefix_invariance_longer_sequence(tc):
+    """Row i attends to keys <= i through its fixed leaf tree, so its bits do
+    not depend on how long the sequence is: the first 1024 positions of a
+    2048-position sequence equal the same 1024 positions computed alone (the
+    consistency a serving loop needs between a prefill and a longer one)."""
+    B, S, NH = 2, 2048, 4
+    g = torch.Generator(device="cuda").manual_seed(11)
+    q, k, v = [torch.randn(B, S, NH, 128, device="cuda", generator=g).to(torch.bfloat16) for _ in range(3)]
+    full = host_bits16(tbik.attention(q, k, v, tc=tc))
+    for L in (1024, 384, 128):
+        part = host_bits16(tbik.attention(q[:, :L].contiguous(), k[:, :L].contiguous(), v[:, :L].contiguous(), tc=tc))
+        assert np.array_equal(part, full[:, :L]), L
+    assert tbik.get_error() == tbik.TBIK_OK
