@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
     const int tid = threadIdx.x;
     int t = blockIdx.x;
     if (t >= tokens) return;
+    const float inv_h = __frcp_rn((float)H);  // exact: H is a power of two
     const int S = NT / T;            // threads per shard (a power of two)
     const int L = S < 32 ? S : 32;   // lanes per shuffle group
     const int G = NT / L;            // group values combined through shared memory
@@ -78,7 +79,10 @@ __global__ void __launch_bounds__(NT) rmsnorm_residual_kernel(const uint16_t* __
         float pv = (tid & 31) < G ? part[it & 1][tid & 31] : 0.0f;
         for (int w = 1; w < G; w <<= 1) pv = __fadd_rn(pv, __shfl_xor_sync(0xffffffffu, pv, w));
         const float ss = __shfl_sync(0xffffffffu, pv, 0);
-        const float ms = __fdiv_rn(ss, (float)H);
+        // H is a power of two (H/8 leaves, a power of two), so ss * (1/H)
+        // with 1/H exact is the correctly rounded ss / H: the same bits as the
+        // division, without its latency in the per-token chain
+        const float ms = __fmul_rn(ss, inv_h);
         const float inv = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
 #pragma unroll
         for (int l = 0; l < LPT; ++l) {
