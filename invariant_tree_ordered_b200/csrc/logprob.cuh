@@ -124,13 +124,30 @@ __global__ void __launch_bounds__(ROW_BLOCK * 32)
             MS stk[24];
             int sp = 0;
             const uint16_t* tb = tab[n == n_hi ? 0 : 1];
-            for (int j = 0; j < n; ++j) {
-                MS cur = leaf_ms(stats, M, nvt, row, lo + j);
-                const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
-                const int npop = code_pops(code);
-                for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
-                if (!((code >> 10) & 1)) stk[sp++] = cur;
-                else v = cur;
+            // The leaves' summaries are loaded four leaves ahead of their use
+            // (a ring of four, unrolled so it stays in registers); the combines
+            // run in the same order as without the look-ahead.
+            MS ring[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                ring[k].m = -INFINITY;
+                ring[k].s = 0.0f;
+                if (k < n) ring[k] = leaf_ms(stats, M, nvt, row, lo + k);
+            }
+            for (int j0 = 0; j0 < n; j0 += 4) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int j = j0 + k;
+                    if (j < n) {
+                        MS cur = ring[k];
+                        if (j + 4 < n) ring[k] = leaf_ms(stats, M, nvt, row, lo + j + 4);
+                        const uint32_t code = use_tab ? tb[j] : encode_leaf_ops(leaf_ops(n, j));
+                        const int npop = code_pops(code);
+                        for (int i = 0; i < npop; ++i) cur = ms_combine(stk[--sp], cur);
+                        if (!((code >> 10) & 1)) stk[sp++] = cur;
+                        else v = cur;
+                    }
+                }
             }
         }
         part[warp][lane] = make_float2(v.m, v.s);
