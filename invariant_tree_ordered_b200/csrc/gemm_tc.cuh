@@ -135,9 +135,35 @@ struct TcParams {
     int stages;
     uint32_t stage_bytes, a_slice;
     int tab_n[2];                    // the (at most two) subtree sizes of the frontier nodes
+    // Pacing (null: none): [0] gives up on pacing for the rest of the launch,
+    // [e] counts the pairs that reached their unit TC_PACE_UNITS * e.  Zeroed
+    // by the host before the launch.
+    unsigned int* pace;
     short lo[TC_MAX_F];
     short nl[TC_MAX_F];
 };
+
+// Pairs keep in step: every TC_PACE_UNITS work units each pair's producer
+// waits, briefly and bounded, until every pair has reached the same unit.
+// The pairs of a vocabulary column then fetch its W_lm tile while the others
+// still hold it in L2 (left alone they drift apart over a launch and part of
+// W_lm is read from DRAM again).  Only timing depends on it, never results.
+// A pair that waits longer than TC_PACE_WAIT cycles (CTAs not all resident,
+// or one pair far behind) switches pacing off for the whole launch.
+constexpr int TC_PACE_UNITS = 16;
+constexpr long long TC_PACE_WAIT = 4000000;
+__device__ __forceinline__ void tc_pace(unsigned int* pace, int epoch, unsigned int npairs) {
+    if (atomicOr(&pace[0], 0u) != 0u) return;
+    atomicAdd(&pace[epoch], 1u);
+    const long long t0 = clock64();
+    while (atomicOr(&pace[epoch], 0u) < npairs) {
+        if (clock64() - t0 > TC_PACE_WAIT || atomicOr(&pace[0], 0u) != 0u) {
+            atomicExch(&pace[0], 1u);
+            return;
+        }
+        __nanosleep(256);
+    }
+}
 
 __device__ __forceinline__ void tc_decode(const TcParams& p, int u, int& tm, int& tn, int& f) {
     int tiles = p.tiles_m * p.tiles_n;
@@ -367,7 +393,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TcCfg<BN>::THREADS, 
             const int stages = p.stages;
             uint32_t q = 0, ph = 0;
             int s = 0;
-            for (int u = pair; u < p.total_units; u += npairs) {
+            // units every pair has (pacing points must be reached by all of them)
+            const int common_units = p.total_units / npairs;
+            int kunit = 0;
+            for (int u = pair; u < p.total_units; u += npairs, ++kunit) {
+                if (p.pace != nullptr && rank == 0 && kunit > 0 && kunit % TC_PACE_UNITS == 0 && kunit < common_units)
+                    tc_pace(p.pace, kunit / TC_PACE_UNITS, (unsigned)npairs);
                 int tm, tn, f;
                 tc_decode(p, u, tm, tn, f);
                 const int k0 = p.lo[f] * p.leaf;

@@ -484,7 +484,8 @@ struct LogprobPlan {
     bool part = false;  // a vocabulary shard's summary (tbik_logprob_partial): T = 1, Lv given
     int Vpad = 0, Lv = 0, nvl = 0, nvt = 0, Lk = 0, tiles_m = 0, units = 0, grid = 0, gs = 0;
     size_t off_stats = 0, off_zt = 0, off_shard = 0, off_scratch = 0, off_z = 0, off_zgemm = 0, off_zflag = 0,
-           total = 0;
+           off_pace = 0, total = 0;
+    int pace_words = 0;  // tensor-core GEMM's pacing counters (0: no pacing)
     GemmPlan zplan;  // exact mode: the logits GEMM
 };
 
@@ -544,6 +545,12 @@ tbik_status plan_logprob(int M, int V, int H, int T, int leaf, unsigned mode, in
         p.off_scratch = off;
         off = align256(off + (size_t)p.grid * p.gs * tc_slot_bytes(TC_BN_WIDE));
     }
+    if (tc) {  // pacing counters: the flag, then one per TC_PACE_UNITS units of every pair
+        const int pairs = p.grid / 2;
+        p.pace_words = 1 + (p.units / (pairs > 0 ? pairs : 1)) / TC_PACE_UNITS + 1;
+        p.off_pace = off;
+        off = align256(off + (size_t)p.pace_words * sizeof(unsigned int));
+    }
     if (p.part) {  // which rows' targets fall in this shard
         p.off_zflag = off;
         off = align256(off + (size_t)M * sizeof(int));
@@ -588,6 +595,9 @@ tbik_status run_logprob(const LogprobPlan& p, const uint16_t* hidden, const uint
         prm.F = 1;
         prm.tiles_m = p.tiles_m, prm.tiles_n = p.nvt;
         prm.group_m = p.tiles_m;  // all row tiles of a vocab tile run together: W_lm is read once
+        prm.pace = reinterpret_cast<unsigned int*>(w8 + p.off_pace);
+        if (cudaMemsetAsync(prm.pace, 0, (size_t)p.pace_words * sizeof(unsigned int), s) != cudaSuccess)
+            return TBIK_ERR_CUDA;
         prm.total_units = p.units;
         prm.direct = 1;
         prm.scratch = p.gs ? reinterpret_cast<float*>(w8 + p.off_scratch) : nullptr;
