@@ -25,15 +25,16 @@
 // rows of its tile or how heads are split across devices.
 //
 // One CTA per SM, persistent over 128-row query tiles of one (batch, head),
-// the longest tiles first; 320 threads:
+// the longest tiles first, dealt out in alternating directions; 320 threads:
 //   warp 0     TMA producer: the Q tile (two 64-dim slices, K-major, 128-byte
 //              swizzle), per leaf K (same layout, two 64-key chunks) and V
 //              (MN-major: per chunk two 64-dim atoms of 64 keys); K of the
 //              next leaf is requested as soon as the scores of the current
 //              one are done, before V of the current one
 //   warp 1     TMEM allocator + MMA issuer: S = Q K^T of the leaf's two chunks
-//              (M=128, N=64 each) into S[0], S[1], then O_{L-1} = P V of the
-//              previous leaf (M=128, N=128, K=128) into O[(L-1)%2]
+//              (M=128, N=64 each) into S[0], S[1] (as soon as the softmax has
+//              read the previous leaf's S into registers), then O_{L-1} = P V
+//              of the previous leaf (M=128, N=128, K=128) into O[(L-1)%2]
 //   warps 2-9  epilogue: warp w owns rows 32*(w%4).. and half h = (w-2)/4:
 //              the softmax of chunk h of each leaf (its maximum taken over
 //              both chunks) and head dims [64h, 64h+64) of the tree.  Loop:
@@ -134,6 +135,14 @@ __device__ __forceinline__ void atc_factors(float am, float bm, float& M, float&
     eb = (finite && bm == M) ? 1.0f : ex2_hw(__fmul_rn(__fsub_rn(bm, M), log2e));
 }
 
+// The k-th query tile of this CTA: the tiles are dealt out in rounds of
+// gridDim.x, in alternating directions, so that every CTA's total of leaves
+// stays close to the mean (the tiles are ordered longest first).
+__device__ __forceinline__ int atc_sched(int k) {
+    const int G = (int)gridDim.x, b = (int)blockIdx.x;
+    return k * G + ((k & 1) ? G - 1 - b : b);
+}
+
 // Query tile t (longest first): position block qt and (batch, head) bh.
 __device__ __forceinline__ void atc_tile(const AttTcParams& p, int t, int& qt, int& bh) {
     const int nbh = p.batch * p.heads;
@@ -156,11 +165,12 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
     uint64_t* v_full = bars + 4;       // V of a leaf landed
     uint64_t* v_empty = bars + 5;      // the leaf's P V MMAs retired
     uint64_t* s_full = bars + 6;       // S of a leaf (both chunks) in TMEM
-    uint64_t* p_full = bars + 7;       // P of a leaf written (S read) by the 8 epilogue warps
+    uint64_t* p_full = bars + 7;       // P of a leaf written by the 8 epilogue warps
     uint64_t* o_full = bars + 8;       // [2] O of a leaf in TMEM
     uint64_t* o_empty = bars + 10;     // [2] O buffer released by the 8 epilogue warps
     uint64_t* done = bars + 12;        // every MMA issued by this CTA retired
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+    uint64_t* s_empty = bars + 13;     // S of a leaf read by the 8 epilogue warps
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,6 +184,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         mbar_init(v_empty, 1);
         mbar_init(s_full, 1);
         mbar_init(p_full, ATC_EPI_WARPS);
+        mbar_init(s_empty, ATC_EPI_WARPS);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&o_full[b], 1);
             mbar_init(&o_empty[b], ATC_EPI_WARPS);
@@ -198,7 +209,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             uint32_t gk = 0, gv = 0, nt = 0;  // K leaves, V leaves and tiles loaded so far by this CTA
-            for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++nt) {
+            for (int t = atc_sched(0); t < p.tiles; t = atc_sched(++nt)) {
                 int qt, bh;
                 atc_tile(p, t, qt, bh);
                 const int b = bh / p.heads, h = bh - b * p.heads;
@@ -242,7 +253,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             const uint32_t idesc_o = idesc_bf16_f32(ATC_BM, ATC_HD, 0, 1);
             const uint32_t q_u = smem_u32(smem + ATC_OFF_Q);
             uint32_t g0 = 0, nt = 0;
-            for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++nt) {
+            for (int t = atc_sched(0); t < p.tiles; t = atc_sched(++nt)) {
                 int qt, bh;
                 atc_tile(p, t, qt, bh);
                 const int nl = qt + 1;
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                         const uint32_t g = g0 + l;
                         if (!mbar_wait(k_full, g & 1, abort_flag, lim)) goto mma_out;
                         // S was read by the softmax of leaf g - 1
-                        if (g >= 1 && !mbar_wait(p_full, (g - 1) & 1, abort_flag, lim)) goto mma_out;
+                        if (g >= 1 && !mbar_wait(s_empty, (g - 1) & 1, abort_flag, lim)) goto mma_out;
                         tc_fence_after();
                         const uint64_t adesc = smem_desc_sw128(q_u, 16, 1024);
 #pragma unroll
@@ -273,8 +284,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     if (l >= 1) {
                         const uint32_t g = g0 + l - 1, b = g & 1, ph = (g >> 1) & 1;
                         if (!mbar_wait(v_full, g & 1, abort_flag, lim)) goto mma_out;
-                        // P of leaf g: already awaited above unless no S was issued in this step
-                        if (l == nl && !mbar_wait(p_full, g & 1, abort_flag, lim)) goto mma_out;
+                        if (!mbar_wait(p_full, g & 1, abort_flag, lim)) goto mma_out;  // P of leaf g written
                         if (g >= 2 && !mbar_wait(&o_empty[b], ph ^ 1, abort_flag, lim)) goto mma_out;
                         tc_fence_after();
 #pragma unroll
@@ -320,7 +330,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
         // that pops a slot and pushes its result into it lets one warp write the
         // new value before the other has read the old one)
         float stk_m[ATC_MAX_GS], stk_s[ATC_MAX_GS];
-        for (int t = blockIdx.x; t < p.tiles; t += gridDim.x) {
+        for (int k = 0, t = atc_sched(0); t < p.tiles; t = atc_sched(++k)) {
             int qt, bh;
             atc_tile(p, t, qt, bh);
             const int bb = bh / p.heads, hh = bh - bb * p.heads;
@@ -371,6 +381,10 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     uint32_t so[64];
                     tmem_ld64_nowait(tl + ATC_S_COL + 64 * half, so);
                     tmem_wait_ld64(so);
+                    // S is in registers: the scores of the next leaf may overwrite it
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(s_empty);
                     float vo[64];
                     const f2x sc2 = pk2(p.scale, p.scale);
 #pragma unroll
