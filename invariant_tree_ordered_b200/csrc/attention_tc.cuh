@@ -341,6 +341,7 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
             float m1 = 0.f, s1 = 0.f, m2 = 0.f, s2 = 0.f, m34 = 0.f, s34 = 0.f;
             uint32_t single_b = 0;
             int gsp = 0;
+            uint32_t lane_code = 0;  // operation code of leaf 32*(l1/32) + lane of this tile's tree
             for (int l = 0; l <= nl; ++l) {
                 if (l < nl) {
                     // ---------------- softmax of leaf l (this warp: chunk `half`)
@@ -471,7 +472,13 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     ab = ab || __shfl_sync(0xffffffffu, okw, 0) == 0;
                     if (ab) continue;  // left at the pair's next barrier (or at the end)
                     tc_fence_after();
-                    const uint32_t code = encode_leaf_ops(leaf_ops(nl, l1));
+                    // the lanes walk the tree for 32 leaves at once; each leaf's code
+                    // is then one shuffle away
+                    if ((l1 & 31) == 0) {
+                        const int lj = l1 + lane;
+                        lane_code = lj < nl ? encode_leaf_ops(leaf_ops(nl, lj)) : 0u;
+                    }
+                    const uint32_t code = __shfl_sync(0xffffffffu, lane_code, l1 & 31);
                     const bool p1 = code & 1, p2 = (code >> 1) & 1, pm = (code >> 2) & 1;
                     const int nb = (code >> 3) & 31;
                     const int cls = (code >> 8) & 3;
