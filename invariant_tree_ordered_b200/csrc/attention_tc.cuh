@@ -467,9 +467,14 @@ __global__ void __launch_bounds__(ATC_THREADS, 1)
                     // ---------------- tree step of leaf l - 1
                     const int l1 = l - 1;
                     const uint32_t g = g0 + l1, b = g & 1, ph = (g >> 1) & 1;
-                    uint32_t okw = 1;
-                    if (lane == 0 && !ab) okw = mbar_wait(&o_full[b], ph, abort_flag, lim) ? 1u : 0u;
-                    ab = ab || __shfl_sync(0xffffffffu, okw, 0) == 0;
+                    // O of leaf l - 1 landed: the softmax of leaf l has waited for it
+                    // before writing P (or this warp left at the pair's barrier), so
+                    // only the tile's last leaf waits here
+                    if (l == nl) {
+                        uint32_t okw = 1;
+                        if (lane == 0 && !ab) okw = mbar_wait(&o_full[b], ph, abort_flag, lim) ? 1u : 0u;
+                        ab = ab || __shfl_sync(0xffffffffu, okw, 0) == 0;
+                    }
                     if (ab) continue;  // left at the pair's next barrier (or at the end)
                     tc_fence_after();
                     // the lanes walk the tree for 32 leaves at once; each leaf's code
