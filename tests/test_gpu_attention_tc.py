@@ -55,6 +55,28 @@ def test_tc_attention_vs_binary64(B, S, NH):
     assert np.all(within_bound(got, exact, v))
 
 
+def test_tc_attention_more_than_32_leaves():
+    """4224 positions: the last query tile has 33 leaves, so the epilogue's lanes
+    walk the leaf tree for a second block of 32 leaves; checked against binary64.
+    The same positions inside an 8192-position sequence (64 leaves, deeper L2
+    stack) give the same bits: a row's result depends only on its own keys."""
+    B, S, NH = 1, 4224, 2
+    q, k, v = qkv(4224, (B, S, NH, 128))
+    got_bits = host_bits16(tbik.attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), tc=True))
+    assert tbik.get_error() == tbik.TBIK_OK
+    got = f32(got_bits)
+    ref = oracle.attention_f64(q, k, v)
+    assert np.all(np.isfinite(got))
+    assert np.all(within_bound(got, ref, v))
+    assert float(np.mean(np.abs(got - ref))) <= 1e-3
+    L = 8192
+    ext = qkv(8192, (B, L - S, NH, 128))
+    q2, k2, v2 = (np.ascontiguousarray(np.concatenate([x, e], axis=1)) for x, e in zip((q, k, v), ext))
+    long_bits = host_bits16(tbik.attention(dev_bf16(q2), dev_bf16(k2), dev_bf16(v2), tc=True))
+    assert tbik.get_error() == tbik.TBIK_OK
+    assert np.array_equal(long_bits[:, :S], got_bits)
+
+
 def test_tc_attention_large_scores():
     # std-4 queries and keys: a wide score range, so the chunk maxima and the
     # exp(m - M) factors of the tree combine matter
