@@ -298,11 +298,16 @@ __device__ __forceinline__ void logprob_leaf_stats(const TcParams& p, float (&v)
                 if (k + 32 >= ncol) v[1][k] = -INFINITY;
             }
         }
-        float m = v[0][0];
+        // the maximum in four independent chains of three-input maxima (max is
+        // exact, so the grouping does not change it)
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int k = 1; k < 32; ++k) m = fmaxf(m, v[0][k]);
+        for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) m = fmaxf(m, v[1][k]);
+            for (int k = 0; k < 32; k += 8)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], v[cc][k + 2 * q], v[cc][k + 2 * q + 1]);
+        const float m = fmax3(fmaxf(mq[0], mq[1]), mq[2], mq[3]);
         const float log2e = 0x1.715476p+0f;
         const float ml = -__fmul_rn(m, log2e);
         float s0 = 0.0f, s1 = 0.0f;
