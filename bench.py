@@ -206,15 +206,18 @@ _ORACLE_INPUTS = {}
 def oracle_step_sample(tokens: int):
     """Time the CPU oracle on `tokens` tokens of the step (every kernel of the path)."""
     import oracle
+    if "weights" not in _ORACLE_INPUTS:  # the same weights for every sample size
+        _ORACLE_INPUTS["weights"] = dict(b=synth.down_proj_weight(F, H, "kn"),
+                                         w=synth.normal_bf16(31, (V, H), std=0.02),
+                                         table=oracle.rope_table(MAX_POS, HEAD_DIM, 1e6))
     if tokens not in _ORACLE_INPUTS:
         std = 0.02 * np.sqrt(H)
         _ORACLE_INPUTS[tokens] = dict(
             d=synth.reduction_inputs(tokens), g=synth.normal_bf16(11, (tokens, F), std=std),
-            u=synth.normal_bf16(12, (tokens, F), std=std), b=synth.down_proj_weight(F, H, "kn"),
-            w=synth.normal_bf16(31, (V, H), std=0.02), targets=synth.uniform_int32(32, tokens, 0, V),
-            table=oracle.rope_table(MAX_POS, HEAD_DIM, 1e6))
-    c_ = _ORACLE_INPUTS[tokens]
-    d, g, u, b, w, targets, table = (c_["d"], c_["g"], c_["u"], c_["b"], c_["w"], c_["targets"], c_["table"])
+            u=synth.normal_bf16(12, (tokens, F), std=std), targets=synth.uniform_int32(32, tokens, 0, V))
+    c_, wt = _ORACLE_INPUTS[tokens], _ORACLE_INPUTS["weights"]
+    d, g, u, targets = c_["d"], c_["g"], c_["u"], c_["targets"]
+    b, w, table = wt["b"], wt["w"], wt["table"]
     t0 = time.perf_counter()
     oracle.rmsnorm_residual(d["x"], d["res"], d["gamma"], eps=1e-6)
     oracle.rope(d["q"], d["pos"], table)
@@ -549,6 +552,19 @@ def run_tbik(args):
                                 "sample": f"{tok} tokens of the step (RMSNorm, RoPE, SwiGLU, down_proj rows, "
                                           f"lm_head logprob rows), single-threaded C oracle, {dt:.1f} s",
                                 **host_cpu()}
+        try:  # the same oracle built with OpenMP: its GEMM outputs and logprob rows on every host core
+            import oracle
+            tok_all = 64
+            with oracle.library(oracle.build_all_cores()):
+                dt_all = oracle_step_sample(tok_all)
+            threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+            line["cpu_baseline_all_cores"] = {
+                "value": tok_all / dt_all, "unit": "tokens/s", "cores": threads,
+                "kind": "oracle (same source built with -fopenmp; same bits)",
+                "sample": f"{tok_all} tokens of the step, the down_proj outputs and logprob rows spread over "
+                          f"{threads} threads, {dt_all:.1f} s"}
+        except Exception as e:  # noqa: BLE001  (an extra figure: its failure must not cost the line)
+            line["cpu_baseline_all_cores"] = {"error": f"{type(e).__name__}: {e}"[:200]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

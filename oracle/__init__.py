@@ -2,7 +2,9 @@
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package.  It wraps ``oracle.c`` (plain single-threaded C,
-compiled on first use into ``liboracle.so`` beside it) with numpy marshalling;
+compiled on first use into ``liboracle.so`` beside it; ``build_all_cores``
+makes an OpenMP build of the same file for timing on all host cores) with
+numpy marshalling;
 all arithmetic happens in the C file.  Nothing here is shared with the CUDA
 library.
 """
@@ -50,6 +52,22 @@ def build(force: bool = False) -> str:
     so = _so_path()
     if force or not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(_SRC):
         flags = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+        if _cpu_has_fma():
+            flags.append("-mfma")
+        tmp = so + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *flags, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, so)
+    return so
+
+
+def build_all_cores(force: bool = False) -> str:
+    """Compile the same oracle.c with -fopenmp into ``liboracle_omp.so``: the
+    pragmas on the independent GEMM outputs and logprob rows spread them over
+    the host's cores (each output is the same serial computation, so the bits
+    equal the default build's).  Used only to time the oracle on all cores."""
+    so = os.path.join(_HERE, "liboracle_omp.so")
+    if force or not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(_SRC):
+        flags = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-fopenmp"]
         if _cpu_has_fma():
             flags.append("-mfma")
         tmp = so + f".tmp{os.getpid()}"

@@ -7,7 +7,12 @@
  * only the tests, smoke() and the benchmark's CPU-baseline leg may load it.
  * Build flags: -O2 -ffp-contract=off -fno-fast-math, x86-64 SSE arithmetic,
  * so every float operation below is one IEEE binary32 round-to-nearest-even
- * operation and fmaf() is the correctly rounded fused multiply-add.
+ * operation and fmaf() is the correctly rounded fused multiply-add.  The
+ * default build is single-threaded.  The independent outputs of the GEMM and
+ * the rows of the logprob carry OpenMP pragmas, which only a second build
+ * with -fopenmp (used to time the oracle on all host cores) acts on: each
+ * output is still the same serial computation, so both builds give the same
+ * bits.
  *
  * Sources (web pages on the subject; cited by title and section):
  *  [TBIK] "Deterministic Inference across Tensor Parallel Sizes That Eliminates
@@ -207,11 +212,18 @@ int oracle_gemm_tree(const uint16_t* A, const uint16_t* B, int b_nk, int M, int 
     int L = K / leaf;
     if (L % T) return -1;
     int Ls = L / T;
-    float* P = (float*)malloc(sizeof(float) * (size_t)L);
-    float* Q = (float*)malloc(sizeof(float) * (size_t)T);
     const uint16_t* Bt = b_nk ? B : transpose_kn(B, K, N);
-    for (int i = 0; i < M; ++i) {
-        for (int n = 0; n < N; ++n) {
+    /* Every output (i, n) is computed on its own, so a build with OpenMP may
+       hand them to several threads, each with its own leaf and shard scratch;
+       the computation of each output is the same serial one (the default build
+       is single-threaded and ignores the pragmas). */
+#pragma omp parallel
+    {
+        float* P = (float*)malloc(sizeof(float) * (size_t)L);
+        float* Q = (float*)malloc(sizeof(float) * (size_t)T);
+#pragma omp for schedule(static)
+        for (long long o = 0; o < (long long)M * N; ++o) {
+            const int i = (int)(o / N), n = (int)(o % N);
             const uint16_t* bcol = Bt + (size_t)n * K;
             for (int j = 0; j < L; ++j) {
                 float acc = 0.0f;
@@ -225,10 +237,10 @@ int oracle_gemm_tree(const uint16_t* A, const uint16_t* B, int b_nk, int M, int 
             }
             C[(size_t)i * N + n] = tree_f32(Q, 0, T);
         }
+        free(P);
+        free(Q);
     }
     if (!b_nk) free((void*)Bt);
-    free(P);
-    free(Q);
     return 0;
 }
 
@@ -469,11 +481,14 @@ int oracle_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* tar
     int Lv = vpad / vleaf;
     if (Lv % T || (noninv && H % T)) return -1;
     int Ls = Lv / T;
-    float* z = (float*)malloc(sizeof(float) * (size_t)V);
-    float* P = (float*)malloc(sizeof(float) * (size_t)Lk);
-    ms_t* leaves = (ms_t*)malloc(sizeof(ms_t) * (size_t)Lv);
-    ms_t* shards = (ms_t*)malloc(sizeof(ms_t) * (size_t)T);
+    /* Rows are independent: a build with OpenMP may spread them over threads
+       (each row with its own scratch, computed exactly as below). */
+#pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < M; ++i) {
+        float* z = (float*)malloc(sizeof(float) * (size_t)V);
+        float* P = (float*)malloc(sizeof(float) * (size_t)Lk);
+        ms_t* leaves = (ms_t*)malloc(sizeof(ms_t) * (size_t)Lv);
+        ms_t* shards = (ms_t*)malloc(sizeof(ms_t) * (size_t)T);
         const uint16_t* h = hidden + (size_t)i * H;
         for (int v = 0; v < V; ++v) {
             const uint16_t* w = W + (size_t)v * H;
@@ -522,11 +537,11 @@ int oracle_logprob(const uint16_t* hidden, const uint16_t* W, const int32_t* tar
             float d = z[tg] - fin.m;
             out[i] = d - log_spec(fin.s);
         }
+        free(z);
+        free(P);
+        free(leaves);
+        free(shards);
     }
-    free(z);
-    free(P);
-    free(leaves);
-    free(shards);
     return 0;
 }
 
